@@ -1,0 +1,407 @@
+"""Benchmark: MoE-block decode tokens/s and achieved HBM bandwidth at batch 1, 18% budget.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--k K] [--batch B] [--rank R]
+
+Workload (default): the Qwen3-30B-A3B-shaped block, d=2048, I=768, E=128, top-8,
+k=138 (18%), r=32, batch 1, BF16 weights N(0, 0.02) with 5% of channels x4,
+x ~ N(0, 1); 1000 decode steps with fresh seeded x per step (synthetic data).
+
+One step = one call of the whole block (router, sketch scoring, top-k,
+gathered SwiGLU + down, low-rank term, combine) on one batch.  The K timed
+steps run as replays of a CUDA graph that holds the 1000-step decode
+sequence; consecutive steps read different weight replicas (R copies of the
+packed layer, R * 1.3 GB >> 126 MB L2), so every step reads its bytes from HBM.
+
+Printed JSON (rank 0, one line): value = tokens/s over all ranks, e2e = the
+same through the public Python/C-ABI call with pinned host x/out copies per
+step, roofline = the step's algorithmic bytes / device time vs the measured
+HBM copy bandwidth, cpu_baseline = the FP64 CPU oracle on a bounded sample.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            m = json.load(f)
+        return float(m["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "token_top_expert_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    r = rec.get(kernel, {}).get(workload)
+    if not r or r.get("source_hash") != kernel_source_hash():
+        return None
+    return r.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def algorithmic_bytes(w, k, rank, union_sizes, dense):
+    """Bytes the method must read for one step: per used expert the sketch
+    (I*d/4), row scales (4I), the union of selected channel records (6d each)
+    and A_e, B_e (4dr).  The dense path reads only channel records."""
+    total = 0
+    for u in union_sizes:
+        if u == 0:
+            continue
+        total += 6 * w.d * int(u)
+        if not dense:
+            total += w.inter * w.d // 4 + 4 * w.inter + 4 * w.d * rank
+    return total
+
+
+def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None):
+    """Time the FP64 CPU oracle, as it stands, on the first tokens of the step
+    sequence (a warm pass first fills its weight caches; the second pass is timed).
+    Returns (tokens/s, tokens, seconds, threads)."""
+    import oracle
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        threads = max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:  # noqa: BLE001
+        threads = 1
+    lay = oracle.SynthLayer(w, max_cache=w.experts)
+    toks = []
+    t0 = time.time()
+    n = 0
+    while n < len(xs) and (max_tokens is None or n < max_tokens):
+        oracle.moe_block(xs[n], lay, w.top_e, k, rank=rank)   # warm: generate + sketch
+        toks.append(n)
+        n += 1
+        if time.time() - t0 > budget_s:
+            break
+    t1 = time.time()
+    for i in toks:
+        oracle.moe_block(xs[i], lay, w.top_e, k, rank=rank)
+    dt = time.time() - t1
+    ntok = len(toks) * xs[0].shape[0]
+    return ntok / dt, ntok, dt, threads
+
+
+def run_reference(args, w, world, rank):
+    """The reference arm: the CPU oracle timed on the same workload (bounded sample)."""
+    if rank != 0:
+        return
+    xs = [synth.activations(w, s, batch=args.batch) for s in range(max(min(args.steps, 1000), 1))]
+    budget = 60.0
+    v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs, budget_s=budget / 4,
+                                         max_tokens=args.steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * args.batch / v,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, args),
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "%d tokens (first steps of the decode sequence), %.1f s" % (ntok, dt)},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+METRIC = "MoE-block decode tokens/s (achieved HBM GB/s vs peak) at B=1, 18% budget"
+
+
+def config_of(w, args):
+    return {"workload": w.name, "d": w.d, "I": w.inter, "E": w.experts, "top_e": w.top_e,
+            "k": args.k, "budget": round(args.k / w.inter, 4), "rank": args.rank,
+            "global_batch": args.batch * args.gpus, "batch_per_gpu": args.batch,
+            "decode_steps": w.steps, "replicas": args.replicas,
+            "l2": "inputs larger than L2: %d weight replicas rotated per step" % args.replicas,
+            "parallelism": "replicas" if args.gpus > 1 else "single"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synth.QWEN30B_BLOCK.name, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--batch", type=int, default=None)
+    ap.add_argument("--rank", type=int, default=None)
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    args = ap.parse_args()
+    w = synth.WORKLOADS[args.workload]
+    args.k = w.k if args.k is None else args.k
+    args.batch = w.batch if args.batch is None else args.batch
+    args.rank = w.rank if args.rank is None else args.rank
+    if args.k == w.inter and args.rank == w.rank and "--rank" not in sys.argv:
+        args.rank = 0  # the dense reference path has no compensation term
+    world, rank, local = dist_setup()
+    args.gpus = world if world > 1 else args.gpus
+
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+        return
+
+    import torch
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    import token_top_expert_b200 as msb
+    from token_top_expert_b200 import build as _b
+    _b.build()
+    msb.load_library()
+    dev = torch.device("cuda", local)
+
+    # ---- weights: generate, pack (host C++ packer), upload, replicate
+    lw = synth.layer_weights(w)
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
+    pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
+    base = msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev)
+    del lw, pk
+    layers = [base] + [base.clone() for _ in range(args.replicas - 1)]
+    B = args.batch
+    nseq = min(w.steps, 1000)
+    xs_host = [synth.activations(w, s, batch=B) for s in range(nseq)]
+    xs = torch.from_numpy(np.stack(xs_host).view(np.int16)).to(dev).view(torch.bfloat16)
+    outs = torch.empty_like(xs)
+    ws = msb.Workspace(dims, B, dev)
+    stream = torch.cuda.Stream(dev)
+    general = args.general
+
+    def step(i, s):
+        msb.moe_sparse_block(xs[i % nseq], layers[i % args.replicas], args.k, out=outs[i % nseq],
+                             workspace=ws, general=general, stream=s)
+
+    # ---- union sizes of every step of the sequence (one traced pass) -> algorithmic bytes
+    dense = args.k == w.inter
+    tr = msb.Trace(dims, B, args.k)
+    bytes_per_step = []
+    with torch.cuda.stream(stream):
+        for i in range(nseq):
+            msb.moe_sparse_block(xs[i], layers[i % args.replicas], args.k, out=outs[i],
+                                 workspace=ws, trace=tr, general=general, stream=stream)
+            if i < 64 or not (B == 1 and not dense):
+                stream.synchronize()
+                bytes_per_step.append(algorithmic_bytes(w, args.k, args.rank,
+                                                        tr.union_count.cpu().tolist(), dense))
+    stream.synchronize()
+    ws.check(stream)
+    step_bytes = float(np.mean(bytes_per_step))
+    router_bytes = 2 * w.d * w.experts
+
+    # ---- warmup (untimed), then capture the decode sequence as one CUDA graph
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i, stream)
+    stream.synchronize()
+    G = min(nseq, args.steps)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i, stream)
+    tail = None
+    if args.steps % G:
+        tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(tail, stream=stream):
+            for i in range(args.steps % G):
+                step(i, stream)
+    graph.replay()
+    stream.synchronize()
+
+    # ---- timed region: exactly K steps
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]
+                    if os.environ.get("CUDA_VISIBLE_DEVICES") else local)
+    with ClockSampler(gpu_index) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps // G):
+                graph.replay()
+            if tail is not None:
+                tail.replay()
+            e1.record(stream)
+        stream.synchronize()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        dist.barrier()
+    ms_per_step = ms / args.steps
+    value = args.steps * B * world / (ms / 1e3)
+    ws.check(stream)
+
+    # ---- e2e: public call per step with pinned host x -> device -> host out
+    xh = torch.from_numpy(np.stack(xs_host).view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty((B, w.d), dtype=torch.bfloat16, device=dev)
+    od = torch.empty_like(xd)
+    ne = min(args.e2e_steps, args.steps)
+    with torch.cuda.stream(stream):
+        for i in range(min(50, ne)):
+            xd.copy_(xh[i % nseq], non_blocking=True)
+            msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
+                                 general=general, stream=stream)
+            oh[i % nseq].copy_(od, non_blocking=True)
+        stream.synchronize()
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(ne):
+            xd.copy_(xh[i % nseq], non_blocking=True)
+            msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
+                                 general=general, stream=stream)
+            oh[i % nseq].copy_(od, non_blocking=True)
+        a1.record(stream)
+        stream.synchronize()
+    e2e_ms = a0.elapsed_time(a1)
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = ne * B * world / (e2e_ms / 1e3)
+
+    peak, peak_kind = peaks()
+    achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
+    kernel = "moe_block_fused" if (B == 1 and not general) else "moe_block_general"
+    traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else ""))
+    launches_per_step = 1 if kernel == "moe_block_fused" else (3 if dense else 5)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world if world > 1 else 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) BF16 weights, 5% rows x4; x ~ N(0,1))",
+        "config": config_of(w, args),
+        "us_per_block": ms_per_step * 1e3,
+        "bytes_per_step": step_bytes, "router_bytes_per_step": router_bytes,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": traffic,
+                     "kernel": kernel,
+                     "note": "achieved = algorithmic bytes per step / device time per step "
+                             "(CUDA events over the timed graph replays, launch gaps included)"},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * w.d * 2,
+                "d2h_bytes_per_step": B * w.d * 2, "steps": ne},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs_host, budget_s=6.0)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": "%d tokens of the same decode sequence (FP64 numpy "
+                                          "oracle, timed second pass), %.1f s" % (ntok, dt)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph, tail
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -202,12 +202,16 @@ class ArrayLayer:
 
 
 class SynthLayer(ArrayLayer):
-    """Weights of one layer regenerated expert by expert from the seeded generator."""
+    """Weights of one layer regenerated expert by expert from the seeded generator.
+    At most ``max_cache`` experts' float64 weights are kept (least recently used
+    are dropped and regenerated on demand); sketches are kept for every expert."""
 
-    def __init__(self, workload, layer=0):
+    def __init__(self, workload, layer=0, max_cache=12):
         self.w, self.layer = workload, layer
         self._cache = {}
         self._sk = {}
+        self._order = []
+        self._max = max_cache
 
     def router(self):
         if "router" not in self._cache:
@@ -215,6 +219,11 @@ class SynthLayer(ArrayLayer):
         return self._cache["router"]
 
     def expert(self, e):
+        if e in self._order:
+            self._order.remove(e)
+        self._order.append(e)
+        while len(self._order) > self._max:
+            self._cache.pop(self._order.pop(0), None)
         if e not in self._cache:
             w, l = self.w, self.layer
             if w.rank:

@@ -1,0 +1,232 @@
+"""Python binding of libmsb: argument marshalling over the C ABI, nothing else.
+
+PyTorch provides device memory and streams; every step of the block runs in
+libmsb's CUDA kernels.  Host-side packing calls libmsb's C++ packer.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+
+import numpy as np
+
+from . import _lib
+from ._lib import MsbDims, MsbError, MsbTrace
+
+
+@dataclasses.dataclass(frozen=True)
+class Dims:
+    d: int
+    inter: int
+    experts: int
+    top_e: int
+    rank: int
+    renorm: int = 1
+
+    @property
+    def ipad(self) -> int:
+        return (self.inter + 15) // 16 * 16
+
+    def c(self) -> MsbDims:
+        return MsbDims(self.d, self.inter, self.experts, self.top_e, self.rank, self.renorm)
+
+
+def _ptr(a) -> int:
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()
+
+
+def _check(rc: int, what: str):
+    if rc != _lib.MSB_OK:
+        raise MsbError(rc, what)
+
+
+# ------------------------------------------------------------------ packing (host)
+
+def sketch_words(dims: Dims) -> int:
+    return _lib.load().msb_sketch_words(ctypes.byref(dims.c()))
+
+
+def pack(gate: np.ndarray, up: np.ndarray, down: np.ndarray, router: np.ndarray, dims: Dims,
+         threads: int = 0) -> dict:
+    """Pack model-layout BF16 weights (uint16 bit arrays) with libmsb's host packer.
+
+    gate, up: [E][I][d]; down: [E][d][I]; router: [d][E].
+    Returns numpy arrays: records [E][I][3d] u16, sketch u32, alpha [E][Ipad] f32,
+    router_t [E][d] u16.
+    """
+    lib = _lib.load()
+    E, I, d = dims.experts, dims.inter, dims.d
+    for a, shape in ((gate, (E, I, d)), (up, (E, I, d)), (down, (E, d, I)), (router, (d, E))):
+        if a.dtype != np.uint16 or a.shape != shape or not a.flags.c_contiguous:
+            raise ValueError("expected contiguous uint16 array of shape %s, got %s %s"
+                             % (shape, a.dtype, a.shape))
+    cd = dims.c()
+    records = np.empty((E, I, 3 * d), np.uint16)
+    sketch = np.empty(lib.msb_sketch_words(ctypes.byref(cd)), np.uint32)
+    alpha = np.empty((E, dims.ipad), np.float32)
+    router_t = np.empty((E, d), np.uint16)
+    rc = lib.msb_pack(_ptr(gate), _ptr(up), _ptr(down), _ptr(router), ctypes.byref(cd),
+                      _ptr(records), _ptr(sketch), _ptr(alpha), _ptr(router_t), threads)
+    _check(rc, "msb_pack")
+    return {"records": records, "sketch": sketch, "alpha": alpha, "router_t": router_t}
+
+
+# ------------------------------------------------------------------ device objects
+
+class PackedLayer:
+    """One MoE layer's packed weights resident on a CUDA device."""
+
+    def __init__(self, dims: Dims, records, sketch, alpha, router_t, lr_a=None, lr_b=None):
+        self.dims = dims
+        self.records, self.sketch, self.alpha, self.router_t = records, sketch, alpha, router_t
+        self.lr_a, self.lr_b = lr_a, lr_b
+
+    @classmethod
+    def from_host(cls, dims: Dims, packed: dict, lr_a: np.ndarray | None, lr_b: np.ndarray | None,
+                  device="cuda"):
+        import torch
+
+        def t(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        return cls(dims, t(packed["records"].view(np.int16)), t(packed["sketch"].view(np.int32)),
+                   t(packed["alpha"]), t(packed["router_t"].view(np.int16)),
+                   None if lr_a is None or dims.rank == 0 else t(lr_a.view(np.int16)),
+                   None if lr_b is None or dims.rank == 0 else t(lr_b.view(np.int16)))
+
+    def clone(self) -> "PackedLayer":
+        """A copy at different addresses (same values)."""
+        c = lambda a: None if a is None else a.clone()
+        return PackedLayer(self.dims, c(self.records), c(self.sketch), c(self.alpha),
+                           c(self.router_t), c(self.lr_a), c(self.lr_b))
+
+    def nbytes(self) -> int:
+        return sum(a.numel() * a.element_size() for a in
+                   (self.records, self.sketch, self.alpha, self.router_t, self.lr_a, self.lr_b)
+                   if a is not None)
+
+
+def workspace_size(dims: Dims, max_batch: int) -> int:
+    return _lib.load().msb_workspace_size(ctypes.byref(dims.c()), max_batch)
+
+
+class Workspace:
+    """Zero-filled device scratch for calls of up to max_batch tokens."""
+
+    def __init__(self, dims: Dims, max_batch: int, device="cuda"):
+        import torch
+        n = workspace_size(dims, max_batch)
+        if n == 0:
+            raise ValueError("invalid dims or batch for a workspace")
+        self.nbytes = n
+        self.buf = torch.zeros(n + 256, dtype=torch.uint8, device=device)
+        base = self.buf.data_ptr()
+        self.ptr = (base + 255) // 256 * 256
+
+    def check(self, stream=None):
+        rc = _lib.load().msb_check(self.ptr, _stream(stream))
+        _check(rc, "kernel")
+
+
+class Trace:
+    """Device buffers receiving a call's routing and selection."""
+
+    def __init__(self, dims: Dims, batch: int, k: int, device="cuda", scores=False,
+                 threshold=False):
+        import torch
+        K = dims.top_e
+        cap = dims.inter if threshold else k
+        self.expert_ids = torch.zeros((batch, K), dtype=torch.int32, device=device)
+        self.expert_w = torch.zeros((batch, K), dtype=torch.float32, device=device)
+        self.sel = torch.zeros((batch, K, cap), dtype=torch.int16, device=device)
+        self.sel_count = torch.zeros((batch, K), dtype=torch.int32, device=device)
+        self.union_count = torch.zeros((dims.experts,), dtype=torch.int32, device=device)
+        self.scores = (torch.zeros((batch, K, dims.ipad), dtype=torch.float32, device=device)
+                       if scores else None)
+
+    def c(self) -> MsbTrace:
+        return MsbTrace(_ptr(self.expert_ids), _ptr(self.expert_w), _ptr(self.sel),
+                        _ptr(self.sel_count), _ptr(self.union_count), _ptr(self.scores))
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _act(x, dims: Dims):
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != dims.d or not x.is_contiguous():
+        raise ValueError("x must be a contiguous bf16 [batch][d] tensor")
+    return x
+
+
+# ------------------------------------------------------------------ the block
+
+def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspace | None = None,
+                     trace: Trace | None = None, general: bool = False, stream=None):
+    """One sparse-MoE block decode step: out[t] = sum_e w_te * (gathered SwiGLU over the
+    k top-scoring channels + A_e B_e x_t).  x: bf16 [B][d] on the GPU."""
+    import torch
+    dims = layer.dims
+    _act(x, dims)
+    B = x.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = Workspace(dims, B, x.device)
+    tr = trace.c() if trace is not None else None
+    rc = _lib.load().moe_sparse_block(
+        _ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
+        _ptr(layer.alpha), k, _ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out),
+        ctypes.byref(dims.c()), workspace.ptr, workspace.nbytes,
+        ctypes.byref(tr) if tr is not None else None,
+        _lib.MSB_FLAG_GENERAL if general else 0, _stream(stream))
+    _check(rc, "moe_sparse_block")
+    return out
+
+
+def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
+                               workspace: Workspace | None = None, trace: Trace | None = None,
+                               stream=None):
+    """The calibrated-threshold comparator: channels with score > tau."""
+    import torch
+    dims = layer.dims
+    _act(x, dims)
+    B = x.shape[0]
+    if out is None:
+        out = torch.empty_like(x)
+    if workspace is None:
+        workspace = Workspace(dims, B, x.device)
+    tr = trace.c() if trace is not None else None
+    rc = _lib.load().moe_sparse_block_threshold(
+        _ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
+        _ptr(layer.alpha), float(tau), _ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out),
+        ctypes.byref(dims.c()), workspace.ptr, workspace.nbytes,
+        ctypes.byref(tr) if tr is not None else None, _stream(stream))
+    _check(rc, "moe_sparse_block_threshold")
+    return out
+
+
+def residual_rmsnorm(h, y, x_next, eps: float = 1e-6, stream=None):
+    """h += y (FP32 residual, y bf16 or None); x_next = BF16(RMSNorm(h))."""
+    B, d = h.shape
+    rc = _lib.load().msb_residual_rmsnorm(_ptr(h), _ptr(y), _ptr(x_next), B, d, float(eps),
+                                          _stream(stream))
+    _check(rc, "msb_residual_rmsnorm")
+    return x_next
+
+
+def calibrate_threshold(scores: np.ndarray, budget: float) -> float:
+    """Offline calibration of the threshold comparator (not part of the decode path):
+    the score above which a fraction `budget` of the pooled calibration scores lie
+    (the (m+1)-th largest, m = floor(N * budget))."""
+    s = np.sort(np.asarray(scores, dtype=np.float64).ravel())[::-1]
+    m = int(np.floor(s.size * budget))
+    return float(s[min(m, s.size - 1)])

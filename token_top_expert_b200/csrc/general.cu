@@ -1,0 +1,706 @@
+// Multi-kernel sparse-MoE block path, any batch size 1..256.
+//
+//   router_kernel   logits, softmax, top-K, grouping of (token, expert) pairs by expert
+//   score_kernel    ternary-sketch channel scores on the tensor cores (+ z = B_e x)
+//   select_kernel   exact top-k (or threshold) per pair, per-expert union bitmap
+//   gather_kernel   gathered channel records -> SwiGLU -> down, A_e z, router-weighted
+//                   reduction into an FP32 accumulator
+//   finalize_kernel FP32 accumulator -> BF16 output (and re-zeroing)
+//
+// Each step follows the block definition of "KAIST drops calibration from MoE
+// decoding ..." ("Top-k instead of a threshold", "A reader built from weights
+// alone"); the batch path reads the union of the tokens' selected channels of
+// each expert once.
+#include "block_scan.cuh"
+#include "common.cuh"
+#include "launch.h"
+
+namespace msb {
+
+constexpr int kNT = 256;          // threads per CTA in every general kernel
+constexpr int kRouterTok = 8;     // tokens per router CTA
+constexpr int kScoreRows = 64;    // sketch rows per score CTA (4 tensor-core row tiles)
+constexpr int kScoreTok = 8;      // tokens per MMA n-tile
+constexpr int kLrRows = 256;      // A_e rows per low-rank CTA
+
+// =====================================================================================
+// router
+// =====================================================================================
+__global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict__ x, int B,
+                                                     const uint16_t* __restrict__ router_t, Dims D,
+                                                     Workspace ws, TraceDev tr) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = D.d, E = D.experts, K = D.top_e;
+  const int t0 = blockIdx.y * kRouterTok;
+  const int nt = min(kRouterTok, B - t0);
+
+  // zero this CTA's share of the output accumulator (rows t0.., a column slice)
+  {
+    const int cols = (d + gridDim.x - 1) / gridDim.x;
+    const int c0 = blockIdx.x * cols, c1 = min(d, c0 + cols);
+    for (int t = 0; t < nt; ++t)
+      for (int c = c0 + threadIdx.x; c < c1; c += kNT) ws.y_acc[(size_t)(t0 + t) * d + c] = 0.f;
+  }
+
+  const int e = blockIdx.x * (kNT / 32) + warp;
+  if (e < E) {
+    float acc[kRouterTok];
+#pragma unroll
+    for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
+    const uint4* wrow = reinterpret_cast<const uint4*>(router_t + (size_t)e * d);
+    for (int i = lane; i < d / 8; i += 32) {
+      const uint4 wv = __ldg(wrow + i);
+#pragma unroll
+      for (int t = 0; t < kRouterTok; ++t)
+        if (t < nt) {
+          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d) + i);
+          acc[t] = dot8(wv, xv, acc[t]);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < kRouterTok; ++t) {
+      const float s = warp_sum(acc[t]);
+      if (t < nt && lane == 0) ws.logits[(size_t)(t0 + t) * E + e] = s;
+    }
+  }
+
+  // ---- last CTA of this token group: softmax + top-K
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t old = atomicAdd(&ws.counters[kCntRouterGroup + blockIdx.y], 1u);
+    s_last = (old == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  if (warp < nt) {
+    const int t = t0 + warp;
+    constexpr int MAXM = MSB_MAX_EXPERTS / 32;
+    float v[MAXM];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m) {
+      const int ee = lane + 32 * m;
+      v[m] = ee < E ? __ldcg(&ws.logits[(size_t)t * E + ee]) : -INFINITY;
+      mx = fmaxf(mx, v[m]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int m = 0; m < MAXM; ++m)
+      if (lane + 32 * m < E) sum += expf(v[m] - mx);
+    sum = warp_sum(sum);
+    uint32_t taken = 0;
+    float pk[MSB_MAX_TOP_E];
+    int ik[MSB_MAX_TOP_E];
+    float psum = 0.f;
+    for (int r = 0; r < K; ++r) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int m = 0; m < MAXM; ++m) {
+        const int ee = lane + 32 * m;
+        if (ee < E && !((taken >> m) & 1u) && (v[m] > bv || (v[m] == bv && ee < bi))) {
+          bv = v[m];
+          bi = ee;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      pk[r] = expf(bv - mx);
+      ik[r] = bi;
+      psum += pk[r];
+    }
+    if (lane == 0) {
+      const float denom = D.renorm ? psum : sum;
+      for (int r = 0; r < K; ++r) {
+        const float w = pk[r] / denom;
+        ws.ids[t * K + r] = ik[r];
+        ws.wts[t * K + r] = w;
+        if (tr.expert_ids) tr.expert_ids[t * K + r] = ik[r];
+        if (tr.expert_w) tr.expert_w[t * K + r] = w;
+      }
+    }
+  }
+  if (threadIdx.x == 0) ws.counters[kCntRouterGroup + blockIdx.y] = 0;
+
+  // ---- last token group overall: group the (token, expert) pairs by expert
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t old = atomicAdd(&ws.counters[kCntRouterAll], 1u);
+    s_last = (old == gridDim.y - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+
+  __shared__ uint32_t cnt[MSB_MAX_EXPERTS];
+  __shared__ uint32_t tokmask[MSB_MAX_EXPERTS][MSB_MAX_BATCH / 32];
+  __shared__ uint32_t offs[MSB_MAX_EXPERTS];
+  __shared__ uint32_t slot[MSB_MAX_EXPERTS];
+  __shared__ uint32_t scan_tmp[kNT / 32 + 1];
+  const int nwords = (B + 31) / 32;
+  for (int i = threadIdx.x; i < E; i += kNT) {
+    cnt[i] = 0;
+    for (int w = 0; w < nwords; ++w) tokmask[i][w] = 0;
+  }
+  __syncthreads();
+  const int P = B * K;
+  for (int p = threadIdx.x; p < P; p += kNT) {
+    const int t = p / K;
+    const int ee = __ldcg(&ws.ids[p]);
+    atomicAdd(&cnt[ee], 1u);
+    atomicOr(&tokmask[ee][t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  // exclusive scans of counts and of "used" flags over experts (2 experts per thread)
+  {
+    const int e0 = 2 * threadIdx.x, e1 = e0 + 1;
+    const uint32_t c0 = e0 < E ? cnt[e0] : 0, c1 = e1 < E ? cnt[e1] : 0;
+    uint32_t tot;
+    const uint32_t pc = block_excl_scan<kNT>(c0 + c1, scan_tmp, &tot);
+    const uint32_t u0 = c0 > 0, u1 = c1 > 0;
+    uint32_t nu;
+    const uint32_t pu = block_excl_scan<kNT>(u0 + u1, scan_tmp, &nu);
+    if (e0 < E) { offs[e0] = pc; slot[e0] = pu; }
+    if (e1 < E) { offs[e1] = pc + c0; slot[e1] = pu + u0; }
+    if (e0 < E && c0) { ws.slot_expert[pu] = e0; ws.slot_off[pu] = pc; }
+    if (e1 < E && c1) { ws.slot_expert[pu + u0] = e1; ws.slot_off[pu + u0] = pc + c0; }
+    if (threadIdx.x == 0) { ws.slot_off[nu] = (int)tot; *ws.nused = (int)nu; }
+  }
+  __syncthreads();
+  for (int p = threadIdx.x; p < P; p += kNT) {
+    const int t = p / K;
+    const int ee = __ldcg(&ws.ids[p]);
+    uint32_t rank = 0;
+    for (int w = 0; w < (t >> 5); ++w) rank += __popc(tokmask[ee][w]);
+    rank += __popc(tokmask[ee][t >> 5] & ((1u << (t & 31)) - 1u));
+    const int pos = (int)(offs[ee] + rank);
+    ws.pair_tok[pos] = t;
+    ws.pair_w[pos] = __ldcg(&ws.wts[p]);
+    ws.pair_slot[pos] = (int)slot[ee];
+    ws.pair_of[p] = pos;
+  }
+  // clear the union bitmaps of every slot
+  const int uw = D.ipad / 32;
+  for (int i = threadIdx.x; i < E * uw; i += kNT) ws.umask[i] = 0u;
+  if (threadIdx.x == 0) ws.counters[kCntRouterAll] = 0;
+}
+
+// =====================================================================================
+// sketch scores (tensor cores) and z = B_e x
+// =====================================================================================
+// Dynamic shared memory: xperm [kScoreTok][KC*32 + 4] uint32, then part [4][64] floats.
+// xperm holds, per token n, chunk kc and lane column c, the eight bf16 pairs
+// (s, p) = B-fragment registers of the four 16-column steps of that chunk.
+__global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__ x,
+                                                    const uint32_t* __restrict__ sketch,
+                                                    const float* __restrict__ alpha,
+                                                    const uint16_t* __restrict__ lr_b, Dims D,
+                                                    Workspace ws, TraceDev tr, int z_only) {
+  extern __shared__ __align__(16) uint32_t smem[];
+  const int u = blockIdx.y;
+  if (u >= *ws.nused) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int d = D.d, KC = d / kColChunk, ipad = D.ipad;
+  const int e = ws.slot_expert[u];
+  const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
+  const int xstride = KC * 32 + 4;
+  uint32_t* xperm = smem;
+  float* part = reinterpret_cast<float*>(smem + kScoreTok * xstride);
+
+  // ---- z = B_e x for the rows of this CTA (row rho handled by CTA rho % gridDim.x)
+  if (D.rank > 0) {
+    for (int item = warp; ; item += kNT / 32) {
+      const int per = cnt;
+      const int local = item / per, ti = item % per;
+      const int rho = blockIdx.x + local * gridDim.x;
+      if (rho >= D.rank) break;
+      const int p = off + ti;
+      const int t = ws.pair_tok[p];
+      const uint4* brow = reinterpret_cast<const uint4*>(lr_b + ((size_t)e * D.rank + rho) * d);
+      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+      float acc = 0.f;
+      for (int i = lane; i < d / 8; i += 32) acc = dot8(__ldg(brow + i), __ldg(xr + i), acc);
+      acc = warp_sum(acc);
+      if (lane == 0) ws.z[(size_t)p * D.rank + rho] = acc;
+    }
+  }
+  if (z_only) return;
+
+  const int tile0 = blockIdx.x * (kScoreRows / kRowTile);
+  const int ntiles = min(kScoreRows / kRowTile, ipad / kRowTile - tile0);
+  if (ntiles <= 0) return;
+  const int rt = warp & 3, kh = warp >> 2;
+  const int kc0 = kh ? KC / 2 : 0, kc1 = kh ? KC : KC / 2;
+  const uint2* codes =
+      reinterpret_cast<const uint2*>(sketch) + ((size_t)(e * (ipad / kRowTile) + tile0 + rt) * KC) * 32 + lane;
+
+  for (int tt = 0; tt < cnt; tt += kScoreTok) {
+    const int ntok = min(kScoreTok, cnt - tt);
+    __syncthreads();
+    // build xperm for tokens pair_tok[off + tt + n]
+    for (int i = threadIdx.x; i < kScoreTok * KC * 32; i += kNT) {
+      const int n = i / (KC * 32);
+      const int rem = i % (KC * 32);
+      const int kc = rem >> 5, cc = (rem >> 3) & 3, q = rem & 7;
+      const int s = q >> 1, p = q & 1;
+      uint32_t v = 0;
+      if (n < ntok) {
+        const int t = ws.pair_tok[off + tt + n];
+        const int col = kc * kColChunk + 16 * s + 2 * cc + 8 * p;
+        v = __ldg(reinterpret_cast<const uint32_t*>(x + (size_t)t * d + col));
+      }
+      xperm[n * xstride + (kc * 4 + cc) * 8 + q] = v;
+    }
+    __syncthreads();
+    float sum[4] = {0.f, 0.f, 0.f, 0.f};
+    if (rt < ntiles) {
+      const uint32_t* xp = xperm + g * xstride + c * 8;
+#pragma unroll 4
+      for (int kc = kc0; kc < kc1; ++kc) {
+        const uint2 w = __ldg(codes + (size_t)kc * 32);
+        const uint4 xa = *reinterpret_cast<const uint4*>(xp + kc * 32);
+        const uint4 xb = *reinterpret_cast<const uint4*>(xp + kc * 32 + 4);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16(acc, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
+                 (w.y << 2) & kSketchMask, xa.x, xa.y);
+        mma_bf16(acc, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
+                 (w.y << 6) & kSketchMask, xa.z, xa.w);
+        mma_bf16(acc, (w.x << 8) & kSketchMask, (w.y << 8) & kSketchMask, (w.x << 10) & kSketchMask,
+                 (w.y << 10) & kSketchMask, xb.x, xb.y);
+        mma_bf16(acc, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask,
+                 (w.x << 14) & kSketchMask, (w.y << 14) & kSketchMask, xb.z, xb.w);
+        sum[0] += acc[0];
+        sum[1] += acc[1];
+        sum[2] += acc[2];
+        sum[3] += acc[3];
+      }
+    }
+    // combine the two k-halves: kh == 1 writes, kh == 0 adds
+    if (kh == 1 && rt < ntiles) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) part[(rt * 32 + lane) * 4 + i] = sum[i];
+    }
+    __syncthreads();
+    if (kh == 0 && rt < ntiles) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) sum[i] += part[(rt * 32 + lane) * 4 + i];
+      const int row0 = (tile0 + rt) * kRowTile + g;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int n = 2 * c + (i & 1);
+        const int row = row0 + (i >> 1) * 8;
+        if (n < ntok) {
+          const int p = off + tt + n;
+          const float s = __ldg(alpha + (size_t)e * ipad + row) * fabsf(sum[i]) * 0.5f;
+          ws.scores[(size_t)p * ipad + row] = s;
+          if (tr.scores) {
+            const int t = ws.pair_tok[p];
+            int r = 0;
+            while (ws.ids[t * D.top_e + r] != e) ++r;
+            tr.scores[((size_t)t * D.top_e + r) * ipad + row] = s;
+          }
+        }
+      }
+    }
+  }
+}
+
+// =====================================================================================
+// exact top-k / threshold selection per (token, expert) pair
+// =====================================================================================
+constexpr int kSelEPT = MSB_MAX_INTER / kNT;  // 16 keys per thread at most
+
+__global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau, Dims D,
+                                                     Workspace ws, TraceDev tr) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t info[4];
+  __shared__ uint32_t scan_tmp[kNT / 32 + 1];
+  __shared__ uint32_t words[MSB_MAX_INTER / 32];
+  const int p = blockIdx.x;
+  const int I = D.inter, ipad = D.ipad;
+  const int ept = (I + kNT - 1) / kNT;
+  const int j0 = threadIdx.x * ept;
+  uint32_t key[kSelEPT];
+  uint32_t valid = 0;
+#pragma unroll
+  for (int m = 0; m < kSelEPT; ++m) {
+    const int j = j0 + m;
+    key[m] = 0;
+    if (m < ept && j < I) {
+      key[m] = __float_as_uint(__ldcg(&ws.scores[(size_t)p * ipad + j]));
+      valid |= 1u << m;
+    }
+  }
+  for (int i = threadIdx.x; i < ipad / 32; i += kNT) words[i] = 0;
+  uint32_t kth = 0, need = 0;
+  if (mode == 0) radix_kth<kNT, kSelEPT>(key, valid, k, hist, info, &kth, &need);
+  const uint32_t tau_bits = __float_as_uint(tau);
+  // flags per element; count gt / eq for the ordered scan
+  uint32_t ngt = 0, neq = 0;
+#pragma unroll
+  for (int m = 0; m < kSelEPT; ++m) {
+    if (!((valid >> m) & 1u)) continue;
+    if (mode == 0) {
+      ngt += key[m] > kth;
+      neq += key[m] == kth;
+    } else {
+      ngt += __uint_as_float(key[m]) > __uint_as_float(tau_bits);
+    }
+  }
+  uint32_t tot;
+  const uint32_t pre = block_excl_scan<kNT>(ngt | (neq << 16), scan_tmp, &tot);
+  uint32_t gt_before = pre & 0xffffu, eq_before = pre >> 16;
+  const int t = ws.pair_tok[p];
+  const int slot = ws.pair_slot[p];
+  const int e = ws.slot_expert[slot];
+  int r = 0;
+  while (ws.ids[t * D.top_e + r] != e) ++r;
+  const size_t trow = (size_t)t * D.top_e + r;
+#pragma unroll
+  for (int m = 0; m < kSelEPT; ++m) {
+    if (!((valid >> m) & 1u)) continue;
+    const int j = j0 + m;
+    bool take;
+    if (mode == 0) {
+      const bool gt = key[m] > kth, eq = key[m] == kth;
+      take = gt || (eq && eq_before < need);
+      const uint32_t pos = gt_before + min(eq_before, need);
+      if (take) {
+        ws.sel[(size_t)p * ipad + pos] = (uint16_t)j;
+        if (tr.sel) tr.sel[trow * k + pos] = (uint16_t)j;
+      }
+      gt_before += gt;
+      eq_before += eq;
+    } else {
+      take = __uint_as_float(key[m]) > __uint_as_float(tau_bits);
+      if (take) {
+        ws.sel[(size_t)p * ipad + gt_before] = (uint16_t)j;
+        if (tr.sel) tr.sel[trow * I + gt_before] = (uint16_t)j;
+      }
+      gt_before += take;
+    }
+    if (take) atomicOr(&words[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+  const int count = mode == 0 ? k : (int)(tot & 0xffffu);
+  for (int i = threadIdx.x; i < ipad / 32; i += kNT) {
+    const uint32_t wv = words[i];
+    ws.selmask[(size_t)p * (ipad / 32) + i] = wv;
+    if (wv) atomicOr(&ws.umask[(size_t)slot * (ipad / 32) + i], wv);
+  }
+  if (threadIdx.x == 0) {
+    ws.selcnt[p] = count;
+    if (tr.sel_count) tr.sel_count[trow] = count;
+  }
+}
+
+// =====================================================================================
+// gathered channel records -> SwiGLU -> down; low-rank A_e z; weighted reduction
+// =====================================================================================
+// Dynamic shared memory: records [CH][3d] bf16 | xs [TG][d] bf16 | small scratch.
+struct GatherCfg {
+  int ch;       // channels per CTA
+  int tg;       // tokens per pass
+  int nchunk;   // channel-chunk CTAs per slot
+  int nlr;      // low-rank CTAs per slot
+  int dense;    // 1: every channel is selected (no sketch)
+};
+
+template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
+__global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict__ x,
+                                                     const uint16_t* __restrict__ records,
+                                                     const uint16_t* __restrict__ lr_a, Dims D,
+                                                     Workspace ws, GatherCfg cfg) {
+  constexpr int TG = 8 / IT;  // tokens per pass
+  extern __shared__ __align__(16) uint8_t gsm[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_list[64];
+  __shared__ int s_n;
+  __shared__ float s_red[kNT / 32][2 * 8];
+  __shared__ float s_h[64][8];
+  const int u = blockIdx.y;
+  if (u >= *ws.nused) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int d = D.d, I = D.inter, ipad = D.ipad, r = D.rank;
+  const int e = ws.slot_expert[u];
+  const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
+
+  // ------------------------------------------------------------- low-rank CTAs
+  if ((int)blockIdx.x >= cfg.nchunk) {
+    const int row = ((int)blockIdx.x - cfg.nchunk) * kLrRows + threadIdx.x;
+    if (row >= d || r == 0) return;
+    const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
+    for (int ti = 0; ti < cnt; ++ti) {
+      const int p = off + ti;
+      const float* z = ws.z + (size_t)p * r;
+      float acc = 0.f;
+      for (int q = 0; q < r; ++q) acc = fmaf(bf16_lo(arow[q]), __ldcg(z + q), acc);
+      atomicAdd(&ws.y_acc[(size_t)ws.pair_tok[p] * d + row], ws.pair_w[p] * acc);
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------- this chunk's channels
+  const int c0 = blockIdx.x * cfg.ch;
+  if (threadIdx.x < 32) {
+    if (cfg.dense) {
+      if (lane == 0) s_n = max(0, min(cfg.ch, I - c0));
+      for (int i = lane; i < cfg.ch; i += 32) s_list[i] = c0 + i;
+    } else {
+      const uint32_t* um = ws.umask + (size_t)u * (ipad / 32);
+      const int nw = ipad / 32;
+      const int per = (nw + 31) / 32;
+      uint32_t wv[4];
+      uint32_t pc = 0;
+      for (int i = 0; i < per; ++i) {
+        const int w = lane * per + i;
+        wv[i] = w < nw ? __ldcg(um + w) : 0u;
+        pc += __popc(wv[i]);
+      }
+      uint32_t inc = pc;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
+      }
+      uint32_t rank = inc - pc;
+      const uint32_t total = __shfl_sync(0xffffffffu, inc, 31);
+      for (int i = 0; i < per; ++i) {
+        uint32_t b = wv[i];
+        while (b) {
+          const int bit = __ffs(b) - 1;
+          b &= b - 1;
+          if (rank >= (uint32_t)c0 && rank < (uint32_t)(c0 + cfg.ch))
+            s_list[rank - c0] = (lane * per + i) * 32 + bit;
+          ++rank;
+        }
+      }
+      if (lane == 0) s_n = max(0, min(cfg.ch, (int)total - c0));
+    }
+  }
+  __syncthreads();
+  const int nch = s_n;
+  if (nch == 0) return;
+
+  uint16_t* rec = reinterpret_cast<uint16_t*>(gsm);
+  uint16_t* xs = rec + (size_t)cfg.ch * 3 * d;
+  const uint32_t rec_bytes = 6u * d;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bar, rec_bytes * nch);
+    for (int i = 0; i < nch; ++i)
+      bulk_g2s(rec + (size_t)i * 3 * d, records + ((size_t)e * I + s_list[i]) * 3 * d, rec_bytes, &bar);
+  }
+  // token x rows are staged per token group below; wait for the records first
+  __syncthreads();
+  if (!mbar_wait(&bar, 0, ws.err)) {
+    mbar_wait(&bar, 0, ws.err);
+    return;
+  }
+
+  for (int tg0 = 0; tg0 < cnt; tg0 += cfg.tg) {
+    const int ntg = min(cfg.tg, cnt - tg0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < ntg * d / 8; i += kNT) {
+      const int n = i / (d / 8), q = i % (d / 8);
+      const int t = ws.pair_tok[off + tg0 + n];
+      reinterpret_cast<uint4*>(xs + (size_t)n * d)[q] =
+          __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + q);
+    }
+    __syncthreads();
+    float y[TG][IT * 8];
+#pragma unroll
+    for (int n = 0; n < TG; ++n)
+#pragma unroll
+      for (int i = 0; i < IT * 8; ++i) y[n][i] = 0.f;
+
+    for (int ci = 0; ci < nch; ++ci) {
+      const int j = s_list[ci];
+      const uint16_t* grow = rec + (size_t)ci * 3 * d;
+      const uint16_t* urow = grow + d;
+      const uint16_t* drow = grow + 2 * d;
+      float pg[TG], pu[TG];
+#pragma unroll
+      for (int n = 0; n < TG; ++n) { pg[n] = 0.f; pu[n] = 0.f; }
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kNT + threadIdx.x) * 8;
+        if (el < d) {
+          const uint4 gv = *reinterpret_cast<const uint4*>(grow + el);
+          const uint4 uv = *reinterpret_cast<const uint4*>(urow + el);
+#pragma unroll
+          for (int n = 0; n < TG; ++n)
+            if (n < ntg) {
+              const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)n * d + el);
+              pg[n] = dot8(gv, xv, pg[n]);
+              pu[n] = dot8(uv, xv, pu[n]);
+            }
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < TG; ++n)
+        if (n < ntg) {
+          const float a = warp_sum(pg[n]);
+          const float b = warp_sum(pu[n]);
+          if (lane == 0) { s_red[warp][2 * n] = a; s_red[warp][2 * n + 1] = b; }
+        }
+      __syncthreads();
+      if (threadIdx.x < ntg) {
+        const int n = threadIdx.x;
+        float gsum = 0.f, usum = 0.f;
+        for (int w = 0; w < kNT / 32; ++w) { gsum += s_red[w][2 * n]; usum += s_red[w][2 * n + 1]; }
+        bool selected = true;
+        if (!cfg.dense) {
+          const int p = off + tg0 + n;
+          selected = (__ldcg(&ws.selmask[(size_t)p * (ipad / 32) + (j >> 5)]) >> (j & 31)) & 1u;
+        }
+        s_h[ci][n] = selected ? silu(gsum) * usum : 0.f;
+      }
+      __syncthreads();
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kNT + threadIdx.x) * 8;
+        if (el < d) {
+          const uint4 dv = *reinterpret_cast<const uint4*>(drow + el);
+          const float dd[8] = {bf16_lo(dv.x), bf16_hi(dv.x), bf16_lo(dv.y), bf16_hi(dv.y),
+                               bf16_lo(dv.z), bf16_hi(dv.z), bf16_lo(dv.w), bf16_hi(dv.w)};
+#pragma unroll
+          for (int n = 0; n < TG; ++n)
+            if (n < ntg) {
+              const float h = s_h[ci][n];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) y[n][it * 8 + i] = fmaf(h, dd[i], y[n][it * 8 + i]);
+            }
+        }
+      }
+    }
+    // weighted reduction into the FP32 accumulator
+#pragma unroll
+    for (int n = 0; n < TG; ++n)
+      if (n < ntg) {
+        const int p = off + tg0 + n;
+        const float w = ws.pair_w[p];
+        float* dst = ws.y_acc + (size_t)ws.pair_tok[p] * d;
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int el = (it * kNT + threadIdx.x) * 8;
+          if (el < d) {
+            red_add_v4(dst + el, w * y[n][it * 8 + 0], w * y[n][it * 8 + 1], w * y[n][it * 8 + 2],
+                       w * y[n][it * 8 + 3]);
+            red_add_v4(dst + el + 4, w * y[n][it * 8 + 4], w * y[n][it * 8 + 5],
+                       w * y[n][it * 8 + 6], w * y[n][it * 8 + 7]);
+          }
+        }
+      }
+  }
+}
+
+// =====================================================================================
+// FP32 accumulator -> BF16 output; union sizes for the trace
+// =====================================================================================
+__global__ void __launch_bounds__(kNT) finalize_kernel(uint16_t* __restrict__ out, int B, Dims D,
+                                                       Workspace ws, TraceDev tr, int dense) {
+  const size_t n8 = (size_t)B * D.d / 8;
+  for (size_t i = blockIdx.x * (size_t)kNT + threadIdx.x; i < n8; i += (size_t)gridDim.x * kNT) {
+    float4* src = reinterpret_cast<float4*>(ws.y_acc) + 2 * i;
+    const float4 a = __ldcg(src), b = __ldcg(src + 1);
+    src[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    src[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint4 o;
+    o.x = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.x)) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.y)) << 16);
+    o.y = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.z)) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a.w)) << 16);
+    o.z = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.x)) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.y)) << 16);
+    o.w = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.z)) |
+          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b.w)) << 16);
+    reinterpret_cast<uint4*>(out)[i] = o;
+  }
+  if (blockIdx.x == 0 && tr.union_count) {
+    const int nu = *ws.nused;
+    for (int e = threadIdx.x; e < D.experts; e += kNT) tr.union_count[e] = 0;
+    __syncthreads();
+    for (int u = threadIdx.x; u < nu; u += kNT) {
+      int c = 0;
+      if (dense) {
+        c = D.inter;
+      } else {
+        for (int w = 0; w < D.ipad / 32; ++w) c += __popc(ws.umask[(size_t)u * (D.ipad / 32) + w]);
+      }
+      tr.union_count[ws.slot_expert[u]] = c;
+    }
+  }
+}
+
+// =====================================================================================
+// host-side launcher
+// =====================================================================================
+int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uint16_t* records,
+                   const uint32_t* sketch, const float* alpha, int k, int mode, float tau,
+                   const uint16_t* lr_a, const uint16_t* lr_b, uint16_t* out, const Dims& D,
+                   const Workspace& ws, const TraceDev& tr, cudaStream_t st) {
+  const int E = D.experts, K = D.top_e, d = D.d;
+  const int dense = (mode == 0 && k == D.inter);
+  const int maxslots = min(E, B * K);
+  {
+    dim3 grid((E + 7) / 8, (B + kRouterTok - 1) / kRouterTok);
+    router_kernel<<<grid, kNT, 0, st>>>(x, B, router_t, D, ws, tr);
+  }
+  const int KC = d / kColChunk;
+  const size_t score_smem = (size_t)kScoreTok * (KC * 32 + 4) * 4 + 4 * 32 * 4 * 4;
+  if (!dense || D.rank > 0) {
+    dim3 grid((D.ipad + kScoreRows - 1) / kScoreRows, maxslots);
+    score_kernel<<<grid, kNT, score_smem, st>>>(x, sketch, alpha, lr_b, D, ws, tr, dense);
+  }
+  if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
+  GatherCfg cfg;
+  const int IT = (d + 2047) / 2048;
+  const int ITc = IT <= 1 ? 1 : IT <= 2 ? 2 : 4;
+  cfg.tg = 8 / ITc;
+  cfg.ch = max(1, min(64, (96 * 1024) / (6 * d)));
+  cfg.nchunk = (D.inter + cfg.ch - 1) / cfg.ch;
+  cfg.nlr = D.rank > 0 ? (d + kLrRows - 1) / kLrRows : 0;
+  cfg.dense = dense;
+  const size_t gsmem = (size_t)cfg.ch * 6 * d + (size_t)cfg.tg * 2 * d;
+  dim3 ggrid(cfg.nchunk + cfg.nlr, maxslots);
+  switch (ITc) {
+    case 1: gather_kernel<1><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
+    case 2: gather_kernel<2><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
+    default: gather_kernel<4><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
+  }
+  {
+    const size_t n8 = (size_t)B * d / 8;
+    const size_t nb = (n8 + kNT - 1) / kNT;
+    const int blocks = (int)(nb < 148 * 4 ? nb : 148 * 4);
+    finalize_kernel<<<blocks, kNT, 0, st>>>(out, B, D, ws, tr, dense);
+  }
+  return cudaGetLastError() == cudaSuccess ? MSB_OK : MSB_ECUDA;
+}
+
+int general_set_smem_limits() {
+  const int big = 200 * 1024;
+  cudaError_t e = cudaSuccess;
+  e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (e != cudaSuccess) return MSB_ECUDA;
+  e = cudaFuncSetAttribute(gather_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (e != cudaSuccess) return MSB_ECUDA;
+  e = cudaFuncSetAttribute(gather_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (e != cudaSuccess) return MSB_ECUDA;
+  e = cudaFuncSetAttribute(gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
+}
+
+}  // namespace msb
