@@ -52,6 +52,8 @@ extern "C" {
 #define MSB_EUNSUPPORTED (-2)  /* sizes beyond the compiled limits below */
 #define MSB_ECUDA (-3)         /* a CUDA launch or runtime call failed */
 #define MSB_ETIMEOUT (-4)      /* (msb_check) a kernel's bounded wait ran out */
+#define MSB_ENONFINITE (-5)    /* (msb_check) the router met NaN/Inf logits: x or W_router
+                                  is not finite (invalid input; the output is undefined) */
 
 /* ------------------------------------------------------------------ limits */
 #define MSB_MAX_D 8192         /* hidden size d: multiple of 64, 64..8192 */
@@ -136,7 +138,8 @@ size_t msb_workspace_size(const msb_dims* dims, int32_t max_batch);
 int32_t msb_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace's sticky error word.
- * Returns MSB_OK, MSB_ETIMEOUT, or MSB_ECUDA if the stream itself failed. */
+ * Returns MSB_OK, MSB_ETIMEOUT, MSB_ENONFINITE, or MSB_ECUDA if the stream
+ * itself failed. */
 int32_t msb_check(void* workspace, void* stream);
 
 const char* msb_strerror(int32_t status);

@@ -15,6 +15,7 @@ MSB_EINVAL = -1
 MSB_EUNSUPPORTED = -2
 MSB_ECUDA = -3
 MSB_ETIMEOUT = -4
+MSB_ENONFINITE = -5
 MSB_FLAG_GENERAL = 1
 
 MSB_MAX_D = 8192

@@ -65,10 +65,10 @@ Layout layout(const Dims& D, int B) {
   L.pair_slot = o;     o = up(o + 4 * P);
   L.pair_of = o;       o = up(o + 4 * P);
   L.scores = o;        o = up(o + 4 * P * D.ipad);
-  L.selmask = o;       o = up(o + 4 * P * (D.ipad / 32 + 1));
+  L.selmask = o;       o = up(o + 4 * P * mask_words(D.ipad));
   L.sel = o;           o = up(o + 2 * P * D.ipad);
   L.selcnt = o;        o = up(o + 4 * P);
-  L.umask = o;         o = up(o + 4 * E * (D.ipad / 32 + 1));
+  L.umask = o;         o = up(o + 4 * E * mask_words(D.ipad));
   L.z = o;             o = up(o + 4 * P * (size_t)(D.rank > 0 ? D.rank : 1));
   L.total = o;
   return L;
@@ -219,7 +219,7 @@ int32_t msb_check(void* workspace, void* stream) {
   if (cudaMemcpyAsync(workspace, &zero, 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MSB_ECUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return MSB_ECUDA;
-  return MSB_ETIMEOUT;
+  return (err & kErrTimeout) ? MSB_ETIMEOUT : MSB_ENONFINITE;
 }
 
 const char* msb_strerror(int32_t status) {
@@ -230,6 +230,7 @@ const char* msb_strerror(int32_t status) {
     case MSB_EUNSUPPORTED: return "size beyond the compiled limits";
     case MSB_ECUDA: return "CUDA launch or runtime error";
     case MSB_ETIMEOUT: return "a kernel's bounded wait ran out";
+    case MSB_ENONFINITE: return "non-finite router logits (x or W_router has NaN/Inf)";
     default: return "unknown status";
   }
 }

@@ -29,9 +29,12 @@ constexpr int kChunkWords = 64;
 constexpr uint32_t kSketchMask = 0xC000C000u;
 
 __host__ __device__ inline int pad16(int v) { return (v + 15) & ~15; }
+// 32-bit words of a per-channel bitmask over ipad channels
+__host__ __device__ inline int mask_words(int ipad) { return (ipad + 31) / 32; }
 
 // ---------------------------------------------------------------- device error word
 constexpr uint32_t kErrTimeout = 1u;
+constexpr uint32_t kErrNonFinite = 2u;  // router saw NaN/Inf logits (invalid input)
 constexpr uint32_t kSpinLimit = 1u << 22;            // polls before a wait gives up ...
 constexpr uint64_t kWaitLimitNs = 2000ull * 1000000;  // ... or 2 s of wall time, whichever first
 

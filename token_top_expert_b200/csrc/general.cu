@@ -114,6 +114,11 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
         const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
       }
+      if (bi >= E) {  // non-finite logits: keep a valid index and flag the call
+        bi = r;
+        bv = mx;
+        if (lane == 0) atomicOr(ws.err, kErrNonFinite);
+      }
       if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
       pk[r] = expf(bv - mx);
       ik[r] = bi;
@@ -191,7 +196,7 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
     ws.pair_of[p] = pos;
   }
   // clear the union bitmaps of every slot
-  const int uw = D.ipad / 32;
+  const int uw = mask_words(D.ipad);
   for (int i = threadIdx.x; i < E * uw; i += kNT) ws.umask[i] = 0u;
   if (threadIdx.x == 0) ws.counters[kCntRouterAll] = 0;
 }
@@ -343,7 +348,7 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
       valid |= 1u << m;
     }
   }
-  for (int i = threadIdx.x; i < ipad / 32; i += kNT) words[i] = 0;
+  for (int i = threadIdx.x; i < mask_words(ipad); i += kNT) words[i] = 0;
   uint32_t kth = 0, need = 0;
   if (mode == 0) radix_kth<kNT, kSelEPT>(key, valid, k, hist, info, &kth, &need);
   const uint32_t tau_bits = __float_as_uint(tau);
@@ -395,10 +400,11 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
   }
   __syncthreads();
   const int count = mode == 0 ? k : (int)(tot & 0xffffu);
-  for (int i = threadIdx.x; i < ipad / 32; i += kNT) {
+  const int mw = mask_words(ipad);
+  for (int i = threadIdx.x; i < mw; i += kNT) {
     const uint32_t wv = words[i];
-    ws.selmask[(size_t)p * (ipad / 32) + i] = wv;
-    if (wv) atomicOr(&ws.umask[(size_t)slot * (ipad / 32) + i], wv);
+    ws.selmask[(size_t)p * mw + i] = wv;
+    if (wv) atomicOr(&ws.umask[(size_t)slot * mw + i], wv);
   }
   if (threadIdx.x == 0) {
     ws.selcnt[p] = count;
@@ -459,8 +465,8 @@ __global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict_
       if (lane == 0) s_n = max(0, min(cfg.ch, I - c0));
       for (int i = lane; i < cfg.ch; i += 32) s_list[i] = c0 + i;
     } else {
-      const uint32_t* um = ws.umask + (size_t)u * (ipad / 32);
-      const int nw = ipad / 32;
+      const int nw = mask_words(ipad);
+      const uint32_t* um = ws.umask + (size_t)u * nw;
       const int per = (nw + 31) / 32;
       uint32_t wv[4];
       uint32_t pc = 0;
@@ -564,7 +570,7 @@ __global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict_
         bool selected = true;
         if (!cfg.dense) {
           const int p = off + tg0 + n;
-          selected = (__ldcg(&ws.selmask[(size_t)p * (ipad / 32) + (j >> 5)]) >> (j & 31)) & 1u;
+          selected = (__ldcg(&ws.selmask[(size_t)p * mask_words(ipad) + (j >> 5)]) >> (j & 31)) & 1u;
         }
         s_h[ci][n] = selected ? silu(gsum) * usum : 0.f;
       }
@@ -638,7 +644,7 @@ __global__ void __launch_bounds__(kNT) finalize_kernel(uint16_t* __restrict__ ou
       if (dense) {
         c = D.inter;
       } else {
-        for (int w = 0; w < D.ipad / 32; ++w) c += __popc(ws.umask[(size_t)u * (D.ipad / 32) + w]);
+        for (int w = 0; w < mask_words(D.ipad); ++w) c += __popc(ws.umask[(size_t)u * mask_words(D.ipad) + w]);
       }
       tr.union_count[ws.slot_expert[u]] = c;
     }
