@@ -370,15 +370,17 @@ def main():
 
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
-    kernel = "moe_block_fused" if (B == 1 and not general) else "moe_block_general"
+    plan = msb.path_info(dims, B, args.k, general=general)
+    kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
     traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else ""))
-    launches_per_step = 1 if kernel == "moe_block_fused" else (3 if dense else 5)
+    launches_per_step = 1 if plan["path"] == "single_launch" else (
+        (3 if args.rank == 0 else 4) if dense else 5)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world if world > 1 else 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,0.02) BF16 weights, 5% rows x4; x ~ N(0,1))",
-        "config": config_of(w, args),
+        "config": dict(config_of(w, args), path=plan),
         "us_per_block": ms_per_step * 1e3,
         "bytes_per_step": step_bytes, "router_bytes_per_step": router_bytes,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",

@@ -144,6 +144,15 @@ int32_t msb_check(void* workspace, void* stream);
 
 const char* msb_strerror(int32_t status);
 
+/* Diagnostics: the path moe_sparse_block takes for these arguments on the
+ * current device.  Fills info (host, 8 int32):
+ *   {path (1 = single launch, 2 = multi-kernel), cluster size, clusters per
+ *    routed expert, channel-record ring slots, dynamic shared-memory bytes,
+ *    resident 16-CTA clusters, resident 8-CTA clusters, 0}.
+ * Returns MSB_OK, MSB_EINVAL / MSB_EUNSUPPORTED for bad sizes, or MSB_ECUDA. */
+int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t flags,
+                      int32_t* info);
+
 /* ------------------------------------------------------------------ the block
  * out[t] = sum over the K routed experts e of token t of
  *          w_{t,e} * ( sum_{j in S_{t,e}} silu(gate_j . x_t) * (up_j . x_t) * down[:, j]

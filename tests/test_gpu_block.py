@@ -31,6 +31,9 @@ def dev_from_arrays(msb, lw, w, rank):
 def test_tiny_block_all_steps(msb, general):
     w = synth.TINY
     dev = device_layer(w)
+    info = msb.path_info(dev.dims, 1, w.k, general=general)
+    print(info)
+    assert info["path"] == ("multi_kernel" if general else "single_launch")
     lay = oracle.SynthLayer(w, max_cache=w.experts)
     worst = 0.0
     for step in range(w.steps):
@@ -48,6 +51,9 @@ def test_tiny_block_all_steps(msb, general):
 def test_qwen_block_batch1(msb, general):
     w = synth.QWEN30B_BLOCK
     dev = device_layer(w)
+    info = msb.path_info(dev.dims, 1, w.k, general=general)
+    print(info)
+    assert info["path"] == ("multi_kernel" if general else "single_launch")
     lay = oracle.SynthLayer(w)
     for step in (0, 1, 7, 123, 999):
         x = synth.activations(w, step)
@@ -57,13 +63,16 @@ def test_qwen_block_batch1(msb, general):
         print(step, st)
 
 
-def test_qwen_block_dense_k768(msb):
+@pytest.mark.parametrize("general", [False, True])
+def test_qwen_block_dense_k768(msb, general):
     w = synth.QWEN30B_BLOCK
     dev = device_layer(w, rank=0)
+    assert msb.path_info(dev.dims, 1, w.inter, general=general)["path"] == (
+        "multi_kernel" if general else "single_launch")
     lay = oracle.SynthLayer(w)
     for step in (0, 5):
         x = synth.activations(w, step)
-        g = run_gpu(x, dev, w.inter)
+        g = run_gpu(x, dev, w.inter, general=general)
         st = compare(x, g, lay, w.top_e, w.inter, mode="dense")
         used = set(int(e) for e in g["ids"][0])
         for e in range(w.experts):
@@ -119,6 +128,8 @@ def test_threshold_comparator(msb):
 def test_large_block(msb, batch):
     w = synth.LARGE_BLOCK
     dev = device_layer(w)
+    if batch == 1:
+        assert msb.path_info(dev.dims, 1, w.k)["path"] == "single_launch"
     lay = oracle.SynthLayer(w)
     x = synth.activations(w, 11, batch=batch)
     g = run_gpu(x, dev, w.k)

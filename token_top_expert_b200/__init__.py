@@ -13,6 +13,7 @@ from .block import (  # noqa: F401
     moe_sparse_block,
     moe_sparse_block_threshold,
     pack,
+    path_info,
     residual_rmsnorm,
     sketch_words,
     workspace_size,

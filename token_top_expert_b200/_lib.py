@@ -29,7 +29,7 @@ MSB_MAX_BATCH = 256
 SYMBOLS = (
     "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_workspace_size",
     "msb_workspace_init", "msb_check", "msb_strerror", "moe_sparse_block",
-    "moe_sparse_block_threshold", "msb_residual_rmsnorm",
+    "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
 )
 
 
@@ -78,6 +78,7 @@ def load() -> ctypes.CDLL:
         "moe_sparse_block_threshold": (I32, [P, I32, P, P, P, P, F32, P, P, P, dims_p, P, SZ,
                                              trace_p, P]),
         "msb_residual_rmsnorm": (I32, [P, P, P, I32, I32, F32, P]),
+        "msb_path_info": (I32, [dims_p, I32, I32, U32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

@@ -214,6 +214,18 @@ def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
     return out
 
 
+def path_info(dims: Dims, batch: int, k: int, general: bool = False) -> dict:
+    """Which path moe_sparse_block takes on the current device, and its plan."""
+    info = (ctypes.c_int32 * 8)()
+    rc = _lib.load().msb_path_info(ctypes.byref(dims.c()), batch, k,
+                                   _lib.MSB_FLAG_GENERAL if general else 0, info)
+    _check(rc, "msb_path_info")
+    v = list(info)
+    return {"path": "single_launch" if v[0] == 1 else "multi_kernel", "cluster_size": v[1],
+            "clusters_per_expert": v[2], "ring_slots": v[3], "smem_bytes": v[4],
+            "resident_clusters16": v[5], "resident_clusters8": v[6]}
+
+
 def residual_rmsnorm(h, y, x_next, eps: float = 1e-6, stream=None):
     """h += y (FP32 residual, y bf16 or None); x_next = BF16(RMSNorm(h))."""
     B, d = h.shape

@@ -255,6 +255,24 @@ int32_t moe_sparse_block_threshold(const void* x, int32_t batch, const void* rou
                       dims, workspace, workspace_bytes, trace, MSB_FLAG_GENERAL, stream);
 }
 
+int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t flags,
+                      int32_t* info) {
+  int rc = check_dims(dims);
+  if (rc != MSB_OK) return rc;
+  if (!info || batch < 1 || k < 1 || k > dims->inter) return MSB_EINVAL;
+  if (batch > MSB_MAX_BATCH) return MSB_EUNSUPPORTED;
+  rc = ensure_setup();
+  if (rc != MSB_OK) return rc;
+  const Dims D = to_dims(*dims);
+  int p[6];
+  fused_plan_info(D, k, p);
+  const bool fused = batch == 1 && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k);
+  info[0] = fused ? 1 : 2;
+  for (int i = 0; i < 6; ++i) info[1 + i] = p[i];
+  info[7] = 0;
+  return MSB_OK;
+}
+
 int32_t msb_residual_rmsnorm(float* h, const void* y, void* x_next, int32_t batch, int32_t d,
                              float eps, void* stream) {
   if (!h || !x_next || batch < 1 || d < 64 || d % 64 != 0 || !(eps >= 0.f)) return MSB_EINVAL;

@@ -108,6 +108,10 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   Misc& M = *reinterpret_cast<Misc*>(sm + P.o_misc);
   uint8_t* big = sm + P.o_big;
 
+  // Every CTA of the cluster must be running before any DSMEM store targets it:
+  // arrive now, wait just before the first remote store (overlaps the loads).
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+
   // ------------------------------------------------------------------ phase A: router
   const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
   if (tid == 0) {
@@ -122,6 +126,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   __syncthreads();
   bool ok = mbar_wait(&M.bar[0], 0, P.err);
   ok = __syncthreads_and(ok);
+  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   if (ok) {
     const uint16_t* rows = reinterpret_cast<const uint16_t*>(big);
     for (int row = warp; row < e_hi - e_lo; row += kFW) {
@@ -557,11 +562,18 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe) {
   return P.smem <= kSmemMax;
 }
 
+// Prefer one 16-CTA cluster per routed expert when K of them are resident at once,
+// else two 8-CTA clusters per expert when 2K are; otherwise whichever shape can be
+// resident at all (clusters that do not fit wait for a free GPC: correct, slower).
 bool choose(FusedParams& P, const Dims& D, int k) {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64 || !g_ready[dev]) return false;
-  if (D.d % (8 * 16) == 0 && g_max_clusters16[dev] >= D.top_e && plan(P, D, k, 16, 1)) return true;
-  if (D.d % (8 * 8) == 0 && g_max_clusters8[dev] >= 2 * D.top_e && plan(P, D, k, 8, 2)) return true;
+  const bool ok16 = D.d % (8 * 16) == 0 && g_max_clusters16[dev] >= 1;
+  const bool ok8 = D.d % (8 * 8) == 0 && g_max_clusters8[dev] >= 1;
+  if (ok16 && g_max_clusters16[dev] >= D.top_e && plan(P, D, k, 16, 1)) return true;
+  if (ok8 && g_max_clusters8[dev] >= 2 * D.top_e && plan(P, D, k, 8, 2)) return true;
+  if (ok16 && plan(P, D, k, 16, 1)) return true;
+  if (ok8 && plan(P, D, k, 8, 2)) return true;
   return false;
 }
 }  // namespace
@@ -597,6 +609,23 @@ int fused_setup() {
   }
   g_ready[dev] = true;
   return MSB_OK;
+}
+
+void fused_plan_info(const Dims& D, int k, int* info) {
+  FusedParams P{};
+  P.dense = (k == D.inter);
+  const int dev = cur_dev();
+  for (int i = 0; i < 6; ++i) info[i] = 0;
+  if (choose(P, D, k)) {
+    info[0] = P.cs;
+    info[1] = P.cpe;
+    info[2] = P.ring;
+    info[3] = P.smem;
+  }
+  if (dev >= 0 && dev < 64) {
+    info[4] = g_max_clusters16[dev];
+    info[5] = g_max_clusters8[dev];
+  }
 }
 
 bool fused_supported(const Dims& D, int k) {

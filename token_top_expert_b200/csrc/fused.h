@@ -11,6 +11,8 @@ namespace msb {
 constexpr int MSB_ENOTFUSED = 1;  // internal: the fused path declines, use the general path
 
 bool fused_supported(const Dims& D, int k);
+// {cluster size, clusters per expert, ring slots, smem bytes, max 16-clusters, max 8-clusters}
+void fused_plan_info(const Dims& D, int k, int* info6);
 int fused_setup();
 int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* records,
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
