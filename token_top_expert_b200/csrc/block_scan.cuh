@@ -1,4 +1,4 @@
-// Block-wide scans and the exact top-k radix select used by the selection kernels.
+// Block-wide scans and the exact top-k radix select used by the selection steps.
 #pragma once
 
 #include "common.cuh"
@@ -37,44 +37,46 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* tmp, u
   return res;
 }
 
-// Exact top-k over non-negative float keys given as their bit patterns (bit
-// order == value order for non-negative floats).  Each thread holds up to EPT
-// keys of a contiguous index range; `valid` masks entries beyond n.
-// Finds the k-th largest key `kth` and `need` = how many keys equal to it are
-// taken (the lowest-index ones), by an MSB-first 8-bit radix descent.
-// Shared scratch: hist[256], info[4].
-template <int NT, int EPT>
-__device__ __forceinline__ void radix_kth(const uint32_t (&key)[EPT], uint32_t valid, int k,
-                                          uint32_t* hist, uint32_t* info, uint32_t* kth,
-                                          uint32_t* need) {
+// Exact top-k over n non-negative float keys held in shared memory as their bit
+// patterns (bit order == value order for non-negative floats).  Finds the k-th
+// largest key `kth` and `need` = how many keys equal to it are taken (the
+// lowest-index ones), by an MSB-first 8-bit radix descent.  Runtime loops keep
+// the code small.  Shared scratch: hist[512] (two alternating histograms, so the
+// next pass's bins are cleared while this pass counts), info[2].
+template <int NT>
+__device__ __forceinline__ void radix_kth_smem(const uint32_t* keys, int n, int k, uint32_t* hist2,
+                                               uint32_t* info, uint32_t* kth, uint32_t* need) {
   uint32_t prefix = 0, mask = 0;
   uint32_t kk = (uint32_t)k;
+  for (int i = threadIdx.x; i < 256; i += NT) hist2[i] = 0;
+  __syncthreads();
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += NT) hist[i] = 0;
-    __syncthreads();
-#pragma unroll
-    for (int m = 0; m < EPT; ++m)
-      if (((valid >> m) & 1u) && (key[m] & mask) == prefix) atomicAdd(&hist[(key[m] >> shift) & 255u], 1u);
+  for (int shift = 24, pass = 0; shift >= 0; shift -= 8, ++pass) {
+    uint32_t* hist = hist2 + 256 * (pass & 1);
+    uint32_t* next = hist2 + 256 * ((pass + 1) & 1);
+    for (int i = threadIdx.x; i < 256; i += NT) next[i] = 0;
+    // shared-memory atomics handle same-bin contention in hardware
+#pragma unroll 1
+    for (int j = threadIdx.x; j < n; j += NT) {
+      const uint32_t key = keys[j];
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
     __syncthreads();
     if (threadIdx.x < 32) {
       const int lane = threadIdx.x;
-      // lane owns digits [8*(31-lane), 8*(31-lane)+8): lane 0 the highest digits
+      // lane owns digits [8*(31-lane), +8): lane 0 the highest digits
       const int base = 8 * (31 - lane);
       uint32_t c[8], s = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i) { c[i] = hist[base + i]; s += c[i]; }
-      // inclusive scan over lanes (lane 0 = highest digits)
       uint32_t inc = s;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
+        uint32_t t = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += t;
       }
-      uint32_t above = inc - s;  // keys with a digit higher than this lane's range
-      // the digit D with above(D) < kk <= above(D) + hist[D], scanning down from the top
-      bool mine = above < kk && kk <= inc;
-      if (mine) {
+      const uint32_t above = inc - s;  // keys with a higher digit than this lane's range
+      if (above < kk && kk <= inc) {
         uint32_t a = above;
 #pragma unroll
         for (int i = 7; i >= 0; --i) {
@@ -87,10 +89,33 @@ __device__ __forceinline__ void radix_kth(const uint32_t (&key)[EPT], uint32_t v
     prefix |= info[0] << shift;
     mask |= 255u << shift;
     kk = info[1];
-    __syncthreads();
   }
+  __syncthreads();
   *kth = prefix;
   *need = kk;
+}
+
+// Given the k-th key and how many of the equal keys to take, write the selected
+// indices (ascending) to sel[0..k).  Thread t owns the contiguous index range
+// [t*ept, (t+1)*ept).  Returns the number written by the block (== k).
+template <int NT>
+__device__ __forceinline__ void scatter_topk(const uint32_t* keys, int n, uint32_t kth,
+                                             uint32_t need, uint16_t* sel, uint32_t* scan_tmp) {
+  const int ept = (n + NT - 1) / NT;
+  const int j0 = threadIdx.x * ept, j1 = min(n, j0 + ept);
+  uint32_t ngt = 0, neq = 0;
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) { ngt += keys[j] > kth; neq += keys[j] == kth; }
+  uint32_t tot;
+  const uint32_t pre = block_excl_scan<NT>(ngt | (neq << 16), scan_tmp, &tot);
+  uint32_t gtb = pre & 0xffffu, eqb = pre >> 16;
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) {
+    const bool gt = keys[j] > kth, eq = keys[j] == kth;
+    if (gt || (eq && eqb < need)) sel[gtb + min(eqb, need)] = (uint16_t)j;
+    gtb += gt;
+    eqb += eq;
+  }
 }
 
 }  // namespace msb

@@ -199,9 +199,9 @@ struct Workspace {
 
 constexpr int kCounters = 1024;
 // counter indices
-constexpr int kCntFused = 0;        // fused kernel: CTAs finished
-constexpr int kCntRouterAll = 1;    // router: token groups finished
-constexpr int kCntRouterGroup = 8;  // router: CTAs finished per token group (up to 64 groups)
+constexpr int kCntRouterAll = 1;      // router: token groups finished
+constexpr int kCntRouterGroup = 8;    // router: CTAs finished per token group (32 groups)
+constexpr int kCntFusedSlices = 64;   // single-launch path: contributions per output slice (16)
 
 struct Dims {
   int d, inter, ipad, experts, top_e, rank, renorm;

@@ -1,23 +1,26 @@
 // Single-launch batch-1 sparse-MoE block (the decode hot path).
 //
-// One thread-block cluster per routed expert (or two clusters of 8 when 16-CTA
-// clusters cannot all be resident).  All exchange inside a cluster goes through
-// distributed shared memory and hardware cluster barriers; the only global
-// synchronisation is the last-arriving CTA that converts the FP32 accumulator
-// to BF16.  Phases:
+// One thread-block cluster per routed expert (or two smaller clusters per
+// expert).  Exchange inside a cluster goes through distributed shared memory and
+// hardware cluster barriers; across clusters only through FP32 atomics into a
+// small accumulator whose last contributor (per output slice) writes BF16.
 //
 //  A  router: the cluster's CTAs each score E/CS experts (x . W_router rows
 //     staged by 1-D bulk copies), broadcast the logits over DSMEM; every CTA then
 //     runs softmax + top-K and cluster c takes the c-th ranked expert.
 //  B  sketch scores: each CTA stages its 16-row tiles of the packed 2-bit sketch,
 //     scores them on the tensor cores (the packed codes are the bf16 A fragment),
-//     broadcasts alpha*|T.x| to the cluster; z = B_e x rows are computed alongside.
+//     broadcasts alpha*|T.x| to the cluster; z = B_e x rows alongside.
 //  C  exact top-k: every CTA selects the same k channels (radix select, ties to the
 //     lower index); each CTA streams its share of the 6d-byte channel records
 //     through a shared-memory ring and accumulates SwiGLU(gate.x, up.x) * down.
-//  D  the cluster reduces its partial outputs over DSMEM (CTA q owns a d/CS
-//     slice), adds A_e z, scales by the router weight and adds into the FP32
-//     accumulator; the last CTA of the grid writes the BF16 output.
+//  D  partial outputs are reduce-added into the owning CTA's slice over DSMEM;
+//     the owner adds A_e z, scales by the router weight and adds into the FP32
+//     accumulator; the last contribution to a slice converts it to BF16.
+//
+// The kernel is launched with programmatic stream serialisation: everything that
+// reads only weights (barrier set-up, router rows) runs before
+// griddepcontrol.wait, so it overlaps the previous launch's tail.
 //
 // "KAIST drops calibration from MoE decoding ...": "Top-k instead of a threshold"
 // (fixed read budget), "A reader built from weights alone" (ternary sketch filter
@@ -37,6 +40,7 @@ constexpr int kFW = kFT / 32;   // warps per CTA
 constexpr int kRingMax = 16;    // record slots
 constexpr int kGroup = 8;       // channels reduced together
 constexpr int kSmemMax = 227 * 1024;
+constexpr int kSmemPair = 110 * 1024;  // at or below this, two CTAs can share an SM
 
 struct FusedParams {
   const uint16_t* x;
@@ -48,7 +52,7 @@ struct FusedParams {
   const uint16_t* lr_b;
   uint16_t* out;
   uint32_t* err;
-  uint32_t* counter;
+  uint32_t* slice_cnt;  // [cs] arrival counters, one per output slice
   float* y_acc;
   TraceDev tr;
   Dims D;
@@ -56,11 +60,12 @@ struct FusedParams {
   int rpc;     // router rows per CTA
   int tpc;     // sketch row tiles per CTA
   int zpc;     // z rows per CTA (max)
-  int slice;   // output elements owned per CTA in the cluster reduction (d / cs)
+  int slice;   // output elements owned per CTA (d / cs)
   int ring;    // record slots
   int group;   // channels per reduction group (<= ring)
   // shared-memory carve-up (byte offsets)
-  int o_x, o_logits, o_scores, o_alpha, o_z, o_sel, o_part, o_ybuf, o_aslice, o_misc, o_big;
+  int o_x, o_xperm, o_logits, o_keys, o_alpha, o_z, o_sel, o_part, o_ylr, o_misc, o_big;
+  int o_aslice_off;  // A_e rows: byte offset inside big, past every other use of big
   int smem;
 };
 
@@ -68,21 +73,153 @@ struct Misc {
   uint64_t bar[2 + kRingMax];
   int ids[MSB_MAX_TOP_E];
   float w[MSB_MAX_TOP_E];
-  uint32_t hist[256];
-  uint32_t info[4];
+  uint32_t hist[512];
+  uint32_t info[2];
   uint32_t scan[kFT / 32 + 1];
   float red[kFW][2 * kGroup];
   float h[kGroup];
+  float maxv;
+  float wsum[kFW];
+  float pe[MSB_MAX_TOP_E];
   int last;
-  int ok;
 };
 
-__device__ __forceinline__ void store_cluster(cg::cluster_group& cl, float* local, int idx, float v,
-                                              int lane, int cs) {
-  // lanes 0..cs-1 each write one destination CTA
-  if (lane < cs) cl.map_shared_rank(local, lane)[idx] = v;
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// The kernel runs once per CTA per launch, so its code is fetched cold every time
+// (on B200, cold straight-line code costs ~0.4 us per KB per SM).  It is written
+// for a small footprint: loops with short bodies, shared helpers kept out of line,
+// fast intrinsics for the few transcendental steps.
+
+// Bounded wait on an mbarrier phase (shared by every wait site).
+__device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  return mbar_wait(bar, parity, err);
+}
+
+// Router top-K over the E logits in shared memory, by rank counting:
+// rank(e) = #{e' : l_e' > l_e or (l_e' == l_e and e' < e)}, two threads per logit.
+// Writes M.ids[0..K) (rank order) and the combine weights M.w[0..K).
+__device__ __noinline__ void router_topk(const float* logits, int E, int K, int renorm, Misc& M,
+                                         uint32_t* err) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < K) M.ids[tid] = -1;
+  __syncthreads();
+  const int halfE = E / 2;
+#pragma unroll 1
+  for (int base = 0; base < 2 * E; base += kFT) {
+    const int item = base + tid, ee = item >> 1, h = item & 1;
+    int rank = 0;
+    float v = 0.f;
+    if (ee < E) {
+      v = logits[ee];
+      const int j1 = h ? E : halfE;
+#pragma unroll 2
+      for (int j = h ? halfE : 0; j < j1; ++j) {
+        const float u = logits[j];
+        rank += (u > v) || (u == v && j < ee);
+      }
+    }
+    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
+    if (ee < E && h == 0) {
+      if (rank < K) M.ids[rank] = ee;
+      if (rank == 0) M.maxv = v;
+    }
+  }
+  __syncthreads();
+  if (tid < K && M.ids[tid] < 0) {  // non-finite logits: keep a valid index and flag the call
+    M.ids[tid] = tid;
+    atomicOr(err, kErrNonFinite);
+  }
+  const float mx = M.maxv;
+  float ps = 0.f;
+#pragma unroll 1
+  for (int ee = tid; ee < E; ee += kFT) ps += __expf(logits[ee] - mx);
+  ps = warp_sum(ps);
+  if (lane == 0) M.wsum[warp] = ps;
+  __syncthreads();
+  if (tid < K) M.pe[tid] = __expf(logits[M.ids[tid]] - mx);
+  __syncthreads();
+  if (tid < K) {
+    float denom = 0.f;
+    if (renorm) {
+      for (int j = 0; j < K; ++j) denom += M.pe[j];
+    } else {
+      for (int w = 0; w < kFW; ++w) denom += M.wsum[w];
+    }
+    M.w[tid] = __fdividef(M.pe[tid], denom);
+  }
+  __syncthreads();
+}
+
+// Exact top-k of the I channel scores (keys = float bits) into sel[0..k), ascending.
+__device__ __noinline__ void select_channels(const uint32_t* keys, int I, int k, uint16_t* sel,
+                                             Misc& M) {
+  uint32_t kth, need;
+  radix_kth_smem<kFT>(keys, I, k, M.hist, M.info, &kth, &need);
+  scatter_topk<kFT>(keys, I, kth, need, sel, M.scan);
+  __syncthreads();
+}
+
+// Sketch scores of this CTA's nt row tiles: warp w takes chunks [kc0, kc1) of every
+// tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B.
+// Partial sums go to part[warp][tile*16 + row].
+__device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm, int nt, int KC,
+                                         float* part_w) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kc0 = warp * KC / kFW, kc1 = (warp + 1) * KC / kFW;
+  const int g = lane >> 2, c = lane & 3;
+  const uint4* xp = xperm + c * 2;
+#pragma unroll 1
+  for (int tl = 0; tl < nt; ++tl) {
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 2
+    for (int kc = kc0; kc < kc1; ++kc) {
+      const uint2 w = codes[((size_t)tl * KC + kc) * 32 + lane];
+      uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
+      if (g == 0) { xa = xp[kc * 8]; xb = xp[kc * 8 + 1]; }
+      // four independent 16-column steps (no accumulator chain between them)
+      float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
+      float m2[4] = {0.f, 0.f, 0.f, 0.f}, m3[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_bf16(m0, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
+               (w.y << 2) & kSketchMask, xa.x, xa.y);
+      mma_bf16(m1, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
+               (w.y << 6) & kSketchMask, xa.z, xa.w);
+      mma_bf16(m2, (w.x << 8) & kSketchMask, (w.y << 8) & kSketchMask, (w.x << 10) & kSketchMask,
+               (w.y << 10) & kSketchMask, xb.x, xb.y);
+      mma_bf16(m3, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask, (w.x << 14) & kSketchMask,
+               (w.y << 14) & kSketchMask, xb.z, xb.w);
+      acc0 += (m0[0] + m1[0]) + (m2[0] + m3[0]);
+      acc1 += (m0[2] + m1[2]) + (m2[2] + m3[2]);
+    }
+    if (c == 0) {
+      part_w[tl * kRowTile + g] = acc0;
+      part_w[tl * kRowTile + g + 8] = acc1;
+    }
+  }
+}
+
+// One warp per channel: h = silu(gate . x) * (up . x) for channel record `rec`.
+__device__ __forceinline__ float channel_h(const uint16_t* rec, const uint16_t* xs, int d) {
+  const int lane = threadIdx.x & 31;
+  const uint4* gr = reinterpret_cast<const uint4*>(rec);
+  const uint4* ur = reinterpret_cast<const uint4*>(rec + d);
+  const uint4* xr = reinterpret_cast<const uint4*>(xs);
+  float g = 0.f, u = 0.f;
+#pragma unroll 2
+  for (int i = lane; i < d / 8; i += 32) {
+    const uint4 xv = xr[i];
+    g = dot8(gr[i], xv, g);
+    u = dot8(ur[i], xv, u);
+  }
+  g = warp_sum(g);
+  u = warp_sum(u);
+  return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
 __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_constant__ FusedParams P) {
   extern __shared__ __align__(128) uint8_t sm[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -97,103 +234,80 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   const int KC = d / kColChunk;
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm + P.o_x);
+  uint32_t* xperm = reinterpret_cast<uint32_t*>(sm + P.o_xperm);
   float* logits = reinterpret_cast<float*>(sm + P.o_logits);
-  float* scores = reinterpret_cast<float*>(sm + P.o_scores);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + P.o_keys);  // channel scores (float bits)
   float* alpha_s = reinterpret_cast<float*>(sm + P.o_alpha);
   float* zs = reinterpret_cast<float*>(sm + P.o_z);
   uint16_t* sel = reinterpret_cast<uint16_t*>(sm + P.o_sel);
   float* part = reinterpret_cast<float*>(sm + P.o_part);
-  float* ybuf = reinterpret_cast<float*>(sm + P.o_ybuf);
-  uint16_t* aslice = reinterpret_cast<uint16_t*>(sm + P.o_aslice);
+  float* ylr = reinterpret_cast<float*>(sm + P.o_ylr);     // A_e z on this CTA's slice
   Misc& M = *reinterpret_cast<Misc*>(sm + P.o_misc);
   uint8_t* big = sm + P.o_big;
+  float* ybuf = reinterpret_cast<float*>(big);             // phase D: partial output (over the ring)
 
-  // Every CTA of the cluster must be running before any DSMEM store targets it:
-  // arrive now, wait just before the first remote store (overlaps the loads).
+  // Every CTA of the cluster must be running before any DSMEM access targets it:
+  // arrive now, wait just before the first remote access.
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
-  // ------------------------------------------------------------------ phase A: router
+  // ------------------------------------------------------------------ prologue (weights only)
   const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
+  const uint32_t rbytes = (uint32_t)(e_hi - e_lo) * 2u * d;
   if (tid == 0) {
+#pragma unroll 1
     for (int i = 0; i < 2 + P.ring; ++i) mbar_init(&M.bar[i], 1);
     fence_mbar_init();
-    const uint32_t rbytes = (uint32_t)(e_hi - e_lo) * 2u * d;
-    mbar_arrive_expect_tx(&M.bar[0], 2u * d + rbytes);
-    bulk_g2s(xs, P.x, 2u * d, &M.bar[0]);
+    mbar_arrive_expect_tx(&M.bar[0], rbytes);
     if (rbytes) bulk_g2s(big, P.router_t + (size_t)e_lo * d, rbytes, &M.bar[0]);
-    M.ok = 1;
   }
+#pragma unroll 1
+  for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
+  // x and the workspace may be written by the previous launch: wait for it here.
+  pdl_wait();
+#pragma unroll 1
+  for (int i = tid; i < d / 8; i += kFT)
+    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
   __syncthreads();
-  bool ok = mbar_wait(&M.bar[0], 0, P.err);
+  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
+#pragma unroll 1
+  for (int i = tid; i < d / 2; i += kFT) {
+    const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
+    xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
+  }
+
+  // ------------------------------------------------------------------ phase A: router
+  bool ok = wait_phase(&M.bar[0], 0, P.err);
   ok = __syncthreads_and(ok);
   asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
   if (ok) {
     const uint16_t* rows = reinterpret_cast<const uint16_t*>(big);
+#pragma unroll 1
     for (int row = warp; row < e_hi - e_lo; row += kFW) {
       const uint4* wr = reinterpret_cast<const uint4*>(rows + (size_t)row * d);
       const uint4* xr = reinterpret_cast<const uint4*>(xs);
       float acc = 0.f;
+#pragma unroll 2
       for (int i = lane; i < d / 8; i += 32) acc = dot8(wr[i], xr[i], acc);
       acc = warp_sum(acc);
-      store_cluster(cluster, logits, e_lo + row, acc, lane, CS);
+      if (lane < CS) cluster.map_shared_rank(logits, lane)[e_lo + row] = acc;
     }
   }
   cluster.sync();
-  if (warp == 0) {
-    constexpr int MAXM = MSB_MAX_EXPERTS / 32;
-    float v[MAXM];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m) {
-      const int ee = lane + 32 * m;
-      v[m] = ee < E ? logits[ee] : -INFINITY;
-      mx = fmaxf(mx, v[m]);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float sum = 0.f;
-#pragma unroll
-    for (int m = 0; m < MAXM; ++m)
-      if (lane + 32 * m < E) sum += expf(v[m] - mx);
-    sum = warp_sum(sum);
-    uint32_t taken = 0;
-    float psum = 0.f;
-    for (int rr = 0; rr < K; ++rr) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int m = 0; m < MAXM; ++m) {
-        const int ee = lane + 32 * m;
-        if (ee < E && !((taken >> m) & 1u) && (v[m] > bv || (v[m] == bv && ee < bi))) {
-          bv = v[m];
-          bi = ee;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if (bi >= E) {  // non-finite logits: keep a valid index and flag the call
-        bi = rr;
-        bv = mx;
-        if (lane == 0) atomicOr(P.err, kErrNonFinite);
-      }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      const float pe = expf(bv - mx);
-      psum += pe;
-      if (lane == 0) { M.ids[rr] = bi; M.w[rr] = pe; }
-    }
-    __syncwarp();
-    if (lane < K) M.w[lane] = M.w[lane] / (D.renorm ? psum : sum);
-  }
-  __syncthreads();
+  router_topk(logits, E, K, D.renorm, M, P.err);
   const int e = M.ids[rc];
   const float we = M.w[rc];
-  if (blockIdx.x == 0 && tid < K) {
-    if (P.tr.expert_ids) P.tr.expert_ids[tid] = M.ids[tid];
-    if (P.tr.expert_w) P.tr.expert_w[tid] = M.w[tid];
+  if (blockIdx.x == 0) {
+    if (tid < K) {
+      if (P.tr.expert_ids) P.tr.expert_ids[tid] = M.ids[tid];
+      if (P.tr.expert_w) P.tr.expert_w[tid] = M.w[tid];
+    }
+    if (P.tr.union_count)
+#pragma unroll 1
+      for (int i = tid; i < E; i += kFT) {
+        int c = 0;
+        for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? P.k : c;
+        P.tr.union_count[i] = c;
+      }
   }
 
   // ------------------------------------------------------------------ phase B: scores, z
@@ -201,11 +315,12 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   const int lt0 = min(ntile_all, q * P.tpc), lt1 = min(ntile_all, lt0 + P.tpc);
   const int nt = lt1 - lt0;
   const uint32_t code_bytes = P.dense ? 0u : (uint32_t)nt * KC * kChunkWords * 4u;
-  int nz = 0;
-  for (int rho = q; rho < r; rho += CS) ++nz;
+  const int nz = r > q ? (r - q + CS - 1) / CS : 0;  // z rows q, q+CS, ... below r
+  const bool lr_out = (half == 0 && r > 0);
+  uint16_t* brows = reinterpret_cast<uint16_t*>(big + code_bytes);
+  uint16_t* aslice = reinterpret_cast<uint16_t*>(big + P.o_aslice_off);
   if (tid == 0 && ok) {
     uint32_t bytes = code_bytes + (P.dense ? 0u : (uint32_t)nt * kRowTile * 4u) + (uint32_t)nz * 2u * d;
-    const bool lr_out = (half == 0 && r > 0);
     if (lr_out) bytes += (uint32_t)P.slice * r * 2u;
     fence_proxy_async();
     mbar_arrive_expect_tx(&M.bar[1], bytes);
@@ -214,122 +329,57 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
       bulk_g2s(alpha_s, P.alpha + (size_t)e * ipad + (size_t)lt0 * kRowTile, nt * kRowTile * 4u,
                &M.bar[1]);
     }
-    uint16_t* brows = reinterpret_cast<uint16_t*>(big + code_bytes);
-    int i = 0;
-    for (int rho = q; rho < r; rho += CS, ++i)
-      bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + rho) * d, 2u * d, &M.bar[1]);
+#pragma unroll 1
+    for (int i = 0; i < nz; ++i)
+      bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[1]);
     if (lr_out)
       bulk_g2s(aslice, P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, (uint32_t)P.slice * r * 2u,
                &M.bar[1]);
   }
-  for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
-  __syncthreads();
-  ok = ok && mbar_wait(&M.bar[1], 0, P.err);
+  ok = ok && wait_phase(&M.bar[1], 0, P.err);
   ok = __syncthreads_and(ok);
-  if (ok && !P.dense && nt > 0) {
-    // items (tile, chunk) in tile-major order; warp w takes a contiguous range
-    const int nitems = nt * KC;
-    const int i0 = warp * nitems / kFW, i1 = (warp + 1) * nitems / kFW;
-    const uint2* codes = reinterpret_cast<const uint2*>(big);
-    const uint32_t* x32 = reinterpret_cast<const uint32_t*>(xs);
-    const int g = lane >> 2, c = lane & 3;
-    int cur = -1;
-    float acc0 = 0.f, acc1 = 0.f;
-    for (int it = i0; it < i1; ++it) {
-      const int tl = it / KC, kc = it - tl * KC;
-      if (tl != cur) {
-        if (cur >= 0 && c == 0) {
-          part[warp * P.tpc * kRowTile + cur * kRowTile + g] = acc0;
-          part[warp * P.tpc * kRowTile + cur * kRowTile + g + 8] = acc1;
-        }
-        cur = tl;
-        acc0 = acc1 = 0.f;
-      }
-      const uint2 w = codes[(size_t)it * 32 + lane];
-      uint32_t b[8];
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        b[2 * s] = g == 0 ? x32[kc * 32 + 8 * s + c] : 0u;
-        b[2 * s + 1] = g == 0 ? x32[kc * 32 + 8 * s + c + 4] : 0u;
-      }
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_bf16(a4, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
-               (w.y << 2) & kSketchMask, b[0], b[1]);
-      mma_bf16(a4, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
-               (w.y << 6) & kSketchMask, b[2], b[3]);
-      mma_bf16(a4, (w.x << 8) & kSketchMask, (w.y << 8) & kSketchMask, (w.x << 10) & kSketchMask,
-               (w.y << 10) & kSketchMask, b[4], b[5]);
-      mma_bf16(a4, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask, (w.x << 14) & kSketchMask,
-               (w.y << 14) & kSketchMask, b[6], b[7]);
-      acc0 += a4[0];
-      acc1 += a4[2];
-    }
-    if (cur >= 0 && c == 0) {
-      part[warp * P.tpc * kRowTile + cur * kRowTile + g] = acc0;
-      part[warp * P.tpc * kRowTile + cur * kRowTile + g + 8] = acc1;
-    }
-  }
+  if (ok && !P.dense && nt > 0)
+    score_tiles(reinterpret_cast<const uint2*>(big), reinterpret_cast<const uint4*>(xperm), nt, KC,
+                part + warp * P.tpc * kRowTile);
   // z rows: z[rho] = B_e[rho] . x, broadcast to the cluster
   if (ok && r > 0) {
-    const uint16_t* brows = reinterpret_cast<const uint16_t*>(big + code_bytes);
+#pragma unroll 1
     for (int i = warp; i < nz; i += kFW) {
       const uint4* br = reinterpret_cast<const uint4*>(brows + (size_t)i * d);
       const uint4* xr = reinterpret_cast<const uint4*>(xs);
       float acc = 0.f;
+#pragma unroll 2
       for (int j = lane; j < d / 8; j += 32) acc = dot8(br[j], xr[j], acc);
       acc = warp_sum(acc);
-      store_cluster(cluster, zs, q + i * CS, acc, lane, CS);
+      if (lane < CS) cluster.map_shared_rank(zs, lane)[q + i * CS] = acc;
     }
   }
   __syncthreads();
   if (ok && !P.dense) {
-    for (int lr = tid; lr < nt * kRowTile; lr += kFT) {
-      float s = 0.f;
+    // score = alpha * |sum of the 8 warps' partials| / 2, broadcast to every CTA
+    const int nrows = nt * kRowTile;
+#pragma unroll 1
+    for (int i = tid; i < nrows * CS; i += kFT) {
+      const int lr = i % nrows, dst = i / nrows;
+      float sc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFW; ++w) s += part[w * P.tpc * kRowTile + lr];
-      s = alpha_s[lr] * fabsf(s) * 0.5f;
+      for (int w = 0; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + lr];
+      sc = alpha_s[lr] * fabsf(sc) * 0.5f;
       const int row = lt0 * kRowTile + lr;
-      for (int dst = 0; dst < CS; ++dst) cluster.map_shared_rank(scores, dst)[row] = s;
-      if (half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + row] = s;
+      cluster.map_shared_rank(keys, dst)[row] = __float_as_uint(sc);
+      if (dst == 0 && half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + row] = sc;
     }
   }
   cluster.sync();
+  pdl_trigger();  // the next launch may start its weight-only prologue
 
   // ------------------------------------------------------------------ phase C: top-k, records
-  if (!P.dense) {
-    constexpr int EPT = MSB_MAX_INTER / kFT;
-    const int ept = (I + kFT - 1) / kFT;
-    const int j0 = tid * ept;
-    uint32_t key[EPT];
-    uint32_t valid = 0;
-#pragma unroll
-    for (int m = 0; m < EPT; ++m) {
-      key[m] = 0;
-      if (m < ept && j0 + m < I) { key[m] = __float_as_uint(scores[j0 + m]); valid |= 1u << m; }
-    }
-    uint32_t kth, need;
-    radix_kth<kFT, EPT>(key, valid, P.k, M.hist, M.info, &kth, &need);
-    uint32_t ngt = 0, neq = 0;
-#pragma unroll
-    for (int m = 0; m < EPT; ++m)
-      if ((valid >> m) & 1u) { ngt += key[m] > kth; neq += key[m] == kth; }
-    uint32_t tot;
-    const uint32_t pre = block_excl_scan<kFT>(ngt | (neq << 16), M.scan, &tot);
-    uint32_t gtb = pre & 0xffffu, eqb = pre >> 16;
-#pragma unroll
-    for (int m = 0; m < EPT; ++m) {
-      if (!((valid >> m) & 1u)) continue;
-      const bool gt = key[m] > kth, eq = key[m] == kth;
-      if (gt || (eq && eqb < need)) sel[gtb + min(eqb, need)] = (uint16_t)(j0 + m);
-      gtb += gt;
-      eqb += eq;
-    }
-    __syncthreads();
-    if (half == 0 && q == 0) {
-      for (int i = tid; i < P.k; i += kFT)
-        if (P.tr.sel) P.tr.sel[(size_t)rc * P.k + i] = sel[i];
-      if (tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
-    }
+  if (!P.dense) select_channels(keys, I, P.k, sel, M);
+  if (!P.dense && half == 0 && q == 0) {
+    if (P.tr.sel)
+#pragma unroll 1
+      for (int i = tid; i < P.k; i += kFT) P.tr.sel[(size_t)rc * P.k + i] = sel[i];
+    if (tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
   }
   // this CTA's share of the k channels
   const int NQ = CS * P.cpe, gq = half * CS + q;
@@ -339,105 +389,54 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   uint16_t* ring = reinterpret_cast<uint16_t*>(big);
   if (tid == 0 && ok) {
     fence_proxy_async();
-    for (int i = 0; i < min(P.ring, nmine); ++i) {
+    const int first = min(P.ring, nmine);
+#pragma unroll 1
+    for (int i = 0; i < first; ++i) {
       const int ch = P.dense ? c0 + i : (int)sel[c0 + i];
       mbar_arrive_expect_tx(&M.bar[2 + i], rec_bytes);
       bulk_g2s(ring + (size_t)i * 3 * d, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
                &M.bar[2 + i]);
     }
   }
-  // x in registers: thread owns elements (it*kFT + tid)*8 .. +8
-  constexpr int ITM = MSB_MAX_D / (kFT * 8);
-  const int IT = (d + kFT * 8 - 1) / (kFT * 8);
-  float y[ITM][8];
-  float xf[ITM][8];
-#pragma unroll
-  for (int it = 0; it < ITM; ++it) {
-    const int el = (it * kFT + tid) * 8;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) { y[it][i] = 0.f; xf[it][i] = 0.f; }
-    if (it < IT && el < d) {
-      const uint4 xv = *reinterpret_cast<const uint4*>(xs + el);
-      xf[it][0] = bf16_lo(xv.x); xf[it][1] = bf16_hi(xv.x);
-      xf[it][2] = bf16_lo(xv.y); xf[it][3] = bf16_hi(xv.y);
-      xf[it][4] = bf16_lo(xv.z); xf[it][5] = bf16_hi(xv.z);
-      xf[it][6] = bf16_lo(xv.w); xf[it][7] = bf16_hi(xv.w);
+  // A_e z on this CTA's output slice, while the first records are in flight
+  if (ok && lr_out) {
+#pragma unroll 1
+    for (int i = tid; i < P.slice; i += kFT) {
+      const uint16_t* arow = aslice + (size_t)i * r;
+      float acc = 0.f;
+#pragma unroll 1
+      for (int rho = 0; rho < r; ++rho) acc = fmaf(bf16_lo(arow[rho]), zs[rho], acc);
+      ylr[i] = acc;
     }
   }
-  __syncthreads();
+  float y[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
+#pragma unroll 1
   for (int g0 = 0; g0 < nmine; g0 += P.group) {
     const int ng = min(P.group, nmine - g0);
-    bool okw = true;
-    for (int i = 0; i < ng; ++i) {
-      const int ci = g0 + i;
-      okw = okw && (!ok || mbar_wait(&M.bar[2 + ci % P.ring], (ci / P.ring) & 1u, P.err));
+    // warp w computes h of channel g0 + w once its record has landed
+    if (warp < ng) {
+      const int ci = g0 + warp;
+      const bool okw = ok && wait_phase(&M.bar[2 + ci % P.ring], (ci / P.ring) & 1u, P.err);
+      float hv = 0.f;
+      if (okw) hv = channel_h(ring + (size_t)(ci % P.ring) * 3 * d, xs, d);
+      if (lane == 0) M.h[warp] = hv;
+      if (!okw && lane == 0) M.h[warp] = 0.f;
     }
-    ok = __syncthreads_and(ok && okw);
-    float v[2 * kGroup];
-#pragma unroll
-    for (int i = 0; i < 2 * kGroup; ++i) v[i] = 0.f;
+    ok = __syncthreads_and(ok);
     if (ok) {
-#pragma unroll
-      for (int i = 0; i < kGroup; ++i) {
-        if (i < ng) {
-          const uint16_t* rec = ring + (size_t)((g0 + i) % P.ring) * 3 * d;
-#pragma unroll
-          for (int it = 0; it < ITM; ++it) {
-            const int el = (it * kFT + tid) * 8;
-            if (it < IT && el < d) {
-              v[i] = dot8f(*reinterpret_cast<const uint4*>(rec + el), xf[it], v[i]);
-              v[kGroup + i] = dot8f(*reinterpret_cast<const uint4*>(rec + d + el), xf[it], v[kGroup + i]);
-            }
-          }
-        }
-      }
-    }
-    // transpose-reduce 16 values across the warp: lane pair (2m, 2m+1) ends with value m
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool up = lane & 16;
-      const float send = up ? v[i] : v[i + 8];
-      const float keep = up ? v[i + 8] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const bool up = lane & 8;
-      const float send = up ? v[i] : v[i + 4];
-      const float keep = up ? v[i + 4] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const bool up = lane & 4;
-      const float send = up ? v[i] : v[i + 2];
-      const float keep = up ? v[i + 2] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    {
-      const bool up = lane & 2;
-      const float send = up ? v[0] : v[1];
-      const float keep = up ? v[1] : v[0];
-      v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
-    }
-    v[0] += __shfl_xor_sync(0xffffffffu, v[0], 1);
-    if ((lane & 1) == 0) M.red[warp][lane >> 1] = v[0];
-    __syncthreads();
-    if (tid < ng) {
-      float gs = 0.f, us = 0.f;
-#pragma unroll
-      for (int w = 0; w < kFW; ++w) { gs += M.red[w][tid]; us += M.red[w][kGroup + tid]; }
-      M.h[tid] = silu(gs) * us;
-    }
-    __syncthreads();
-    if (ok) {
+      // y += h_i * down_i over this thread's elements
+#pragma unroll 1
       for (int i = 0; i < ng; ++i) {
         const uint16_t* rec = ring + (size_t)((g0 + i) % P.ring) * 3 * d + 2 * d;
         const float h = M.h[i];
 #pragma unroll
-        for (int it = 0; it < ITM; ++it) {
+        for (int it = 0; it < IT; ++it) {
           const int el = (it * kFT + tid) * 8;
-          if (it < IT && el < d) {
+          if (el < d) {
             const uint4 dv = *reinterpret_cast<const uint4*>(rec + el);
             y[it][0] = fmaf(h, bf16_lo(dv.x), y[it][0]);
             y[it][1] = fmaf(h, bf16_hi(dv.x), y[it][1]);
@@ -455,6 +454,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     // refill the slots just consumed
     if (tid == 0 && ok) {
       fence_proxy_async();
+#pragma unroll 1
       for (int i = g0; i < g0 + ng; ++i) {
         const int nx = i + P.ring;
         if (nx < nmine) {
@@ -469,43 +469,47 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   }
 
   // ------------------------------------------------------------------ phase D: reduce, combine
+  // partial output to this CTA's shared buffer; each owner then sums its slice over
+  // the cluster with 16-byte DSMEM loads
 #pragma unroll
-  for (int it = 0; it < ITM; ++it) {
+  for (int it = 0; it < IT; ++it) {
     const int el = (it * kFT + tid) * 8;
-    if (it < IT && el < d) {
+    if (el < d) {
       *reinterpret_cast<float4*>(ybuf + el) = make_float4(y[it][0], y[it][1], y[it][2], y[it][3]);
       *reinterpret_cast<float4*>(ybuf + el + 4) = make_float4(y[it][4], y[it][5], y[it][6], y[it][7]);
     }
   }
   cluster.sync();
   if (ok) {
-    for (int i = tid; i < P.slice; i += kFT) {
-      const int el = q * P.slice + i;
-      float acc = 0.f;
-      for (int j = 0; j < CS; ++j) acc += cluster.map_shared_rank(ybuf, j)[el];
-      if (half == 0 && r > 0) {
-        const uint16_t* ar = aslice + (size_t)i * r;
-        for (int rho = 0; rho < r; ++rho) acc = fmaf(bf16_lo(ar[rho]), zs[rho], acc);
+#pragma unroll 1
+    for (int j = tid; j < P.slice / 4; j += kFT) {
+      const int el = q * P.slice + 4 * j;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int src = 0; src < CS; ++src) {
+        const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ybuf, src) + el);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      atomicAdd(P.y_acc + el, we * acc);
+      if (lr_out) {
+        acc.x += ylr[4 * j]; acc.y += ylr[4 * j + 1]; acc.z += ylr[4 * j + 2]; acc.w += ylr[4 * j + 3];
+      }
+      red_add_v4(P.y_acc + el, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
     }
   }
+  cluster.sync();  // no CTA leaves while its buffer may still be read
   __threadfence();
-  cluster.sync();
-  if (tid == 0) M.last = (atomicAdd(P.counter, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (tid == 0) M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K * P.cpe - 1));
   __syncthreads();
   if (M.last) {
+    // every contribution to this slice has arrived: convert, re-zero, reset
     __threadfence();
-    for (int i = tid; i < d; i += kFT) {
-      const float v = atomicExch(P.y_acc + i, 0.f);
-      P.out[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+#pragma unroll 1
+    for (int i = tid; i < P.slice; i += kFT) {
+      const float v = atomicExch(P.y_acc + q * P.slice + i, 0.f);
+      P.out[q * P.slice + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
-    if (P.tr.union_count) {
-      for (int i = tid; i < E; i += kFT) P.tr.union_count[i] = 0;
-      __syncthreads();
-      if (tid < K) P.tr.union_count[M.ids[tid]] = P.k;
-    }
-    if (tid == 0) *P.counter = 0u;
+    if (tid == 0) P.slice_cnt[q] = 0u;
   }
 }
 
@@ -525,9 +529,19 @@ int cur_dev() {
 
 int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
-// Fill the carve-up for cluster size cs; returns false if it does not fit.
-bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe) {
+using KernelFn = void (*)(FusedParams);
+
+KernelFn kernel_for(int d) {
+  const int it = (d + 2047) / 2048;
+  if (it <= 1) return fused_block_kernel<1>;
+  if (it <= 2) return fused_block_kernel<2>;
+  return fused_block_kernel<4>;
+}
+
+// Fill the carve-up for cluster size cs within `limit` bytes of shared memory.
+bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe, int limit) {
   const int d = D.d, E = D.experts, ipad = D.ipad, r = D.rank;
+  if (d % (8 * cs) != 0) return false;
   P.cs = cs;
   P.cpe = cpe;
   P.rpc = (E + cs - 1) / cs;
@@ -536,77 +550,92 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe) {
   P.slice = d / cs;
   int o = 0;
   P.o_x = o;      o = align_up(o + 2 * d, 128);
+  P.o_xperm = o;  o = align_up(o + 2 * d, 128);
   P.o_logits = o; o = align_up(o + 4 * E, 128);
-  P.o_scores = o; o = align_up(o + 4 * ipad, 128);
+  P.o_keys = o;   o = align_up(o + 4 * ipad, 128);
   P.o_alpha = o;  o = align_up(o + 4 * P.tpc * kRowTile, 128);
   P.o_z = o;      o = align_up(o + 4 * (r > 0 ? r : 1), 128);
   P.o_sel = o;    o = align_up(o + 2 * ipad, 128);
   P.o_part = o;   o = align_up(o + 4 * kFW * P.tpc * kRowTile, 128);
-  P.o_ybuf = o;   o = align_up(o + 4 * d, 128);
-  P.o_aslice = o; o = align_up(o + 2 * P.slice * (r > 0 ? r : 0), 128);
+  P.o_ylr = o;    o = align_up(o + 4 * P.slice, 128);
   P.o_misc = o;   o = align_up(o + (int)sizeof(Misc), 128);
   P.o_big = o;
-  const int avail = kSmemMax - o;
+  // big, in time order: phase A router rows | phase B sketch tiles + B_e rows |
+  // phase C record ring | phase D partial output (d floats, over the drained ring);
+  // this CTA's A_e rows sit past all of them (loaded in phase B, read in phase C).
+  const int aslice_bytes = align_up(P.slice * r * 2, 128);
+  const int avail = limit - o - aslice_bytes;
   const int need_a = P.rpc * 2 * d;
   const int need_b = (P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4) + P.zpc * 2 * d;
+  const int need_d = 4 * d;
   const int rec = 6 * d;
   int ring = avail / rec;
   if (ring > kRingMax) ring = kRingMax;
-  if (ring < 2 || need_a > avail || need_b > avail) return false;
+  if (ring < 2 || need_a > avail || need_b > avail || need_d > avail) return false;
+  const int per_cta = (k + cs * cpe - 1) / (cs * cpe);  // channels a CTA reads
+  if (ring > per_cta) ring = per_cta < 2 ? 2 : per_cta;
   P.ring = ring;
-  P.group = ring < kGroup ? ring : kGroup;
+  P.group = ring < kFW ? ring : kFW;  // one warp per channel of a group
+  if (P.group > 4 && ring < per_cta) P.group = 4;  // refill sooner when the ring is short
   int big = ring * rec;
   if (need_a > big) big = need_a;
   if (need_b > big) big = need_b;
-  P.smem = o + big;
-  return P.smem <= kSmemMax;
+  if (need_d > big) big = need_d;
+  P.o_aslice_off = big;
+  P.smem = o + big + aslice_bytes;
+  return P.smem <= limit;
 }
 
-// Prefer one 16-CTA cluster per routed expert when K of them are resident at once,
-// else two 8-CTA clusters per expert when 2K are; otherwise whichever shape can be
-// resident at all (clusters that do not fit wait for a free GPC: correct, slower).
+// Prefer plans whose CTAs can pair on an SM (all clusters then fit the GPCs), then
+// one 16-CTA cluster per routed expert when all K are resident, then two 8-CTA
+// clusters per expert; otherwise any plan (non-resident clusters run later).
 bool choose(FusedParams& P, const Dims& D, int k) {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64 || !g_ready[dev]) return false;
-  const bool ok16 = D.d % (8 * 16) == 0 && g_max_clusters16[dev] >= 1;
-  const bool ok8 = D.d % (8 * 8) == 0 && g_max_clusters8[dev] >= 1;
-  if (ok16 && g_max_clusters16[dev] >= D.top_e && plan(P, D, k, 16, 1)) return true;
-  if (ok8 && g_max_clusters8[dev] >= 2 * D.top_e && plan(P, D, k, 8, 2)) return true;
-  if (ok16 && plan(P, D, k, 16, 1)) return true;
-  if (ok8 && plan(P, D, k, 8, 2)) return true;
+  const int K = D.top_e;
+  const bool have16 = g_max_clusters16[dev] >= 1, have8 = g_max_clusters8[dev] >= 1;
+  if (have16 && plan(P, D, k, 16, 1, kSmemPair)) return true;
+  if (have8 && plan(P, D, k, 8, 2, kSmemPair)) return true;
+  if (have16 && g_max_clusters16[dev] >= K && plan(P, D, k, 16, 1, kSmemMax)) return true;
+  if (have8 && g_max_clusters8[dev] >= 2 * K && plan(P, D, k, 8, 2, kSmemMax)) return true;
+  if (have16 && plan(P, D, k, 16, 1, kSmemMax)) return true;
+  if (have8 && plan(P, D, k, 8, 2, kSmemMax)) return true;
   return false;
+}
+
+int query_clusters(KernelFn fn, int cs, int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs * 16, 1, 1);
+  cfg.blockDim = dim3(kFT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  return n;
 }
 }  // namespace
 
 int fused_setup() {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64) return MSB_ECUDA;
-  if (cudaFuncSetAttribute(fused_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kSmemMax) != cudaSuccess)
-    return MSB_ECUDA;
-  if (cudaFuncSetAttribute(fused_block_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
-      cudaSuccess) {
-    cudaGetLastError();
-  }
-  for (int cs : {16, 8}) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(cs * 16, 1, 1);
-    cfg.blockDim = dim3(kFT, 1, 1);
-    cfg.dynamicSmemBytes = kSmemMax;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, fused_block_kernel, &cfg) != cudaSuccess) {
+  for (KernelFn fn : {fused_block_kernel<1>, fused_block_kernel<2>, fused_block_kernel<4>}) {
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
+        cudaSuccess)
+      return MSB_ECUDA;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       cudaGetLastError();
-      n = 0;
-    }
-    (cs == 16 ? g_max_clusters16 : g_max_clusters8)[dev] = n;
   }
+  g_max_clusters16[dev] = query_clusters(fused_block_kernel<1>, 16, kSmemMax);
+  g_max_clusters8[dev] = query_clusters(fused_block_kernel<1>, 8, kSmemMax);
   g_ready[dev] = true;
   return MSB_OK;
 }
@@ -615,6 +644,7 @@ void fused_plan_info(const Dims& D, int k, int* info) {
   FusedParams P{};
   P.dense = (k == D.inter);
   const int dev = cur_dev();
+  #pragma unroll 1
   for (int i = 0; i < 6; ++i) info[i] = 0;
   if (choose(P, D, k)) {
     info[0] = P.cs;
@@ -648,7 +678,7 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
   P.lr_b = lr_b;
   P.out = out;
   P.err = err;
-  P.counter = counters + kCntFused;
+  P.slice_cnt = counters + kCntFusedSlices;
   P.y_acc = y_acc;
   P.tr = tr;
   P.D = D;
@@ -660,14 +690,16 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
   cfg.blockDim = dim3(kFT, 1, 1);
   cfg.dynamicSmemBytes = P.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = P.cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, fused_block_kernel, P);
+  cfg.numAttrs = 2;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(D.d), P);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 

@@ -325,82 +325,53 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
 // =====================================================================================
 // exact top-k / threshold selection per (token, expert) pair
 // =====================================================================================
-constexpr int kSelEPT = MSB_MAX_INTER / kNT;  // 16 keys per thread at most
-
 __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau, Dims D,
                                                      Workspace ws, TraceDev tr) {
-  __shared__ uint32_t hist[256];
-  __shared__ uint32_t info[4];
-  __shared__ uint32_t scan_tmp[kNT / 32 + 1];
+  __shared__ uint32_t keys[MSB_MAX_INTER];
+  __shared__ uint16_t sel_s[MSB_MAX_INTER];
   __shared__ uint32_t words[MSB_MAX_INTER / 32];
+  __shared__ uint32_t hist[512];
+  __shared__ uint32_t info[2];
+  __shared__ uint32_t scan_tmp[kNT / 32 + 1];
+  __shared__ uint32_t s_count;
   const int p = blockIdx.x;
-  const int I = D.inter, ipad = D.ipad;
-  const int ept = (I + kNT - 1) / kNT;
-  const int j0 = threadIdx.x * ept;
-  uint32_t key[kSelEPT];
-  uint32_t valid = 0;
-#pragma unroll
-  for (int m = 0; m < kSelEPT; ++m) {
-    const int j = j0 + m;
-    key[m] = 0;
-    if (m < ept && j < I) {
-      key[m] = __float_as_uint(__ldcg(&ws.scores[(size_t)p * ipad + j]));
-      valid |= 1u << m;
-    }
+  const int I = D.inter, ipad = D.ipad, mw = mask_words(ipad);
+  for (int j = threadIdx.x; j < I; j += kNT)
+    keys[j] = __float_as_uint(__ldcg(&ws.scores[(size_t)p * ipad + j]));
+  for (int i = threadIdx.x; i < mw; i += kNT) words[i] = 0;
+  __syncthreads();
+  if (mode == 0) {
+    uint32_t kth, need;
+    radix_kth_smem<kNT>(keys, I, k, hist, info, &kth, &need);
+    scatter_topk<kNT>(keys, I, kth, need, sel_s, scan_tmp);
+    if (threadIdx.x == 0) s_count = (uint32_t)k;
+  } else {
+    const int ept = (I + kNT - 1) / kNT;
+    const int j0 = threadIdx.x * ept, j1 = min(I, j0 + ept);
+    uint32_t n = 0;
+    for (int j = j0; j < j1; ++j) n += __uint_as_float(keys[j]) > tau;
+    uint32_t tot;
+    uint32_t pos = block_excl_scan<kNT>(n, scan_tmp, &tot);
+    for (int j = j0; j < j1; ++j)
+      if (__uint_as_float(keys[j]) > tau) sel_s[pos++] = (uint16_t)j;
+    if (threadIdx.x == 0) s_count = tot;
   }
-  for (int i = threadIdx.x; i < mask_words(ipad); i += kNT) words[i] = 0;
-  uint32_t kth = 0, need = 0;
-  if (mode == 0) radix_kth<kNT, kSelEPT>(key, valid, k, hist, info, &kth, &need);
-  const uint32_t tau_bits = __float_as_uint(tau);
-  // flags per element; count gt / eq for the ordered scan
-  uint32_t ngt = 0, neq = 0;
-#pragma unroll
-  for (int m = 0; m < kSelEPT; ++m) {
-    if (!((valid >> m) & 1u)) continue;
-    if (mode == 0) {
-      ngt += key[m] > kth;
-      neq += key[m] == kth;
-    } else {
-      ngt += __uint_as_float(key[m]) > __uint_as_float(tau_bits);
-    }
-  }
-  uint32_t tot;
-  const uint32_t pre = block_excl_scan<kNT>(ngt | (neq << 16), scan_tmp, &tot);
-  uint32_t gt_before = pre & 0xffffu, eq_before = pre >> 16;
+  __syncthreads();
+  const int count = (int)s_count;
   const int t = ws.pair_tok[p];
   const int slot = ws.pair_slot[p];
   const int e = ws.slot_expert[slot];
   int r = 0;
   while (ws.ids[t * D.top_e + r] != e) ++r;
   const size_t trow = (size_t)t * D.top_e + r;
-#pragma unroll
-  for (int m = 0; m < kSelEPT; ++m) {
-    if (!((valid >> m) & 1u)) continue;
-    const int j = j0 + m;
-    bool take;
-    if (mode == 0) {
-      const bool gt = key[m] > kth, eq = key[m] == kth;
-      take = gt || (eq && eq_before < need);
-      const uint32_t pos = gt_before + min(eq_before, need);
-      if (take) {
-        ws.sel[(size_t)p * ipad + pos] = (uint16_t)j;
-        if (tr.sel) tr.sel[trow * k + pos] = (uint16_t)j;
-      }
-      gt_before += gt;
-      eq_before += eq;
-    } else {
-      take = __uint_as_float(key[m]) > __uint_as_float(tau_bits);
-      if (take) {
-        ws.sel[(size_t)p * ipad + gt_before] = (uint16_t)j;
-        if (tr.sel) tr.sel[trow * I + gt_before] = (uint16_t)j;
-      }
-      gt_before += take;
-    }
-    if (take) atomicOr(&words[j >> 5], 1u << (j & 31));
+  const int cap = mode == 0 ? k : I;
+  for (int i = threadIdx.x; i < count; i += kNT) {
+    const int j = sel_s[i];
+    ws.sel[(size_t)p * ipad + i] = (uint16_t)j;
+    if (tr.sel) tr.sel[trow * cap + i] = (uint16_t)j;
+    atomicOr(&words[j >> 5], 1u << (j & 31));
   }
   __syncthreads();
-  const int count = mode == 0 ? k : (int)(tot & 0xffffu);
-  const int mw = mask_words(ipad);
   for (int i = threadIdx.x; i < mw; i += kNT) {
     const uint32_t wv = words[i];
     ws.selmask[(size_t)p * mw + i] = wv;
