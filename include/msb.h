@@ -192,6 +192,31 @@ int32_t moe_sparse_block_threshold(const void* x, int32_t batch, const void* rou
                                    void* workspace, size_t workspace_bytes,
                                    const msb_trace* trace, void* stream);
 
+/* The batch-1 block for callers that cannot allocate device memory.  The source
+ * pages have no counterpart to this entry point: it serves callers that own no
+ * device allocator -- a plugin that its host framework hands only input and
+ * output buffers, or code running where a cudaMalloc would synchronise the
+ * device or is not permitted.  Such a caller passes only the inputs and the
+ * output; nothing else is allocated.
+ *
+ * Same arguments and result as moe_sparse_block with batch = 1 and no
+ * workspace.  The scratch (error word, arrival counters, a d-float FP32
+ * accumulator) is a static device array of the library, about 37 KB, held on
+ * every GPU that loads the library until the process exits.  Limits: d <=
+ * MSB_NOALLOC_MAX_D, and the shapes must fit the single-launch kernel; otherwise
+ * MSB_EUNSUPPORTED (argument errors give MSB_EINVAL, as for moe_sparse_block).
+ * The first call on a device looks up the array's device address (do that
+ * first call before any stream capture).  Every call clears the part of the
+ * array it uses on `stream` and then launches; all calls share the array, so
+ * calls that overlap on the GPU (unordered streams) race.  A bounded wait that
+ * ran out inside the kernel is not reported by this entry point (there is no
+ * workspace for msb_check to read); the output of such a call is undefined. */
+#define MSB_NOALLOC_MAX_D 8192
+int32_t moe_sparse_block_noalloc(const void* x, const void* router_t, const void* records,
+                                 const uint32_t* sketch, const float* alpha, int32_t k,
+                                 const void* lr_a, const void* lr_b, void* out,
+                                 const msb_dims* dims, const msb_trace* trace, void* stream);
+
 /* Stack glue between decode layers (attention omitted):
  *   h[t] += y[t]            (h float [batch][d], y bf16 [batch][d]; y may be NULL: no add)
  *   x_next[t] = BF16( h[t] / sqrt(mean(h[t]^2) + eps) )   (RMSNorm, unit weight)

@@ -11,6 +11,7 @@ from .block import (  # noqa: F401
     Workspace,
     calibrate_threshold,
     moe_sparse_block,
+    moe_sparse_block_noalloc,
     moe_sparse_block_threshold,
     pack,
     path_info,

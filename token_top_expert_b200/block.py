@@ -192,6 +192,26 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
     return out
 
 
+def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Trace | None = None,
+                             stream=None):
+    """The batch-1 block without a workspace (scratch is a static device array of
+    the library), for callers that cannot allocate device memory."""
+    import torch
+    dims = layer.dims
+    _act(x, dims)
+    if x.shape[0] != 1:
+        raise ValueError("moe_sparse_block_noalloc takes one token")
+    if out is None:
+        out = torch.empty_like(x)
+    tr = trace.c() if trace is not None else None
+    rc = _lib.load().moe_sparse_block_noalloc(
+        _ptr(x), _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch), _ptr(layer.alpha),
+        k, _ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out), ctypes.byref(dims.c()),
+        ctypes.byref(tr) if tr is not None else None, _stream(stream))
+    _check(rc, "moe_sparse_block_noalloc")
+    return out
+
+
 def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
                                workspace: Workspace | None = None, trace: Trace | None = None,
                                stream=None):
