@@ -213,6 +213,163 @@ def config_of(w, args):
             "parallelism": "replicas" if args.gpus > 1 else "single"}
 
 
+def run_stack(args, w, world, rank, local):
+    """Stacked decode: `layers` MoE blocks with per-layer seeded weights, pre-norm
+    residual glue (h <- h + MoE_l(BF16(RMSNorm(h)))), attention omitted.  A step is
+    one token (or batch) through every layer."""
+    import torch
+    import token_top_expert_b200 as msb
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    L = w.layers
+    B = args.batch
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
+    layers = []
+    t0 = time.time()
+    for l in range(L):
+        lw = synth.layer_weights(w, l)
+        pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
+        layers.append(msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev))
+        del lw, pk
+    setup_s = time.time() - t0
+    nseq = 16
+    h0 = torch.from_numpy(np.stack([synth.stack_initial_hidden(w, s, B) for s in range(nseq)])).to(dev)
+    h = torch.empty((B, w.d), dtype=torch.float32, device=dev)
+    xb = torch.empty((B, w.d), dtype=torch.bfloat16, device=dev)
+    yb = torch.empty_like(xb)
+    ws = msb.Workspace(dims, B, dev)
+    stream = torch.cuda.Stream(dev)
+    dense = args.k == w.inter
+
+    def step(s, trace=None):
+        h.copy_(h0[s % nseq])
+        for l in range(L):
+            msb.residual_rmsnorm(h, yb if l > 0 else None, xb, stream=stream)
+            msb.moe_sparse_block(xb, layers[l], args.k, out=yb, workspace=ws, trace=trace,
+                                 stream=stream)
+        msb.residual_rmsnorm(h, yb, xb, stream=stream)
+
+    # bytes of one step, from traced calls
+    tr = msb.Trace(dims, B, args.k)
+    byts = 0
+    with torch.cuda.stream(stream):
+        h.copy_(h0[0])
+        for l in range(L):
+            msb.residual_rmsnorm(h, yb if l > 0 else None, xb, stream=stream)
+            msb.moe_sparse_block(xb, layers[l], args.k, out=yb, workspace=ws, trace=tr, stream=stream)
+            stream.synchronize()
+            byts += algorithmic_bytes(w, args.k, args.rank, tr.union_count.cpu().tolist(), dense)
+        for i in range(args.warmup):
+            step(i)
+    stream.synchronize()
+    ws.check(stream)
+    G = min(nseq, args.steps)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i)
+    graph.replay()
+    stream.synchronize()
+    reps = max(1, args.steps // G)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(reps):
+                graph.replay()
+            e1.record(stream)
+        stream.synchronize()
+    ms = e0.elapsed_time(e1)
+    steps = reps * G
+    ms_per_step = ms / steps
+    peak, peak_kind = peaks()
+    achieved = byts / (ms_per_step * 1e-3) / 1e9
+    plan = msb.path_info(dims, B, args.k)
+    line = {
+        "metric": "stacked MoE decode tokens/s (%d layers)" % L, "value": steps * B / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (per-layer seeded BF16 weights; h0 ~ N(0,1))",
+        "config": dict(config_of(w, args), layers=L, path=plan,
+                       l2="inputs larger than L2: %.1f GB of packed weights" %
+                          (sum(x.nbytes() for x in layers) / 1e9)),
+        "us_per_layer": ms_per_step * 1e3 / L, "bytes_per_step": byts,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
+        "gpu_launches": steps * (2 * L + 1) * (1 if plan["path"] == "single_launch" else 5),
+        "clocks": clk.summary(), "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+
+
+def run_threshold(args, w, world, rank, local):
+    """The calibrated-threshold comparator on the same scores: tau is calibrated on
+    held-out tokens for the budget k/I, then the decode steps read whatever passes."""
+    import torch
+    import token_top_expert_b200 as msb
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B = args.batch
+    lw = synth.layer_weights(w)
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
+    layer = msb.PackedLayer.from_host(dims, msb.pack(lw.gate, lw.up, lw.down, lw.router, dims),
+                                      lw.lr_a, lw.lr_b, device=dev)
+    del lw
+    ws = msb.Workspace(dims, max(B, 8), dev)
+    # calibration: 256 held-out tokens, GPU scores of their routed experts
+    pooled = []
+    for i in range(32):
+        xc = torch.from_numpy(synth.calibration_activations(w, i, 8).view(np.int16)).to(dev).view(torch.bfloat16)
+        tr = msb.Trace(dims, 8, args.k, scores=True)
+        msb.moe_sparse_block(xc, layer, args.k, workspace=ws, trace=tr, general=True)
+        pooled.append(tr.scores[:, :, :w.inter].float().cpu().numpy().ravel())
+    tau = msb.calibrate_threshold(np.concatenate(pooled), args.k / w.inter)
+    nseq = 64
+    xs = torch.from_numpy(np.stack([synth.activations(w, s, batch=B) for s in range(nseq)]).view(np.int16)).to(dev).view(torch.bfloat16)
+    out = torch.empty_like(xs[0])
+    counts = []
+    byts = []
+    tr = msb.Trace(dims, B, args.k, threshold=True)
+    for s in range(nseq):
+        msb.moe_sparse_block_threshold(xs[s], layer, tau, out=out, workspace=ws, trace=tr)
+        torch.cuda.synchronize()
+        counts.append(tr.sel_count.cpu().numpy().ravel().copy())
+        byts.append(algorithmic_bytes(w, args.k, args.rank, tr.union_count.cpu().tolist(), False))
+    counts = np.concatenate(counts) / w.inter
+    stream = torch.cuda.Stream(dev)
+    with torch.cuda.stream(stream):
+        for s in range(args.warmup):
+            msb.moe_sparse_block_threshold(xs[s % nseq], layer, tau, out=out, workspace=ws, stream=stream)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for s in range(nseq):
+            msb.moe_sparse_block_threshold(xs[s], layer, tau, out=out, workspace=ws, stream=stream)
+    reps = max(1, args.steps // nseq)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        graph.replay()
+        e0.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / (reps * nseq)
+    line = {"metric": "threshold comparator: read fraction per (token, expert) and tokens/s",
+            "tau": tau, "budget": args.k / w.inter,
+            "read_fraction": {"mean": float(counts.mean()), "std": float(counts.std()),
+                              "min": float(counts.min()), "max": float(counts.max())},
+            "value": B / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms, "batch": B,
+            "bytes_per_step": float(np.mean(byts)), "config": config_of(w, args),
+            "data": "synthetic; tau from 256 held-out tokens (weights and routing as the bench)",
+            "note": "single weight replica (the comparator's read variance is the point)"}
+    print(json.dumps(line), flush=True)
+    del graph
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -227,6 +384,8 @@ def main():
     ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--threshold", action="store_true",
+                    help="measure the calibrated-threshold comparator instead of top-k")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     args.k = w.k if args.k is None else args.k
@@ -239,6 +398,14 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, world, rank)
+        return
+    if w.layers > 1 or args.threshold:
+        from token_top_expert_b200 import build as _bld
+        _bld.build()
+        if w.layers > 1:
+            run_stack(args, w, world, rank, local)
+        else:
+            run_threshold(args, w, world, rank, local)
         return
 
     import torch

@@ -95,6 +95,85 @@ __device__ __forceinline__ void radix_kth_smem(const uint32_t* keys, int n, int 
   *need = kk;
 }
 
+// Exact k-th largest of n <= 4096 non-negative float keys (bit patterns) in shared
+// memory, fast path: one counting pass over a 4096-bin histogram of the top 12 key
+// bits (hist must be zero on entry; the sign bit is 0), a block scan to find the
+// bin holding the k-th key, then the keys of that bin (usually a handful) are
+// gathered and ranked.  When that bin holds more than 64 keys (heavy ties) it
+// falls back to radix_kth_smem, reusing hist's first 512 words.  scratch: >= 200
+// words of shared memory.  Results are identical to radix_kth_smem's.
+template <int NT>
+__device__ __forceinline__ void hist_kth_smem(const uint32_t* keys, int n, int k, uint32_t* hist,
+                                              uint32_t* scratch, uint32_t* kth, uint32_t* need) {
+  const int tid = threadIdx.x;
+  if (tid == 0) scratch[66] = 0;  // candidate counter
+#pragma unroll 1
+  for (int j = tid; j < n; j += NT) atomicAdd(&hist[keys[j] >> 19], 1u);
+  __syncthreads();
+  // thread t owns the 4096/NT bins just below those of thread t-1 (thread 0: the top)
+  constexpr int PER = 4096 / NT;
+  static_assert(PER % 4 == 0, "bins per thread");
+  const int base = 4096 - PER * (tid + 1);
+  uint32_t c[PER];
+#pragma unroll
+  for (int i = 0; i < PER; i += 4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(hist + base + i);
+    c[i] = v.x; c[i + 1] = v.y; c[i + 2] = v.z; c[i + 3] = v.w;
+  }
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) local += c[i];
+  uint32_t total;
+  const uint32_t above = block_excl_scan<NT>(local, scratch, &total);
+  if (above < (uint32_t)k && (uint32_t)k <= above + local) {
+    uint32_t a = above;
+#pragma unroll
+    for (int i = PER - 1; i >= 0; --i) {
+      if (a < (uint32_t)k && (uint32_t)k <= a + c[i]) {
+        scratch[64] = (uint32_t)(base + i);  // the bin
+        scratch[65] = (uint32_t)k - a;       // rank of the k-th key inside the bin (1-based)
+        scratch[67] = c[i];                  // keys in the bin
+      }
+      a += c[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t bin = scratch[64], rem = scratch[65], cnt = scratch[67];
+  if (cnt > 64) {  // rare (heavy ties): exact fallback
+    __syncthreads();
+    radix_kth_smem<NT>(keys, n, k, hist, scratch + 68, kth, need);
+    return;
+  }
+  // gather the bin's keys (any order) with their indices
+  uint32_t* ck = scratch + 72;        // [64]
+  uint32_t* ci = scratch + 72 + 64;   // [64]
+#pragma unroll 1
+  for (int j = tid; j < n; j += NT) {
+    const uint32_t key = keys[j];
+    if ((key >> 19) == bin) {
+      const uint32_t slot = atomicAdd(&scratch[66], 1u);
+      ck[slot] = key;
+      ci[slot] = (uint32_t)j;
+    }
+  }
+  __syncthreads();
+  // rank inside the bin by (key desc, index asc); the k-th has rank rem - 1
+  if (tid < (int)cnt) {
+    const uint32_t mk = ck[tid], mi = ci[tid];
+    uint32_t rank = 0, gt = 0;
+#pragma unroll 4
+    for (int i = 0; i < (int)cnt; ++i) {
+      const uint32_t ok_ = ck[i], oi = ci[i];
+      rank += (ok_ > mk) || (ok_ == mk && oi < mi);
+      gt += ok_ > mk;
+    }
+    if (rank == rem - 1) { scratch[68] = mk; scratch[69] = rem - gt; }
+  }
+  __syncthreads();
+  *kth = scratch[68];
+  *need = scratch[69];
+}
+
 // Given the k-th key and how many of the equal keys to take, write the selected
 // indices (ascending) to sel[0..k).  Thread t owns the contiguous index range
 // [t*ept, (t+1)*ept).  Returns the number written by the block (== k).

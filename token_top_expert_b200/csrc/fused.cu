@@ -40,7 +40,8 @@ constexpr int kFW = kFT / 32;   // warps per CTA
 constexpr int kRingMax = 16;    // record slots
 constexpr int kGroup = 8;       // channels reduced together
 constexpr int kSmemMax = 227 * 1024;
-constexpr int kSmemPair = 110 * 1024;  // at or below this, two CTAs can share an SM
+constexpr int kSmemPair = 110 * 1024;  // fallback pairing limit if the device cannot be queried
+constexpr int kAregs = 8;              // register quads for the slice's A_e rows (8 bf16 each)
 
 struct FusedParams {
   const uint16_t* x;
@@ -64,8 +65,10 @@ struct FusedParams {
   int ring;    // record slots
   int group;   // channels per reduction group (<= ring)
   // shared-memory carve-up (byte offsets)
-  int o_x, o_xperm, o_logits, o_keys, o_alpha, o_z, o_sel, o_part, o_ylr, o_misc, o_big;
+  int o_x, o_z, o_sel, o_ylr, o_misc, o_big;  // shared-memory offsets
+  int o_logits, o_xperm, o_keys, o_alpha, o_part, o_hist;  // byte offsets inside big
   int o_aslice_off;  // A_e rows: byte offset inside big, past every other use of big
+  int aslice_regs;   // 1: A_e rows of the slice are held in registers instead
   int smem;
 };
 
@@ -73,14 +76,13 @@ struct Misc {
   uint64_t bar[2 + kRingMax];
   int ids[MSB_MAX_TOP_E];
   float w[MSB_MAX_TOP_E];
-  uint32_t hist[512];
   uint32_t info[2];
   uint32_t scan[kFT / 32 + 1];
-  float red[kFW][2 * kGroup];
   float h[kGroup];
   float maxv;
   float wsum[kFW];
   float pe[MSB_MAX_TOP_E];
+  uint32_t sscr[208];  // select scratch (block scan, results, candidates)
   int last;
 };
 
@@ -134,12 +136,13 @@ __device__ __noinline__ void router_topk(const float* logits, int E, int K, int 
     atomicOr(err, kErrNonFinite);
   }
   const float mx = M.maxv;
-  float ps = 0.f;
+  if (!renorm) {  // the softmax denominator over all E experts is only needed without renorm
+    float ps = 0.f;
 #pragma unroll 1
-  for (int ee = tid; ee < E; ee += kFT) ps += __expf(logits[ee] - mx);
-  ps = warp_sum(ps);
-  if (lane == 0) M.wsum[warp] = ps;
-  __syncthreads();
+    for (int ee = tid; ee < E; ee += kFT) ps += __expf(logits[ee] - mx);
+    ps = warp_sum(ps);
+    if (lane == 0) M.wsum[warp] = ps;
+  }
   if (tid < K) M.pe[tid] = __expf(logits[M.ids[tid]] - mx);
   __syncthreads();
   if (tid < K) {
@@ -155,10 +158,11 @@ __device__ __noinline__ void router_topk(const float* logits, int E, int K, int 
 }
 
 // Exact top-k of the I channel scores (keys = float bits) into sel[0..k), ascending.
+// hist4096: 4096 zeroed words of shared memory.
 __device__ __noinline__ void select_channels(const uint32_t* keys, int I, int k, uint16_t* sel,
-                                             Misc& M) {
+                                             uint32_t* hist4096, Misc& M) {
   uint32_t kth, need;
-  radix_kth_smem<kFT>(keys, I, k, M.hist, M.info, &kth, &need);
+  hist_kth_smem<kFT>(keys, I, k, hist4096, M.sscr, &kth, &need);
   scatter_topk<kFT>(keys, I, kth, need, sel, M.scan);
   __syncthreads();
 }
@@ -234,16 +238,22 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   const int KC = d / kColChunk;
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(sm + P.o_x);
-  uint32_t* xperm = reinterpret_cast<uint32_t*>(sm + P.o_xperm);
-  float* logits = reinterpret_cast<float*>(sm + P.o_logits);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(sm + P.o_keys);  // channel scores (float bits)
-  float* alpha_s = reinterpret_cast<float*>(sm + P.o_alpha);
   float* zs = reinterpret_cast<float*>(sm + P.o_z);
   uint16_t* sel = reinterpret_cast<uint16_t*>(sm + P.o_sel);
-  float* part = reinterpret_cast<float*>(sm + P.o_part);
   float* ylr = reinterpret_cast<float*>(sm + P.o_ylr);     // A_e z on this CTA's slice
   Misc& M = *reinterpret_cast<Misc*>(sm + P.o_misc);
   uint8_t* big = sm + P.o_big;
+  // `big` is reused phase by phase (offsets from the plan):
+  //   A: router rows at 0, logits (remote-written) after them
+  //   B: sketch tiles at 0, B_e rows, alpha, partial sums, x fragments, scores (remote-written)
+  //   C: the record ring at 0          D: the partial output at 0
+  //   A_e rows sit past all of these (loaded in B, read after the ring drains)
+  float* logits = reinterpret_cast<float*>(big + P.o_logits);
+  uint32_t* xperm = reinterpret_cast<uint32_t*>(big + P.o_xperm);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(big + P.o_keys);  // channel scores (float bits)
+  float* alpha_s = reinterpret_cast<float*>(big + P.o_alpha);
+  float* part = reinterpret_cast<float*>(big + P.o_part);
+  uint32_t* hist4096 = reinterpret_cast<uint32_t*>(big + P.o_hist);  // phase C select
   float* ybuf = reinterpret_cast<float*>(big);             // phase D: partial output (over the ring)
 
   // Every CTA of the cluster must be running before any DSMEM access targets it:
@@ -261,19 +271,13 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     if (rbytes) bulk_g2s(big, P.router_t + (size_t)e_lo * d, rbytes, &M.bar[0]);
   }
 #pragma unroll 1
-  for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
+  for (int i = tid; i < P.slice; i += kFT) ylr[i] = 0.f;
   // x and the workspace may be written by the previous launch: wait for it here.
   pdl_wait();
 #pragma unroll 1
   for (int i = tid; i < d / 8; i += kFT)
     reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
   __syncthreads();
-  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
-#pragma unroll 1
-  for (int i = tid; i < d / 2; i += kFT) {
-    const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
-    xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
-  }
 
   // ------------------------------------------------------------------ phase A: router
   bool ok = wait_phase(&M.bar[0], 0, P.err);
@@ -319,9 +323,10 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   const bool lr_out = (half == 0 && r > 0);
   uint16_t* brows = reinterpret_cast<uint16_t*>(big + code_bytes);
   uint16_t* aslice = reinterpret_cast<uint16_t*>(big + P.o_aslice_off);
+  const bool lr_smem = lr_out && !P.aslice_regs;
   if (tid == 0 && ok) {
     uint32_t bytes = code_bytes + (P.dense ? 0u : (uint32_t)nt * kRowTile * 4u) + (uint32_t)nz * 2u * d;
-    if (lr_out) bytes += (uint32_t)P.slice * r * 2u;
+    if (lr_smem) bytes += (uint32_t)P.slice * r * 2u;
     fence_proxy_async();
     mbar_arrive_expect_tx(&M.bar[1], bytes);
     if (code_bytes) {
@@ -332,9 +337,31 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
 #pragma unroll 1
     for (int i = 0; i < nz; ++i)
       bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[1]);
-    if (lr_out)
+    if (lr_smem)
       bulk_g2s(aslice, P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, (uint32_t)P.slice * r * 2u,
                &M.bar[1]);
+  }
+  // A_e rows of this CTA's output slice into registers (8 bf16 per quad), when they fit
+  uint4 areg[kAregs];
+  const int nachunk = (lr_out && P.aslice_regs) ? P.slice * r / 8 : 0;
+#pragma unroll
+  for (int u = 0; u < kAregs; ++u) {
+    const int j = tid + u * kFT;
+    areg[u] = make_uint4(0u, 0u, 0u, 0u);
+    if (ok && j < nachunk)
+      areg[u] = __ldg(reinterpret_cast<const uint4*>(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r) + j);
+  }
+  // phase-B scratch in big (past the tiles and B_e rows, which are still landing)
+#pragma unroll 1
+  for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
+  if (!P.dense)
+#pragma unroll 1
+    for (int i = tid; i < 1024; i += kFT) reinterpret_cast<uint4*>(hist4096)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
+#pragma unroll 1
+  for (int i = tid; i < d / 2; i += kFT) {
+    const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
+    xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
   }
   ok = ok && wait_phase(&M.bar[1], 0, P.err);
   ok = __syncthreads_and(ok);
@@ -355,26 +382,29 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
   }
   __syncthreads();
-  if (ok && !P.dense) {
-    // score = alpha * |sum of the 8 warps' partials| / 2, broadcast to every CTA
-    const int nrows = nt * kRowTile;
+  const int nrows = (ok && !P.dense) ? nt * kRowTile : 0;
+  // score = alpha * |sum of the 8 warps' partials| / 2 (into part's first row) ...
 #pragma unroll 1
-    for (int i = tid; i < nrows * CS; i += kFT) {
-      const int lr = i % nrows, dst = i / nrows;
-      float sc = 0.f;
+  for (int lr = tid; lr < nrows; lr += kFT) {
+    float sc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + lr];
-      sc = alpha_s[lr] * fabsf(sc) * 0.5f;
-      const int row = lt0 * kRowTile + lr;
-      cluster.map_shared_rank(keys, dst)[row] = __float_as_uint(sc);
-      if (dst == 0 && half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + row] = sc;
-    }
+    for (int w = 1; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + lr];
+    sc = alpha_s[lr] * fabsf(sc + part[lr]) * 0.5f;
+    part[lr] = sc;
+    if (half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + lt0 * kRowTile + lr] = sc;
   }
+  __syncthreads();
+  // ... then broadcast to every CTA of the cluster: item i -> (row i / CS, CTA i % CS)
+  const int lg = CS == 16 ? 4 : 3;
+#pragma unroll 1
+  for (int i = tid; i < nrows * CS; i += kFT)
+    cluster.map_shared_rank(keys, i & (CS - 1))[lt0 * kRowTile + (i >> lg)] =
+        __float_as_uint(part[i >> lg]);
   cluster.sync();
   pdl_trigger();  // the next launch may start its weight-only prologue
 
   // ------------------------------------------------------------------ phase C: top-k, records
-  if (!P.dense) select_channels(keys, I, P.k, sel, M);
+  if (!P.dense) select_channels(keys, I, P.k, sel, hist4096, M);
   if (!P.dense && half == 0 && q == 0) {
     if (P.tr.sel)
 #pragma unroll 1
@@ -396,17 +426,6 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
       mbar_arrive_expect_tx(&M.bar[2 + i], rec_bytes);
       bulk_g2s(ring + (size_t)i * 3 * d, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
                &M.bar[2 + i]);
-    }
-  }
-  // A_e z on this CTA's output slice, while the first records are in flight
-  if (ok && lr_out) {
-#pragma unroll 1
-    for (int i = tid; i < P.slice; i += kFT) {
-      const uint16_t* arow = aslice + (size_t)i * r;
-      float acc = 0.f;
-#pragma unroll 1
-      for (int rho = 0; rho < r; ++rho) acc = fmaf(bf16_lo(arow[rho]), zs[rho], acc);
-      ylr[i] = acc;
     }
   }
   float y[IT][8];
@@ -468,6 +487,39 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
   }
 
+  // A_e z on this CTA's output slice
+  if (ok && lr_out) {
+    if (P.aslice_regs) {
+      const int cpr = r / 8;  // register quads per A_e row
+#pragma unroll
+      for (int u = 0; u < kAregs; ++u) {
+        const int j = tid + u * kFT;
+        if (j < nachunk) {
+          const int row = j / cpr, rho0 = (j - row * cpr) * 8;
+          const float* zz = zs + rho0;
+          float acc = bf16_lo(areg[u].x) * zz[0];
+          acc = fmaf(bf16_hi(areg[u].x), zz[1], acc);
+          acc = fmaf(bf16_lo(areg[u].y), zz[2], acc);
+          acc = fmaf(bf16_hi(areg[u].y), zz[3], acc);
+          acc = fmaf(bf16_lo(areg[u].z), zz[4], acc);
+          acc = fmaf(bf16_hi(areg[u].z), zz[5], acc);
+          acc = fmaf(bf16_lo(areg[u].w), zz[6], acc);
+          acc = fmaf(bf16_hi(areg[u].w), zz[7], acc);
+          atomicAdd(&ylr[row], acc);
+        }
+      }
+    } else {
+#pragma unroll 1
+      for (int i = tid; i < P.slice; i += kFT) {
+        const uint16_t* arow = aslice + (size_t)i * r;
+        float acc = 0.f;
+#pragma unroll 1
+        for (int rho = 0; rho < r; ++rho) acc = fmaf(bf16_lo(arow[rho]), zs[rho], acc);
+        ylr[i] = acc;
+      }
+    }
+  }
+
   // ------------------------------------------------------------------ phase D: reduce, combine
   // partial output to this CTA's shared buffer; each owner then sums its slice over
   // the cluster with 16-byte DSMEM loads
@@ -519,6 +571,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
 namespace {
 int g_max_clusters16[64];
 int g_max_clusters8[64];
+int g_pair_smem[64];  // largest dynamic shared memory that still lets two CTAs share an SM
 bool g_ready[64];
 
 int cur_dev() {
@@ -550,24 +603,27 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe, int limit) {
   P.slice = d / cs;
   int o = 0;
   P.o_x = o;      o = align_up(o + 2 * d, 128);
-  P.o_xperm = o;  o = align_up(o + 2 * d, 128);
-  P.o_logits = o; o = align_up(o + 4 * E, 128);
-  P.o_keys = o;   o = align_up(o + 4 * ipad, 128);
-  P.o_alpha = o;  o = align_up(o + 4 * P.tpc * kRowTile, 128);
   P.o_z = o;      o = align_up(o + 4 * (r > 0 ? r : 1), 128);
   P.o_sel = o;    o = align_up(o + 2 * ipad, 128);
-  P.o_part = o;   o = align_up(o + 4 * kFW * P.tpc * kRowTile, 128);
   P.o_ylr = o;    o = align_up(o + 4 * P.slice, 128);
   P.o_misc = o;   o = align_up(o + (int)sizeof(Misc), 128);
   P.o_big = o;
-  // big, in time order: phase A router rows | phase B sketch tiles + B_e rows |
-  // phase C record ring | phase D partial output (d floats, over the drained ring);
-  // this CTA's A_e rows sit past all of them (loaded in phase B, read in phase C).
-  const int aslice_bytes = align_up(P.slice * r * 2, 128);
-  const int avail = limit - o - aslice_bytes;
-  const int need_a = P.rpc * 2 * d;
-  const int need_b = (P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4) + P.zpc * 2 * d;
+  // offsets inside big (see the kernel): phase A and phase B scratch
+  const int need_rows = align_up(P.rpc * 2 * d, 128);
+  P.o_logits = need_rows;
+  const int need_a = need_rows + align_up(4 * E, 128);
+  int b = (P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4) + P.zpc * 2 * d;
+  b = align_up(b, 128);
+  P.o_alpha = b;  b = align_up(b + 4 * P.tpc * kRowTile, 128);
+  P.o_part = b;   b = align_up(b + 4 * kFW * P.tpc * kRowTile, 128);
+  P.o_xperm = b;  b = align_up(b + 2 * d, 128);
+  P.o_keys = b;   b = align_up(b + 4 * ipad, 128);
+  P.o_hist = b;   b = align_up(b + (P.dense ? 0 : 4 * 4096), 128);
+  const int need_b = b;
   const int need_d = 4 * d;
+  P.aslice_regs = (r > 0 && r % 8 == 0 && P.slice * r / 8 <= kAregs * kFT) ? 1 : 0;
+  const int aslice_bytes = P.aslice_regs ? 0 : align_up(P.slice * r * 2, 128);
+  const int avail = limit - o - aslice_bytes;
   const int rec = 6 * d;
   int ring = avail / rec;
   if (ring > kRingMax) ring = kRingMax;
@@ -576,13 +632,12 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe, int limit) {
   if (ring > per_cta) ring = per_cta < 2 ? 2 : per_cta;
   P.ring = ring;
   P.group = ring < kFW ? ring : kFW;  // one warp per channel of a group
-  if (P.group > 4 && ring < per_cta) P.group = 4;  // refill sooner when the ring is short
-  int big = ring * rec;
-  if (need_a > big) big = need_a;
-  if (need_b > big) big = need_b;
-  if (need_d > big) big = need_d;
-  P.o_aslice_off = big;
-  P.smem = o + big + aslice_bytes;
+  int bigb = ring * rec;
+  if (need_a > bigb) bigb = need_a;
+  if (need_b > bigb) bigb = need_b;
+  if (need_d > bigb) bigb = need_d;
+  P.o_aslice_off = bigb;
+  P.smem = o + bigb + aslice_bytes;
   return P.smem <= limit;
 }
 
@@ -593,9 +648,10 @@ bool choose(FusedParams& P, const Dims& D, int k) {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64 || !g_ready[dev]) return false;
   const int K = D.top_e;
+  const int pair = g_pair_smem[dev];
   const bool have16 = g_max_clusters16[dev] >= 1, have8 = g_max_clusters8[dev] >= 1;
-  if (have16 && plan(P, D, k, 16, 1, kSmemPair)) return true;
-  if (have8 && plan(P, D, k, 8, 2, kSmemPair)) return true;
+  if (have16 && plan(P, D, k, 16, 1, pair)) return true;
+  if (have8 && plan(P, D, k, 8, 2, pair)) return true;
   if (have16 && g_max_clusters16[dev] >= K && plan(P, D, k, 16, 1, kSmemMax)) return true;
   if (have8 && g_max_clusters8[dev] >= 2 * K && plan(P, D, k, 8, 2, kSmemMax)) return true;
   if (have16 && plan(P, D, k, 16, 1, kSmemMax)) return true;
@@ -634,6 +690,15 @@ int fused_setup() {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       cudaGetLastError();
   }
+  int per_sm = 0, reserved = 0;
+  if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+    cudaGetLastError();
+    per_sm = 2 * (kSmemPair + 1024);
+    reserved = 1024;
+  }
+  g_pair_smem[dev] = per_sm / 2 - reserved;
+  if (g_pair_smem[dev] > kSmemMax) g_pair_smem[dev] = kSmemMax;
   g_max_clusters16[dev] = query_clusters(fused_block_kernel<1>, 16, kSmemMax);
   g_max_clusters8[dev] = query_clusters(fused_block_kernel<1>, 8, kSmemMax);
   g_ready[dev] = true;

@@ -330,8 +330,8 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
   __shared__ uint32_t keys[MSB_MAX_INTER];
   __shared__ uint16_t sel_s[MSB_MAX_INTER];
   __shared__ uint32_t words[MSB_MAX_INTER / 32];
-  __shared__ uint32_t hist[512];
-  __shared__ uint32_t info[2];
+  __shared__ uint32_t hist4096[4096];
+  __shared__ uint32_t sscr[208];
   __shared__ uint32_t scan_tmp[kNT / 32 + 1];
   __shared__ uint32_t s_count;
   const int p = blockIdx.x;
@@ -339,10 +339,11 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
   for (int j = threadIdx.x; j < I; j += kNT)
     keys[j] = __float_as_uint(__ldcg(&ws.scores[(size_t)p * ipad + j]));
   for (int i = threadIdx.x; i < mw; i += kNT) words[i] = 0;
+  for (int i = threadIdx.x; i < 4096; i += kNT) hist4096[i] = 0;
   __syncthreads();
   if (mode == 0) {
     uint32_t kth, need;
-    radix_kth_smem<kNT>(keys, I, k, hist, info, &kth, &need);
+    hist_kth_smem<kNT>(keys, I, k, hist4096, sscr, &kth, &need);
     scatter_topk<kNT>(keys, I, kth, need, sel_s, scan_tmp);
     if (threadIdx.x == 0) s_count = (uint32_t)k;
   } else {
