@@ -193,6 +193,37 @@ def test_zero_rows_and_duplicate_scores(msb):
             assert not ({16, 18, 20} & sel)
 
 
+@pytest.mark.parametrize("general", [False, True])
+def test_nonfinite_input_is_flagged_then_recovers(msb, general):
+    """A NaN in x makes every router logit NaN: the call is flagged (msb_check
+    returns MSB_ENONFINITE, the output is undefined) and the next call on the same
+    workspace is exact again (accumulators and counters were restored)."""
+    import torch
+    import token_top_expert_b200 as m
+    from parity import to_bf16_tensor
+    w = synth.QWEN30B_BLOCK
+    dev = device_layer(w)
+    ws = m.Workspace(dev.dims, 1)
+    x = synth.activations(w, 9)
+    bad = x.copy()
+    bad[0, 17] = 0x7FC0  # bf16 quiet NaN
+    m.moe_sparse_block(to_bf16_tensor(bad), dev, w.k, workspace=ws, general=general)
+    torch.cuda.synchronize()
+    with pytest.raises(m.MsbError) as exc:
+        ws.check()
+    assert exc.value.status == -5
+    tr = m.Trace(dev.dims, 1, w.k, scores=True)
+    out = m.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, trace=tr, general=general)
+    torch.cuda.synchronize()
+    ws.check()
+    from parity import from_bf16_tensor
+    g = {"y": oracle.bf16_to_f64(from_bf16_tensor(out)), "ids": tr.expert_ids.cpu().numpy(),
+         "w": tr.expert_w.cpu().numpy(), "sel": tr.sel.cpu().numpy().view(np.uint16),
+         "sel_count": tr.sel_count.cpu().numpy(), "union": tr.union_count.cpu().numpy(),
+         "scores": tr.scores.cpu().numpy()}
+    compare(x, g, oracle.SynthLayer(w), w.top_e, w.k)
+
+
 def test_selection_is_deterministic(msb):
     w = synth.QWEN30B_BLOCK
     dev = device_layer(w)

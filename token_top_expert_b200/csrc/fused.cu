@@ -38,10 +38,12 @@ namespace msb {
 constexpr int kFT = 256;        // threads per CTA
 constexpr int kFW = kFT / 32;   // warps per CTA
 constexpr int kRingMax = 16;    // record slots
-constexpr int kGroup = 8;       // channels reduced together
 constexpr int kSmemMax = 227 * 1024;
 constexpr int kSmemPair = 110 * 1024;  // fallback pairing limit if the device cannot be queried
 constexpr int kAregs = 8;              // register quads for the slice's A_e rows (8 bf16 each)
+constexpr int kMyselMax = 256;         // channels one CTA reads at most
+constexpr int kSelBins = 2048;         // select histogram bins (256 per octave below the largest key)
+constexpr int kCandMax = 64;           // keys ranked directly in the k-th key's bin
 
 struct FusedParams {
   const uint16_t* x;
@@ -58,15 +60,18 @@ struct FusedParams {
   TraceDev tr;
   Dims D;
   int k, dense, cs, cpe;
+  int epad;    // router logits padded to a multiple of 64 (with -inf)
   int rpc;     // router rows per CTA
   int tpc;     // sketch row tiles per CTA
   int zpc;     // z rows per CTA (max)
   int slice;   // output elements owned per CTA (d / cs)
   int ring;    // record slots
+  int rs;      // ring slot stride in bf16 elements: 3d + 8 (16 bytes of stagger between
+               // slots, so rows of consecutive slots fall in different banks)
   int group;   // channels per reduction group (<= ring)
   // shared-memory carve-up (byte offsets)
-  int o_x, o_z, o_sel, o_ylr, o_misc, o_big;  // shared-memory offsets
-  int o_logits, o_xperm, o_keys, o_alpha, o_part, o_hist;  // byte offsets inside big
+  int o_z, o_ylr, o_misc, o_big;  // shared-memory offsets
+  int o_logits, o_xperm, o_keys, o_alpha, o_part, o_hist, o_xbig;  // offsets in big
   int o_aslice_off;  // A_e rows: byte offset inside big, past every other use of big
   int aslice_regs;   // 1: A_e rows of the slice are held in registers instead
   int smem;
@@ -75,14 +80,19 @@ struct FusedParams {
 struct Misc {
   uint64_t bar[2 + kRingMax];
   int ids[MSB_MAX_TOP_E];
-  float w[MSB_MAX_TOP_E];
+  float lv[MSB_MAX_TOP_E];  // routed logits in rank order
   uint32_t info[2];
-  uint32_t scan[kFT / 32 + 1];
-  float h[kGroup];
-  float maxv;
-  float wsum[kFW];
-  float pe[MSB_MAX_TOP_E];
-  uint32_t sscr[208];  // select scratch (block scan, results, candidates)
+  float h[kRingMax];
+  float red[kFW][2 * kRingMax];  // per-warp (gate . x, up . x) of a group's channels
+  // channel select scratch
+  uint32_t wt[kFW], wt2[kFW];  // per-warp totals of the two block scans
+  uint32_t kb, rem, cnt, ccount, kth, need;
+  uint32_t ck[kCandMax];       // keys of the bin holding the k-th key, and their indices
+  uint32_t ci[kCandMax];
+  uint32_t cmax[16];           // largest score key of each CTA of the cluster
+  uint32_t lmax;               // largest score key of this CTA
+  uint32_t tie;                // router: a rank slot was claimed twice
+  uint16_t mysel[kMyselMax];  // this CTA's share of the selected channels
   int last;
 };
 
@@ -101,69 +111,202 @@ __device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint32_t
   return mbar_wait(bar, parity, err);
 }
 
-// Router top-K over the E logits in shared memory, by rank counting:
-// rank(e) = #{e' : l_e' > l_e or (l_e' == l_e and e' < e)}, two threads per logit.
-// Writes M.ids[0..K) (rank order) and the combine weights M.w[0..K).
-__device__ __noinline__ void router_topk(const float* logits, int E, int K, int renorm, Misc& M,
+// Router top-K over the E logits in shared memory (padded with -inf to Epad, a
+// multiple of 64), by rank counting, P = 256/E threads per logit (at most 4) on
+// 16-value vector steps.  Fast pass: rank = #{e' : l_e' > l_e}; the owner of rank
+// j < K claims slot j.  Without ties among the top K every claim lands in its own
+// slot and these ranks are exact; two logits with the same value have the same
+// count, so a tie shows as a second claim on one slot, and then the exact pass
+// ranks by #{e' : l_e' > l_e} + #{e' < e : l_e' == l_e} (ties to the lower index).
+// M.ids must be -1 and M.tie 0 on entry.  Ends with a barrier.
+__device__ __noinline__ void router_rank(const float* logits, int E, int Epad, int K, Misc& M,
                                          uint32_t* err) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < K) M.ids[tid] = -1;
-  __syncthreads();
-  const int halfE = E / 2;
+  const int tid = threadIdx.x;
+  const int lgP = E <= 64 ? 2 : (E <= 128 ? 1 : 0);
+  const int span = Epad >> lgP;
 #pragma unroll 1
-  for (int base = 0; base < 2 * E; base += kFT) {
-    const int item = base + tid, ee = item >> 1, h = item & 1;
-    int rank = 0;
-    float v = 0.f;
-    if (ee < E) {
-      v = logits[ee];
-      const int j1 = h ? E : halfE;
-#pragma unroll 2
-      for (int j = h ? halfE : 0; j < j1; ++j) {
-        const float u = logits[j];
-        rank += (u > v) || (u == v && j < ee);
+  for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll 1
+    for (int base = 0; base < (E << lgP); base += kFT) {
+      const int item = base + tid, ee = item >> lgP, h = item & ((1 << lgP) - 1);
+      float gt = 0.f;
+      float v = 0.f;
+      if (ee < E) {
+        v = logits[ee];
+        if (pass == 0) {
+          if (!isfinite(v)) atomicOr(err, kErrNonFinite);
+          const float4* lp = reinterpret_cast<const float4*>(logits + h * span);
+#pragma unroll 4
+          for (int c = 0; c < span / 4; ++c) {
+            const float4 u = lp[c];
+            gt += (u.x > v ? 1.f : 0.f) + (u.y > v ? 1.f : 0.f);
+            gt += (u.z > v ? 1.f : 0.f) + (u.w > v ? 1.f : 0.f);
+          }
+        } else {
+          int r = 0;
+#pragma unroll 1
+          for (int j = h * span; j < (h + 1) * span; ++j) {
+            const float u = logits[j];
+            r += (u > v) || (u == v && j < ee);
+          }
+          gt = (float)r;
+        }
+      }
+      if (lgP >= 1) gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+      if (lgP >= 2) gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+      const int rank = (int)gt;
+      if (ee < E && h == 0 && rank < K) {
+        if (atomicCAS(&M.ids[rank], -1, ee) != -1) M.tie = 1u;
+        M.lv[rank] = v;
       }
     }
-    rank += __shfl_xor_sync(0xffffffffu, rank, 1);
-    if (ee < E && h == 0) {
-      if (rank < K) M.ids[rank] = ee;
-      if (rank == 0) M.maxv = v;
-    }
+    __syncthreads();
+    if (pass == 1 || M.tie == 0u) break;
+    if (tid < K) M.ids[tid] = -1;
+    __syncthreads();
   }
-  __syncthreads();
-  if (tid < K && M.ids[tid] < 0) {  // non-finite logits: keep a valid index and flag the call
-    M.ids[tid] = tid;
-    atomicOr(err, kErrNonFinite);
-  }
-  const float mx = M.maxv;
-  if (!renorm) {  // the softmax denominator over all E experts is only needed without renorm
-    float ps = 0.f;
-#pragma unroll 1
-    for (int ee = tid; ee < E; ee += kFT) ps += __expf(logits[ee] - mx);
-    ps = warp_sum(ps);
-    if (lane == 0) M.wsum[warp] = ps;
-  }
-  if (tid < K) M.pe[tid] = __expf(logits[M.ids[tid]] - mx);
-  __syncthreads();
-  if (tid < K) {
-    float denom = 0.f;
-    if (renorm) {
-      for (int j = 0; j < K; ++j) denom += M.pe[j];
-    } else {
-      for (int w = 0; w < kFW; ++w) denom += M.wsum[w];
-    }
-    M.w[tid] = __fdividef(M.pe[tid], denom);
-  }
-  __syncthreads();
 }
 
-// Exact top-k of the I channel scores (keys = float bits) into sel[0..k), ascending.
-// hist4096: 4096 zeroed words of shared memory.
-__device__ __noinline__ void select_channels(const uint32_t* keys, int I, int k, uint16_t* sel,
-                                             uint32_t* hist4096, Misc& M) {
+// Combine weight of the routed expert of rank j (every lane of the warp calls it,
+// after router_rank): softmax over the K routed logits (renorm) or over all E
+// logits.  lv[0] is the largest logit.
+__device__ __forceinline__ float router_weight(const float* logits, int E, int K, int renorm,
+                                               const Misc& M, int j) {
+  const int lane = threadIdx.x & 31;
+  const float mx = M.lv[0];
+  const float pl = lane < K ? __expf(M.lv[lane] - mx) : 0.f;
+  float denom = 0.f;
+  if (renorm) {
+    denom = pl;
+  } else {
+#pragma unroll 1
+    for (int i = lane; i < E; i += 32) denom += __expf(logits[i] - mx);
+  }
+  denom = warp_sum(denom);
+  return __fdividef(__shfl_sync(0xffffffffu, pl, j), denom);
+}
+
+// Exact top-k of the n channel scores (keys = float bits, so integer order is value
+// order), ties to the lower index; writes this CTA's share, positions [c0, c1) of
+// the ascending selected list, to M.mysel and (when trace is set) the whole list to
+// trace.  Keys are binned by (maxkey - key) >> 15 (256 bins per octave below the
+// largest key, bin 0 the largest, the last bin catching the rest): one counting
+// pass and one scan find the bin of the k-th key, whose keys are then ranked
+// directly; a bin with more than kCandMax keys falls back to a radix descent.
+// hist: kSelBins zeroed words.  M.ccount must be 0 on entry.
+__device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, uint32_t maxkey,
+                                          uint32_t* hist, Misc& M, int c0, int c1, uint16_t* trace) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll 4
+  for (int j = tid; j < n; j += kFT) atomicAdd(&hist[min((uint32_t)(kSelBins - 1), (maxkey - keys[j]) >> 15)], 1u);
+  __syncthreads();
+  // thread t owns bins [8t, 8t + 8)
+  uint32_t c[8];
+  {
+    const uint4 a = reinterpret_cast<const uint4*>(hist)[2 * tid];
+    const uint4 b = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
+    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
+  }
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) local += c[i];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) M.wt[warp] = incl;
+  __syncthreads();
+  uint32_t above = incl - local;
+#pragma unroll
+  for (int w = 0; w < kFW; ++w) above += w < warp ? M.wt[w] : 0u;
+  const uint32_t kk = (uint32_t)k;
+  if (above < kk && kk <= above + local) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (above < kk && kk <= above + c[i]) { M.kb = 8 * tid + i; M.rem = kk - above; M.cnt = c[i]; }
+      above += c[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
   uint32_t kth, need;
-  hist_kth_smem<kFT>(keys, I, k, hist4096, M.sscr, &kth, &need);
-  scatter_topk<kFT>(keys, I, kth, need, sel, M.scan);
+  if (cnt > (uint32_t)kCandMax) {
+    radix_kth_smem<kFT>(keys, n, k, hist, M.info, &kth, &need);
+  } else {
+    const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 4
+    for (int j0 = warp * 32; j0 < n; j0 += kFT) {  // warp-uniform trip count
+      const int j = j0 + lane;
+      const uint32_t key = j < n ? keys[j] : 0u;
+      const bool m = j < n && min((uint32_t)(kSelBins - 1), (maxkey - key) >> 15) == kb;
+      const uint32_t mb = __ballot_sync(0xffffffffu, m);
+      if (mb) {
+        const int leader = __ffs(mb) - 1;
+        uint32_t slot0 = 0;
+        if (lane == leader) slot0 = atomicAdd(&M.ccount, (uint32_t)__popc(mb));
+        slot0 = __shfl_sync(0xffffffffu, slot0, leader);
+        if (m) {
+          const uint32_t slot = slot0 + __popc(mb & lt);
+          M.ck[slot] = key;
+          M.ci[slot] = (uint32_t)j;
+        }
+      }
+    }
+    __syncthreads();
+    // rank inside the bin by (key desc, index asc): the k-th key has rank rem - 1
+    if (tid < (int)cnt) {
+      const uint32_t mk = M.ck[tid], mi = M.ci[tid];
+      uint32_t rank = 0, gt = 0;
+#pragma unroll 4
+      for (int i = 0; i < (int)cnt; ++i) {
+        const uint32_t ok_ = M.ck[i], oi = M.ci[i];
+        rank += (ok_ > mk) || (ok_ == mk && oi < mi);
+        gt += ok_ > mk;
+      }
+      if (rank == rem - 1) { M.kth = mk; M.need = rem - gt; }
+    }
+    __syncthreads();
+    kth = M.kth;
+    need = M.need;
+  }
+  // scatter: warp w owns indices [w * span, (w + 1) * span); ballots give positions
+  const int span = 32 * ((n + kFT - 1) / kFT);
+  const int wb = warp * span, we = min(n, wb + span);
+  uint32_t ngt = 0, neq = 0;
+#pragma unroll 4
+  for (int j0 = wb; j0 < we; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < we ? keys[j] : 0u;
+    ngt += __popc(__ballot_sync(0xffffffffu, j < we && key > kth));
+    neq += __popc(__ballot_sync(0xffffffffu, j < we && key == kth));
+  }
+  if (lane == 0) M.wt2[warp] = ngt | (neq << 16);
+  __syncthreads();
+  uint32_t gtb = 0, eqb = 0;
+#pragma unroll
+  for (int w = 0; w < kFW; ++w) {
+    const uint32_t v = w < warp ? M.wt2[w] : 0u;
+    gtb += v & 0xffffu;
+    eqb += v >> 16;
+  }
+  const uint32_t ltm = (1u << lane) - 1u;
+#pragma unroll 4
+  for (int j0 = wb; j0 < we; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < we ? keys[j] : 0u;
+    const uint32_t bg = __ballot_sync(0xffffffffu, j < we && key > kth);
+    const uint32_t be = __ballot_sync(0xffffffffu, j < we && key == kth);
+    const uint32_t eqr = eqb + __popc(be & ltm);
+    if (((bg >> lane) & 1u) || (((be >> lane) & 1u) && eqr < need)) {
+      const int pos = (int)(gtb + __popc(bg & ltm) + min(eqr, need));
+      if (pos >= c0 && pos < c1) M.mysel[pos - c0] = (uint16_t)j;
+      if (trace) trace[pos] = (uint16_t)j;
+    }
+    gtb += __popc(bg);
+    eqb += __popc(be);
+  }
   __syncthreads();
 }
 
@@ -205,24 +348,6 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
   }
 }
 
-// One warp per channel: h = silu(gate . x) * (up . x) for channel record `rec`.
-__device__ __forceinline__ float channel_h(const uint16_t* rec, const uint16_t* xs, int d) {
-  const int lane = threadIdx.x & 31;
-  const uint4* gr = reinterpret_cast<const uint4*>(rec);
-  const uint4* ur = reinterpret_cast<const uint4*>(rec + d);
-  const uint4* xr = reinterpret_cast<const uint4*>(xs);
-  float g = 0.f, u = 0.f;
-#pragma unroll 2
-  for (int i = lane; i < d / 8; i += 32) {
-    const uint4 xv = xr[i];
-    g = dot8(gr[i], xv, g);
-    u = dot8(ur[i], xv, u);
-  }
-  g = warp_sum(g);
-  u = warp_sum(u);
-  return __fdividef(g, 1.0f + __expf(-g)) * u;
-}
-
 template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
 __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_constant__ FusedParams P) {
   extern __shared__ __align__(128) uint8_t sm[];
@@ -237,9 +362,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   const int d = D.d, E = D.experts, I = D.inter, ipad = D.ipad, r = D.rank, K = D.top_e;
   const int KC = d / kColChunk;
 
-  uint16_t* xs = reinterpret_cast<uint16_t*>(sm + P.o_x);
   float* zs = reinterpret_cast<float*>(sm + P.o_z);
-  uint16_t* sel = reinterpret_cast<uint16_t*>(sm + P.o_sel);
   float* ylr = reinterpret_cast<float*>(sm + P.o_ylr);     // A_e z on this CTA's slice
   Misc& M = *reinterpret_cast<Misc*>(sm + P.o_misc);
   uint8_t* big = sm + P.o_big;
@@ -248,12 +371,13 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   //   B: sketch tiles at 0, B_e rows, alpha, partial sums, x fragments, scores (remote-written)
   //   C: the record ring at 0          D: the partial output at 0
   //   A_e rows sit past all of these (loaded in B, read after the ring drains)
+  uint16_t* xs = reinterpret_cast<uint16_t*>(big + P.o_xbig);  // phases A-B (C reads x from L1/L2)
   float* logits = reinterpret_cast<float*>(big + P.o_logits);
   uint32_t* xperm = reinterpret_cast<uint32_t*>(big + P.o_xperm);
   uint32_t* keys = reinterpret_cast<uint32_t*>(big + P.o_keys);  // channel scores (float bits)
   float* alpha_s = reinterpret_cast<float*>(big + P.o_alpha);
   float* part = reinterpret_cast<float*>(big + P.o_part);
-  uint32_t* hist4096 = reinterpret_cast<uint32_t*>(big + P.o_hist);  // phase C select
+  uint32_t* hist = reinterpret_cast<uint32_t*>(big + P.o_hist);  // phase C select
   float* ybuf = reinterpret_cast<float*>(big);             // phase D: partial output (over the ring)
 
   // Every CTA of the cluster must be running before any DSMEM access targets it:
@@ -272,6 +396,9 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   }
 #pragma unroll 1
   for (int i = tid; i < P.slice; i += kFT) ylr[i] = 0.f;
+  for (int i = E + tid; i < P.epad; i += kFT) logits[i] = -INFINITY;
+  if (tid < K) M.ids[tid] = -1;
+  if (tid == 0) { M.lmax = 0u; M.ccount = 0u; M.tie = 0u; }
   // x and the workspace may be written by the previous launch: wait for it here.
   pdl_wait();
 #pragma unroll 1
@@ -297,19 +424,25 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
   }
   cluster.sync();
-  router_topk(logits, E, K, D.renorm, M, P.err);
-  const int e = M.ids[rc];
-  const float we = M.w[rc];
+  router_rank(logits, E, P.epad, K, M, P.err);
+  int e = M.ids[rc];
+  if (e < 0) {  // a rank left empty (non-finite logits): keep a valid index, the call is flagged
+    e = rc;
+    if (tid == 0) atomicOr(P.err, kErrNonFinite);
+  }
+  const float we = router_weight(logits, E, K, D.renorm, M, rc);
   if (blockIdx.x == 0) {
-    if (tid < K) {
-      if (P.tr.expert_ids) P.tr.expert_ids[tid] = M.ids[tid];
-      if (P.tr.expert_w) P.tr.expert_w[tid] = M.w[tid];
+    if (warp == 0) {  // (the weight of a non-renormalised softmax is a warp-wide sum)
+      const float wl = router_weight(logits, E, K, D.renorm, M, lane < K ? lane : 0);
+
+      if (lane < K && P.tr.expert_ids) P.tr.expert_ids[lane] = M.ids[lane] < 0 ? lane : M.ids[lane];
+      if (lane < K && P.tr.expert_w) P.tr.expert_w[lane] = wl;
     }
     if (P.tr.union_count)
 #pragma unroll 1
       for (int i = tid; i < E; i += kFT) {
         int c = 0;
-        for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? P.k : c;
+        for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? P.k : c;  // (-1 never matches)
         P.tr.union_count[i] = c;
       }
   }
@@ -356,7 +489,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
   if (!P.dense)
 #pragma unroll 1
-    for (int i = tid; i < 1024; i += kFT) reinterpret_cast<uint4*>(hist4096)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < kSelBins / 4; i += kFT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
   // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
 #pragma unroll 1
   for (int i = tid; i < d / 2; i += kFT) {
@@ -384,6 +517,7 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   __syncthreads();
   const int nrows = (ok && !P.dense) ? nt * kRowTile : 0;
   // score = alpha * |sum of the 8 warps' partials| / 2 (into part's first row) ...
+  uint32_t lmax = 0;
 #pragma unroll 1
   for (int lr = tid; lr < nrows; lr += kFT) {
     float sc = 0.f;
@@ -391,10 +525,15 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     for (int w = 1; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + lr];
     sc = alpha_s[lr] * fabsf(sc + part[lr]) * 0.5f;
     part[lr] = sc;
+    lmax = max(lmax, __float_as_uint(sc));
     if (half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + lt0 * kRowTile + lr] = sc;
   }
+  lmax = __reduce_max_sync(0xffffffffu, lmax);
+  if (lane == 0 && lmax) atomicMax(&M.lmax, lmax);
   __syncthreads();
-  // ... then broadcast to every CTA of the cluster: item i -> (row i / CS, CTA i % CS)
+  // ... then broadcast to every CTA of the cluster: item i -> (row i / CS, CTA i % CS),
+  // with this CTA's largest key
+  if (tid < CS) cluster.map_shared_rank(M.cmax, tid)[q] = M.lmax;
   const int lg = CS == 16 ? 4 : 3;
 #pragma unroll 1
   for (int i = tid; i < nrows * CS; i += kFT)
@@ -404,17 +543,22 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   pdl_trigger();  // the next launch may start its weight-only prologue
 
   // ------------------------------------------------------------------ phase C: top-k, records
-  if (!P.dense) select_channels(keys, I, P.k, sel, hist4096, M);
-  if (!P.dense && half == 0 && q == 0) {
-    if (P.tr.sel)
-#pragma unroll 1
-      for (int i = tid; i < P.k; i += kFT) P.tr.sel[(size_t)rc * P.k + i] = sel[i];
-    if (tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
-  }
-  // this CTA's share of the k channels
+  // this CTA's share of the k channels: positions [c0, c1) of the ascending list
   const int NQ = CS * P.cpe, gq = half * CS + q;
   const int c0 = (int)((long)gq * P.k / NQ), c1 = (int)((long)(gq + 1) * P.k / NQ);
   const int nmine = c1 - c0;
+  if (!P.dense) {
+    uint32_t maxkey = 0;
+#pragma unroll 1
+    for (int i = 0; i < CS; ++i) maxkey = max(maxkey, M.cmax[i]);
+    uint16_t* trace = (half == 0 && q == 0 && P.tr.sel) ? P.tr.sel + (size_t)rc * P.k : nullptr;
+    select_share(keys, I, P.k, maxkey, hist, M, c0, c1, trace);
+    if (half == 0 && q == 0 && tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
+  } else {
+#pragma unroll 1
+    for (int i = tid; i < nmine; i += kFT) M.mysel[i] = (uint16_t)(c0 + i);
+    __syncthreads();
+  }
   const uint32_t rec_bytes = 6u * d;
   uint16_t* ring = reinterpret_cast<uint16_t*>(big);
   if (tid == 0 && ok) {
@@ -422,72 +566,13 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     const int first = min(P.ring, nmine);
 #pragma unroll 1
     for (int i = 0; i < first; ++i) {
-      const int ch = P.dense ? c0 + i : (int)sel[c0 + i];
+      const int ch = M.mysel[i];
       mbar_arrive_expect_tx(&M.bar[2 + i], rec_bytes);
-      bulk_g2s(ring + (size_t)i * 3 * d, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
+      bulk_g2s(ring + (size_t)i * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
                &M.bar[2 + i]);
     }
   }
-  float y[IT][8];
-#pragma unroll
-  for (int it = 0; it < IT; ++it)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
-#pragma unroll 1
-  for (int g0 = 0; g0 < nmine; g0 += P.group) {
-    const int ng = min(P.group, nmine - g0);
-    // warp w computes h of channel g0 + w once its record has landed
-    if (warp < ng) {
-      const int ci = g0 + warp;
-      const bool okw = ok && wait_phase(&M.bar[2 + ci % P.ring], (ci / P.ring) & 1u, P.err);
-      float hv = 0.f;
-      if (okw) hv = channel_h(ring + (size_t)(ci % P.ring) * 3 * d, xs, d);
-      if (lane == 0) M.h[warp] = hv;
-      if (!okw && lane == 0) M.h[warp] = 0.f;
-    }
-    ok = __syncthreads_and(ok);
-    if (ok) {
-      // y += h_i * down_i over this thread's elements
-#pragma unroll 1
-      for (int i = 0; i < ng; ++i) {
-        const uint16_t* rec = ring + (size_t)((g0 + i) % P.ring) * 3 * d + 2 * d;
-        const float h = M.h[i];
-#pragma unroll
-        for (int it = 0; it < IT; ++it) {
-          const int el = (it * kFT + tid) * 8;
-          if (el < d) {
-            const uint4 dv = *reinterpret_cast<const uint4*>(rec + el);
-            y[it][0] = fmaf(h, bf16_lo(dv.x), y[it][0]);
-            y[it][1] = fmaf(h, bf16_hi(dv.x), y[it][1]);
-            y[it][2] = fmaf(h, bf16_lo(dv.y), y[it][2]);
-            y[it][3] = fmaf(h, bf16_hi(dv.y), y[it][3]);
-            y[it][4] = fmaf(h, bf16_lo(dv.z), y[it][4]);
-            y[it][5] = fmaf(h, bf16_hi(dv.z), y[it][5]);
-            y[it][6] = fmaf(h, bf16_lo(dv.w), y[it][6]);
-            y[it][7] = fmaf(h, bf16_hi(dv.w), y[it][7]);
-          }
-        }
-      }
-    }
-    __syncthreads();
-    // refill the slots just consumed
-    if (tid == 0 && ok) {
-      fence_proxy_async();
-#pragma unroll 1
-      for (int i = g0; i < g0 + ng; ++i) {
-        const int nx = i + P.ring;
-        if (nx < nmine) {
-          const int ch = P.dense ? c0 + nx : (int)sel[c0 + nx];
-          const int slot = nx % P.ring;
-          mbar_arrive_expect_tx(&M.bar[2 + slot], rec_bytes);
-          bulk_g2s(ring + (size_t)slot * 3 * d, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
-                   &M.bar[2 + slot]);
-        }
-      }
-    }
-  }
-
-  // A_e z on this CTA's output slice
+  // A_e z on this CTA's output slice, while the records are in flight
   if (ok && lr_out) {
     if (P.aslice_regs) {
       const int cpr = r / 8;  // register quads per A_e row
@@ -520,6 +605,111 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
   }
 
+  // Per group: gate . x and up . x of the group's channels on the tensor cores (A =
+  // the records' gate/up rows, bf16 straight from the ring via ldmatrix; B = x, read
+  // through L1; warp w takes k-steps [ks0, ks1) and the warps' partials meet in
+  // M.red), then h, then y += h_i * down_i with every thread owning 8-element groups.
+  const int KS = d / 16;
+  const int ks0 = warp * KS / kFW, ks1 = (warp + 1) * KS / kFW;
+  const uint32_t* x32 = reinterpret_cast<const uint32_t*>(P.x);
+  const int c4 = lane & 3, g8 = lane >> 2;
+  float y[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
+#pragma unroll 1
+  for (int g0 = 0; g0 < nmine; g0 += P.group) {
+    const int ng = min(P.group, nmine - g0);
+#pragma unroll 1
+    for (int i = 0; i < ng; ++i)
+      ok = ok && wait_phase(&M.bar[2 + (g0 + i) % P.ring], ((g0 + i) / P.ring) & 1u, P.err);
+#pragma unroll 1
+    for (int tb = 0; tb < ng; tb += 8) {
+      // this lane's ldmatrix row: channel tb + lane % 8 (rows past ng repeat channel tb;
+      // their results are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 * (lane / 16)
+      const int ch = (tb + (lane & 7) < ng) ? tb + (lane & 7) : tb;
+      uint32_t a_addr = smem_addr(ring + (size_t)((g0 + ch) % P.ring) * P.rs + ((lane >> 3) & 1) * d +
+                                  8 * (lane >> 4)) + 32u * ks0;
+      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      int ks = ks0;
+      if (ok) {
+#pragma unroll 1
+        for (; ks + 4 <= ks1; ks += 4, a_addr += 128u) {
+          uint32_t a[4][4], b[4][2];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            ldsm_x4(a_addr + 32u * u, a[u][0], a[u][1], a[u][2], a[u][3]);
+            b[u][0] = __ldg(x32 + (ks + u) * 8 + c4);
+            b[u][1] = __ldg(x32 + (ks + u) * 8 + 4 + c4);
+          }
+          mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b[0][0], b[0][1]);
+          mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b[1][0], b[1][1]);
+          mma_bf16(acc0, a[2][0], a[2][1], a[2][2], a[2][3], b[2][0], b[2][1]);
+          mma_bf16(acc1, a[3][0], a[3][1], a[3][2], a[3][3], b[3][0], b[3][1]);
+        }
+#pragma unroll 1
+        for (; ks < ks1; ++ks, a_addr += 32u) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(a_addr, a0, a1, a2, a3);
+          mma_bf16(acc0, a0, a1, a2, a3, __ldg(x32 + ks * 8 + c4), __ldg(x32 + ks * 8 + 4 + c4));
+        }
+      }
+      // column 0 of D: lanes with lane % 4 == 0 hold gate (row g8) and up (row g8 + 8)
+      if (c4 == 0 && tb + g8 < ng) {
+        M.red[warp][2 * (tb + g8)] = acc0[0] + acc1[0];
+        M.red[warp][2 * (tb + g8) + 1] = acc0[2] + acc1[2];
+      }
+    }
+    ok = __syncthreads_and(ok);
+    if (tid < ng) {
+      float g = 0.f, u = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFW; ++w) { g += M.red[w][2 * tid]; u += M.red[w][2 * tid + 1]; }
+      M.h[tid] = __fdividef(g, 1.0f + __expf(-g)) * u;
+    }
+    __syncthreads();
+    if (ok) {
+      // y += h_i * down_i over this thread's elements
+#pragma unroll 4
+      for (int i = 0; i < ng; ++i) {
+        const uint16_t* rec = ring + (size_t)((g0 + i) % P.ring) * P.rs + 2 * d;
+        const float h = M.h[i];
+#pragma unroll
+        for (int it = 0; it < IT; ++it) {
+          const int el = (it * kFT + tid) * 8;
+          if (el < d) {
+            const uint4 dv = *reinterpret_cast<const uint4*>(rec + el);
+            y[it][0] = fmaf(h, bf16_lo(dv.x), y[it][0]);
+            y[it][1] = fmaf(h, bf16_hi(dv.x), y[it][1]);
+            y[it][2] = fmaf(h, bf16_lo(dv.y), y[it][2]);
+            y[it][3] = fmaf(h, bf16_hi(dv.y), y[it][3]);
+            y[it][4] = fmaf(h, bf16_lo(dv.z), y[it][4]);
+            y[it][5] = fmaf(h, bf16_hi(dv.z), y[it][5]);
+            y[it][6] = fmaf(h, bf16_lo(dv.w), y[it][6]);
+            y[it][7] = fmaf(h, bf16_hi(dv.w), y[it][7]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // refill the slots just consumed
+    if (tid == 0 && ok) {
+      fence_proxy_async();
+#pragma unroll 1
+      for (int i = g0; i < g0 + ng; ++i) {
+        const int nx = i + P.ring;
+        if (nx < nmine) {
+          const int ch = M.mysel[nx];
+          const int slot = nx % P.ring;
+          mbar_arrive_expect_tx(&M.bar[2 + slot], rec_bytes);
+          bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
+                   &M.bar[2 + slot]);
+        }
+      }
+    }
+  }
+
   // ------------------------------------------------------------------ phase D: reduce, combine
   // partial output to this CTA's shared buffer; each owner then sums its slice over
   // the cluster with 16-byte DSMEM loads
@@ -536,12 +726,15 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
 #pragma unroll 1
     for (int j = tid; j < P.slice / 4; j += kFT) {
       const int el = q * P.slice + 4 * j;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-      for (int src = 0; src < CS; ++src) {
-        const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ybuf, src) + el);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
+      // all CS remote loads in flight at once
+      float4 v[16];
+#pragma unroll
+      for (int src = 0; src < 16; ++src)
+        if (src < CS) v[src] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ybuf, src) + el);
+      float4 acc = v[0];
+#pragma unroll
+      for (int src = 1; src < 16; ++src)
+        if (src < CS) { acc.x += v[src].x; acc.y += v[src].y; acc.z += v[src].z; acc.w += v[src].w; }
       if (lr_out) {
         acc.x += ylr[4 * j]; acc.y += ylr[4 * j + 1]; acc.z += ylr[4 * j + 2]; acc.w += ylr[4 * j + 3];
       }
@@ -602,36 +795,40 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe, int limit) {
   P.zpc = (r + cs - 1) / cs;
   P.slice = d / cs;
   int o = 0;
-  P.o_x = o;      o = align_up(o + 2 * d, 128);
   P.o_z = o;      o = align_up(o + 4 * (r > 0 ? r : 1), 128);
-  P.o_sel = o;    o = align_up(o + 2 * ipad, 128);
   P.o_ylr = o;    o = align_up(o + 4 * P.slice, 128);
   P.o_misc = o;   o = align_up(o + (int)sizeof(Misc), 128);
   P.o_big = o;
   // offsets inside big (see the kernel): phase A and phase B scratch
   const int need_rows = align_up(P.rpc * 2 * d, 128);
   P.o_logits = need_rows;
-  const int need_a = need_rows + align_up(4 * E, 128);
+  P.epad = (E + 63) / 64 * 64;
+  const int need_a = need_rows + align_up(4 * P.epad, 128);
   int b = (P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4) + P.zpc * 2 * d;
   b = align_up(b, 128);
   P.o_alpha = b;  b = align_up(b + 4 * P.tpc * kRowTile, 128);
   P.o_part = b;   b = align_up(b + 4 * kFW * P.tpc * kRowTile, 128);
   P.o_xperm = b;  b = align_up(b + 2 * d, 128);
   P.o_keys = b;   b = align_up(b + 4 * ipad, 128);
-  P.o_hist = b;   b = align_up(b + (P.dense ? 0 : 4 * 4096), 128);
-  const int need_b = b;
+  P.o_hist = b;   b = align_up(b + (P.dense ? 0 : 4 * kSelBins), 128);
+  // x lives past both phases' scratch until the ring takes over
+  P.o_xbig = align_up(need_a > b ? need_a : b, 128);
+  const int need_b = align_up(P.o_xbig + 2 * d, 128);
   const int need_d = 4 * d;
+  if ((k + cs * cpe - 1) / (cs * cpe) > kMyselMax) return false;
   P.aslice_regs = (r > 0 && r % 8 == 0 && P.slice * r / 8 <= kAregs * kFT) ? 1 : 0;
   const int aslice_bytes = P.aslice_regs ? 0 : align_up(P.slice * r * 2, 128);
   const int avail = limit - o - aslice_bytes;
-  const int rec = 6 * d;
+  P.rs = 3 * d + 8;
+  const int rec = 2 * P.rs;
   int ring = avail / rec;
   if (ring > kRingMax) ring = kRingMax;
   if (ring < 2 || need_a > avail || need_b > avail || need_d > avail) return false;
   const int per_cta = (k + cs * cpe - 1) / (cs * cpe);  // channels a CTA reads
   if (ring > per_cta) ring = per_cta < 2 ? 2 : per_cta;
   P.ring = ring;
-  P.group = ring < kFW ? ring : kFW;  // one warp per channel of a group
+  // one group when every record fits the ring, else two groups in flight
+  P.group = per_cta <= ring ? ring : (ring + 1) / 2;
   int bigb = ring * rec;
   if (need_a > bigb) bigb = need_a;
   if (need_b > bigb) bigb = need_b;

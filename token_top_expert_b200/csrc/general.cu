@@ -80,12 +80,15 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
     constexpr int MAXM = MSB_MAX_EXPERTS / 32;
     float v[MAXM];
     float mx = -INFINITY;
+    bool bad = false;
 #pragma unroll
     for (int m = 0; m < MAXM; ++m) {
       const int ee = lane + 32 * m;
       v[m] = ee < E ? __ldcg(&ws.logits[(size_t)t * E + ee]) : -INFINITY;
+      bad = bad || (ee < E && !isfinite(v[m]));
       mx = fmaxf(mx, v[m]);
     }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) atomicOr(ws.err, kErrNonFinite);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float sum = 0.f;
