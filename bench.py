@@ -222,16 +222,29 @@ def run_stack(args, w, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     L = w.layers
-    B = args.batch
-    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
-    layers = []
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, w.rank, 1)
+    built = []
     t0 = time.time()
     for l in range(L):
         lw = synth.layer_weights(w, l)
         pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
-        layers.append(msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev))
+        built.append(msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev))
         del lw, pk
     setup_s = time.time() - t0
+    grid = [(args.k, args.batch)]
+    if args.stack_grid:
+        grid = [(k, b) for b in (1, 32) for k in (100, 138, w.inter)]
+    for k, B in grid:
+        r = 0 if k == w.inter else w.rank
+        layers = built if r == w.rank else [lay.without_lowrank() for lay in built]
+        run_stack_one(args, w, local, dev, layers, k, B, r, setup_s)
+
+
+def run_stack_one(args, w, local, dev, layers, k, B, rank, setup_s):
+    import torch
+    import token_top_expert_b200 as msb
+    L = w.layers
+    dims = layers[0].dims
     nseq = 16
     h0 = torch.from_numpy(np.stack([synth.stack_initial_hidden(w, s, B) for s in range(nseq)])).to(dev)
     h = torch.empty((B, w.d), dtype=torch.float32, device=dev)
@@ -239,26 +252,26 @@ def run_stack(args, w, world, rank, local):
     yb = torch.empty_like(xb)
     ws = msb.Workspace(dims, B, dev)
     stream = torch.cuda.Stream(dev)
-    dense = args.k == w.inter
+    dense = k == w.inter
 
     def step(s, trace=None):
         h.copy_(h0[s % nseq])
         for l in range(L):
             msb.residual_rmsnorm(h, yb if l > 0 else None, xb, stream=stream)
-            msb.moe_sparse_block(xb, layers[l], args.k, out=yb, workspace=ws, trace=trace,
+            msb.moe_sparse_block(xb, layers[l], k, out=yb, workspace=ws, trace=trace,
                                  stream=stream)
         msb.residual_rmsnorm(h, yb, xb, stream=stream)
 
     # bytes of one step, from traced calls
-    tr = msb.Trace(dims, B, args.k)
+    tr = msb.Trace(dims, B, k)
     byts = 0
     with torch.cuda.stream(stream):
         h.copy_(h0[0])
         for l in range(L):
             msb.residual_rmsnorm(h, yb if l > 0 else None, xb, stream=stream)
-            msb.moe_sparse_block(xb, layers[l], args.k, out=yb, workspace=ws, trace=tr, stream=stream)
+            msb.moe_sparse_block(xb, layers[l], k, out=yb, workspace=ws, trace=tr, stream=stream)
             stream.synchronize()
-            byts += algorithmic_bytes(w, args.k, args.rank, tr.union_count.cpu().tolist(), dense)
+            byts += algorithmic_bytes(w, k, rank, tr.union_count.cpu().tolist(), dense)
         for i in range(args.warmup):
             step(i)
     stream.synchronize()
@@ -285,13 +298,14 @@ def run_stack(args, w, world, rank, local):
     ms_per_step = ms / steps
     peak, peak_kind = peaks()
     achieved = byts / (ms_per_step * 1e-3) / 1e9
-    plan = msb.path_info(dims, B, args.k)
+    plan = msb.path_info(dims, B, k)
     line = {
         "metric": "stacked MoE decode tokens/s (%d layers)" % L, "value": steps * B / (ms / 1e3),
         "unit": "tokens/s", "n_gpus": 1, "steps": steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (per-layer seeded BF16 weights; h0 ~ N(0,1))",
-        "config": dict(config_of(w, args), layers=L, path=plan,
+        "config": dict(config_of(w, args), k=k, budget=round(k / w.inter, 4), rank=rank, global_batch=B,
+                       batch_per_gpu=B, replicas=1, layers=L, path=plan,
                        l2="inputs larger than L2: %.1f GB of packed weights" %
                           (sum(x.nbytes() for x in layers) / 1e9)),
         "us_per_layer": ms_per_step * 1e3 / L, "bytes_per_step": byts,
@@ -384,6 +398,8 @@ def main():
     ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--stack-grid", action="store_true",
+                    help="stacked workload: run k in {13%%, 18%%, 100%%} x batch in {1, 32} on one set of layers")
     ap.add_argument("--threshold", action="store_true",
                     help="measure the calibrated-threshold comparator instead of top-k")
     args = ap.parse_args()

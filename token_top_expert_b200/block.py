@@ -104,6 +104,12 @@ class PackedLayer:
         return PackedLayer(self.dims, c(self.records), c(self.sketch), c(self.alpha),
                            c(self.router_t), c(self.lr_a), c(self.lr_b))
 
+    def without_lowrank(self) -> "PackedLayer":
+        """The same weights (shared, not copied) with rank 0: no compensation term."""
+        d = self.dims
+        return PackedLayer(Dims(d.d, d.inter, d.experts, d.top_e, 0, d.renorm), self.records,
+                           self.sketch, self.alpha, self.router_t, None, None)
+
     def nbytes(self) -> int:
         return sum(a.numel() * a.element_size() for a in
                    (self.records, self.sketch, self.alpha, self.router_t, self.lr_a, self.lr_b)

@@ -311,8 +311,10 @@ __device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, ui
 }
 
 // Sketch scores of this CTA's nt row tiles: warp w takes chunks [kc0, kc1) of every
-// tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B.
-// Partial sums go to part[warp][tile*16 + row].
+// tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B (every
+// column of B holds x; only column 0 of D is read).  Four accumulators, one per
+// 16-column step of a chunk, chain through the chunks.  Partial sums go to
+// part[warp][tile*16 + row].
 __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm, int nt, int KC,
                                          float* part_w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -321,15 +323,12 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
   const uint4* xp = xperm + c * 2;
 #pragma unroll 1
   for (int tl = 0; tl < nt; ++tl) {
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 2
+    float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
+    float m2[4] = {0.f, 0.f, 0.f, 0.f}, m3[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int kc = kc0; kc < kc1; ++kc) {
       const uint2 w = codes[((size_t)tl * KC + kc) * 32 + lane];
-      uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
-      if (g == 0) { xa = xp[kc * 8]; xb = xp[kc * 8 + 1]; }
-      // four independent 16-column steps (no accumulator chain between them)
-      float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
-      float m2[4] = {0.f, 0.f, 0.f, 0.f}, m3[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint4 xa = xp[kc * 8], xb = xp[kc * 8 + 1];
       mma_bf16(m0, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
                (w.y << 2) & kSketchMask, xa.x, xa.y);
       mma_bf16(m1, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
@@ -338,12 +337,10 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
                (w.y << 10) & kSketchMask, xb.x, xb.y);
       mma_bf16(m3, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask, (w.x << 14) & kSketchMask,
                (w.y << 14) & kSketchMask, xb.z, xb.w);
-      acc0 += (m0[0] + m1[0]) + (m2[0] + m3[0]);
-      acc1 += (m0[2] + m1[2]) + (m2[2] + m3[2]);
     }
     if (c == 0) {
-      part_w[tl * kRowTile + g] = acc0;
-      part_w[tl * kRowTile + g + 8] = acc1;
+      part_w[tl * kRowTile + g] = (m0[0] + m1[0]) + (m2[0] + m3[0]);
+      part_w[tl * kRowTile + g + 8] = (m0[2] + m1[2]) + (m2[2] + m3[2]);
     }
   }
 }
@@ -545,12 +542,12 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   // ------------------------------------------------------------------ phase C: top-k, records
   // this CTA's share of the k channels: positions [c0, c1) of the ascending list
   const int NQ = CS * P.cpe, gq = half * CS + q;
-  const int c0 = (int)((long)gq * P.k / NQ), c1 = (int)((long)(gq + 1) * P.k / NQ);
+  const int c0 = gq * P.k / NQ, c1 = (gq + 1) * P.k / NQ;
   const int nmine = c1 - c0;
   if (!P.dense) {
     uint32_t maxkey = 0;
-#pragma unroll 1
-    for (int i = 0; i < CS; ++i) maxkey = max(maxkey, M.cmax[i]);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) maxkey = i < CS ? max(maxkey, M.cmax[i]) : maxkey;
     uint16_t* trace = (half == 0 && q == 0 && P.tr.sel) ? P.tr.sel + (size_t)rc * P.k : nullptr;
     select_share(keys, I, P.k, maxkey, hist, M, c0, c1, trace);
     if (half == 0 && q == 0 && tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
@@ -561,15 +558,14 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   }
   const uint32_t rec_bytes = 6u * d;
   uint16_t* ring = reinterpret_cast<uint16_t*>(big);
-  if (tid == 0 && ok) {
+  if (warp == 0 && ok) {  // lane i issues the copy into slot i
     fence_proxy_async();
     const int first = min(P.ring, nmine);
-#pragma unroll 1
-    for (int i = 0; i < first; ++i) {
-      const int ch = M.mysel[i];
-      mbar_arrive_expect_tx(&M.bar[2 + i], rec_bytes);
-      bulk_g2s(ring + (size_t)i * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
-               &M.bar[2 + i]);
+    if (lane < first) {
+      const int ch = M.mysel[lane];
+      mbar_arrive_expect_tx(&M.bar[2 + lane], rec_bytes);
+      bulk_g2s(ring + (size_t)lane * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
+               &M.bar[2 + lane]);
     }
   }
   // A_e z on this CTA's output slice, while the records are in flight
@@ -618,18 +614,25 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   for (int it = 0; it < IT; ++it)
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
+  // channel g0 + i of a group sits in slot s0 + i (wrapping at the ring size, where the
+  // slot's phase parity flips); s0 and its parity par0 advance group by group
+  int s0 = 0;
+  uint32_t par0 = 0;
 #pragma unroll 1
   for (int g0 = 0; g0 < nmine; g0 += P.group) {
     const int ng = min(P.group, nmine - g0);
 #pragma unroll 1
-    for (int i = 0; i < ng; ++i)
-      ok = ok && wait_phase(&M.bar[2 + (g0 + i) % P.ring], ((g0 + i) / P.ring) & 1u, P.err);
+    for (int i = 0; i < ng; ++i) {
+      const int sl = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
+      ok = ok && wait_phase(&M.bar[2 + sl], s0 + i < P.ring ? par0 : par0 ^ 1u, P.err);
+    }
 #pragma unroll 1
     for (int tb = 0; tb < ng; tb += 8) {
       // this lane's ldmatrix row: channel tb + lane % 8 (rows past ng repeat channel tb;
       // their results are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 * (lane / 16)
       const int ch = (tb + (lane & 7) < ng) ? tb + (lane & 7) : tb;
-      uint32_t a_addr = smem_addr(ring + (size_t)((g0 + ch) % P.ring) * P.rs + ((lane >> 3) & 1) * d +
+      const int csl = s0 + ch < P.ring ? s0 + ch : s0 + ch - P.ring;
+      uint32_t a_addr = smem_addr(ring + (size_t)csl * P.rs + ((lane >> 3) & 1) * d +
                                   8 * (lane >> 4)) + 32u * ks0;
       float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
       int ks = ks0;
@@ -673,7 +676,8 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
       // y += h_i * down_i over this thread's elements
 #pragma unroll 4
       for (int i = 0; i < ng; ++i) {
-        const uint16_t* rec = ring + (size_t)((g0 + i) % P.ring) * P.rs + 2 * d;
+        const int sl = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
+        const uint16_t* rec = ring + (size_t)sl * P.rs + 2 * d;
         const float h = M.h[i];
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
@@ -694,19 +698,21 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
     __syncthreads();
     // refill the slots just consumed
-    if (tid == 0 && ok) {
+    if (warp == 0 && ok) {  // channel g0 + i + ring goes where g0 + i was; lane i issues it
       fence_proxy_async();
-#pragma unroll 1
-      for (int i = g0; i < g0 + ng; ++i) {
-        const int nx = i + P.ring;
-        if (nx < nmine) {
-          const int ch = M.mysel[nx];
-          const int slot = nx % P.ring;
-          mbar_arrive_expect_tx(&M.bar[2 + slot], rec_bytes);
-          bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
-                   &M.bar[2 + slot]);
-        }
+      const int i = lane, nx = g0 + lane + P.ring;
+      if (i < ng && nx < nmine) {
+        const int ch = M.mysel[nx];
+        const int slot = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
+        mbar_arrive_expect_tx(&M.bar[2 + slot], rec_bytes);
+        bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
+                 &M.bar[2 + slot]);
       }
+    }
+    s0 += ng;
+    if (s0 >= P.ring) {
+      s0 -= P.ring;
+      par0 ^= 1u;
     }
   }
 
