@@ -390,37 +390,70 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
 // =====================================================================================
 // gathered channel records -> SwiGLU -> down; low-rank A_e z; weighted reduction
 // =====================================================================================
-// Dynamic shared memory: records [CH][3d] bf16 | xs [TG][d] bf16 | small scratch.
+// Each chunk CTA takes up to kGCh channels of one expert's union list and every token
+// routed to that expert, 8 tokens at a time, on the tensor cores:
+//   gate/up   D[16 rows][8 tokens] = [gate rows | up rows] (ldmatrix from the records
+//             in shared memory) x the tokens' x rows (B fragments read through L1);
+//             warp w takes k-steps [w KS/8, (w+1) KS/8), the warps' partials meet in
+//             shared memory;
+//   h         silu(g) u, times the pair's selection bit and router weight;
+//   down      D[16][8 columns] = [h_hi ; h_lo] (8 tokens x 16 channels, h split into
+//             two bf16 halves so that the product keeps ~16 significant bits) x the
+//             records' down columns (ldmatrix.trans), rows t and t+8 summed into the
+//             FP32 accumulator of token t with 8-byte reduction-adds.
+// Dynamic shared memory: records [ch][3d + 8] bf16 (16 bytes of stagger per slot).
 struct GatherCfg {
-  int ch;       // channels per CTA
-  int tg;       // tokens per pass
+  int ch;       // channels per CTA (<= kGCh)
   int nchunk;   // channel-chunk CTAs per slot
   int nlr;      // low-rank CTAs per slot
   int dense;    // 1: every channel is selected (no sketch)
 };
+constexpr int kGCh = 8;
 
-template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
-__global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict__ x,
-                                                     const uint16_t* __restrict__ records,
-                                                     const uint16_t* __restrict__ lr_a, Dims D,
-                                                     Workspace ws, GatherCfg cfg) {
-  constexpr int TG = 8 / IT;  // tokens per pass
-  extern __shared__ __align__(16) uint8_t gsm[];
+__device__ __forceinline__ void red_add_v2(float* dst, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1,%2};" ::"l"(dst), "f"(a), "f"(b) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r0), "=r"(r1)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(lo)) |
+         ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
+}
+
+__global__ void __launch_bounds__(kNT, 2) gather_kernel(const uint16_t* __restrict__ x,
+                                                        const uint16_t* __restrict__ records,
+                                                        const uint16_t* __restrict__ lr_a, Dims D,
+                                                        Workspace ws, GatherCfg cfg) {
+  extern __shared__ __align__(128) uint8_t gsm[];
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_list[64];
+  __shared__ int s_list[kGCh];
   __shared__ int s_n;
-  __shared__ float s_red[kNT / 32][2 * 8];
-  __shared__ float s_h[64][8];
+  __shared__ int s_tok[8];
+  __shared__ float s_w[8];
+  __shared__ float s_red[kNT / 32][16][8];
+  __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels 8..15 zero
   const int u = blockIdx.y;
   if (u >= *ws.nused) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = D.d, I = D.inter, ipad = D.ipad, r = D.rank;
   const int e = ws.slot_expert[u];
   const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
 
   // ------------------------------------------------------------- low-rank CTAs
   if ((int)blockIdx.x >= cfg.nchunk) {
-    const int row = ((int)blockIdx.x - cfg.nchunk) * kLrRows + threadIdx.x;
+    const int row = ((int)blockIdx.x - cfg.nchunk) * kLrRows + tid;
     if (row >= d || r == 0) return;
     const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
     for (int ti = 0; ti < cnt; ++ti) {
@@ -435,10 +468,10 @@ __global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict_
 
   // ------------------------------------------------------------- this chunk's channels
   const int c0 = blockIdx.x * cfg.ch;
-  if (threadIdx.x < 32) {
+  if (tid < 32) {
     if (cfg.dense) {
       if (lane == 0) s_n = max(0, min(cfg.ch, I - c0));
-      for (int i = lane; i < cfg.ch; i += 32) s_list[i] = c0 + i;
+      if (lane < cfg.ch) s_list[lane] = c0 + lane;
     } else {
       const int nw = mask_words(ipad);
       const uint32_t* um = ws.umask + (size_t)u * nw;
@@ -475,116 +508,120 @@ __global__ void __launch_bounds__(kNT) gather_kernel(const uint16_t* __restrict_
   if (nch == 0) return;
 
   uint16_t* rec = reinterpret_cast<uint16_t*>(gsm);
-  uint16_t* xs = rec + (size_t)cfg.ch * 3 * d;
+  const int rs = 3 * d + 8;  // slot stride (elements)
   const uint32_t rec_bytes = 6u * d;
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     mbar_init(&bar, 1);
     fence_mbar_init();
     mbar_arrive_expect_tx(&bar, rec_bytes * nch);
     for (int i = 0; i < nch; ++i)
-      bulk_g2s(rec + (size_t)i * 3 * d, records + ((size_t)e * I + s_list[i]) * 3 * d, rec_bytes, &bar);
+      bulk_g2s(rec + (size_t)i * rs, records + ((size_t)e * I + s_list[i]) * 3 * d, rec_bytes, &bar);
   }
-  // token x rows are staged per token group below; wait for the records first
+  for (int i = tid; i < 8 * 2 * kGCh; i += kNT) (&s_h[0][0])[i] = 0.f;
   __syncthreads();
   if (!mbar_wait(&bar, 0, ws.err)) {
     mbar_wait(&bar, 0, ws.err);
     return;
   }
 
-  for (int tg0 = 0; tg0 < cnt; tg0 += cfg.tg) {
-    const int ntg = min(cfg.tg, cnt - tg0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < ntg * d / 8; i += kNT) {
-      const int n = i / (d / 8), q = i % (d / 8);
-      const int t = ws.pair_tok[off + tg0 + n];
-      reinterpret_cast<uint4*>(xs + (size_t)n * d)[q] =
-          __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + q);
+  const int c4 = lane & 3, g8 = lane >> 2;
+  const int KS = d / 16;
+  const int ks0 = warp * KS / (kNT / 32), ks1 = (warp + 1) * KS / (kNT / 32);
+  // gate/up ldmatrix row of this lane: channel lane % 8 (channels past nch repeat
+  // channel 0; their rows are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 (lane / 16)
+  const int gch = (lane & 7) < nch ? (lane & 7) : 0;
+  const uint32_t a_base =
+      smem_addr(rec + (size_t)gch * rs + ((lane >> 3) & 1) * d + 8 * (lane >> 4)) + 32u * ks0;
+  // down ldmatrix.trans row of this lane: channel lane % 8 (channels 8..15 of the k-step
+  // and channels past nch read channel 0; their h is zero), element block 8 (lane / 16)
+  const int dch = (lane & 7) < nch ? (lane & 7) : 0;
+  const uint32_t b_base = smem_addr(rec + (size_t)dch * rs + 2 * d + 8 * (lane >> 4));
+  const int NTW = d / 64;  // 8-column output tiles per warp
+  const int nt0 = warp * NTW;
+  const int nmw = mask_words(ipad);
+
+  for (int tg0 = 0; tg0 < cnt; tg0 += 8) {
+    const int ntg = min(8, cnt - tg0);
+    __syncthreads();  // s_tok, s_w, s_h of the previous token group are free
+    if (tid < 8) {
+      const int p = off + tg0 + min(tid, ntg - 1);
+      s_tok[tid] = ws.pair_tok[p];
+      s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
     }
     __syncthreads();
-    float y[TG][IT * 8];
-#pragma unroll
-    for (int n = 0; n < TG; ++n)
-#pragma unroll
-      for (int i = 0; i < IT * 8; ++i) y[n][i] = 0.f;
-
-    for (int ci = 0; ci < nch; ++ci) {
-      const int j = s_list[ci];
-      const uint16_t* grow = rec + (size_t)ci * 3 * d;
-      const uint16_t* urow = grow + d;
-      const uint16_t* drow = grow + 2 * d;
-      float pg[TG], pu[TG];
-#pragma unroll
-      for (int n = 0; n < TG; ++n) { pg[n] = 0.f; pu[n] = 0.f; }
-#pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        const int el = (it * kNT + threadIdx.x) * 8;
-        if (el < d) {
-          const uint4 gv = *reinterpret_cast<const uint4*>(grow + el);
-          const uint4 uv = *reinterpret_cast<const uint4*>(urow + el);
-#pragma unroll
-          for (int n = 0; n < TG; ++n)
-            if (n < ntg) {
-              const uint4 xv = *reinterpret_cast<const uint4*>(xs + (size_t)n * d + el);
-              pg[n] = dot8(gv, xv, pg[n]);
-              pu[n] = dot8(uv, xv, pu[n]);
-            }
-        }
+    // ---- gate/up partials over this warp's k-steps
+    {
+      const uint32_t* xrow = reinterpret_cast<const uint32_t*>(x + (size_t)s_tok[g8] * d);
+      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t a_addr = a_base;
+      int ks = ks0;
+      for (; ks + 2 <= ks1; ks += 2, a_addr += 64u) {
+        uint32_t a[2][4];
+        ldsm_x4(a_addr, a[0][0], a[0][1], a[0][2], a[0][3]);
+        ldsm_x4(a_addr + 32u, a[1][0], a[1][1], a[1][2], a[1][3]);
+        const uint32_t b00 = __ldg(xrow + ks * 8 + c4), b01 = __ldg(xrow + ks * 8 + 4 + c4);
+        const uint32_t b10 = __ldg(xrow + ks * 8 + 8 + c4), b11 = __ldg(xrow + ks * 8 + 12 + c4);
+        mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b00, b01);
+        mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b10, b11);
       }
+      if (ks < ks1) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(a_addr, a0, a1, a2, a3);
+        mma_bf16(acc0, a0, a1, a2, a3, __ldg(xrow + ks * 8 + c4), __ldg(xrow + ks * 8 + 4 + c4));
+      }
+      s_red[warp][g8][2 * c4] = acc0[0] + acc1[0];
+      s_red[warp][g8][2 * c4 + 1] = acc0[1] + acc1[1];
+      s_red[warp][g8 + 8][2 * c4] = acc0[2] + acc1[2];
+      s_red[warp][g8 + 8][2 * c4 + 1] = acc0[3] + acc1[3];
+    }
+    __syncthreads();
+    // ---- h[token][channel] = silu(g) u, times the selection bit and the router weight
+    if (tid < 8 * kGCh) {
+      const int c = tid & (kGCh - 1), t = tid / kGCh;
+      float h = 0.f;
+      if (c < nch && t < ntg) {
+        float g = 0.f, uu = 0.f;
 #pragma unroll
-      for (int n = 0; n < TG; ++n)
-        if (n < ntg) {
-          const float a = warp_sum(pg[n]);
-          const float b = warp_sum(pu[n]);
-          if (lane == 0) { s_red[warp][2 * n] = a; s_red[warp][2 * n + 1] = b; }
-        }
-      __syncthreads();
-      if (threadIdx.x < ntg) {
-        const int n = threadIdx.x;
-        float gsum = 0.f, usum = 0.f;
-        for (int w = 0; w < kNT / 32; ++w) { gsum += s_red[w][2 * n]; usum += s_red[w][2 * n + 1]; }
+        for (int w = 0; w < kNT / 32; ++w) { g += s_red[w][c][t]; uu += s_red[w][8 + c][t]; }
         bool selected = true;
         if (!cfg.dense) {
-          const int p = off + tg0 + n;
-          selected = (__ldcg(&ws.selmask[(size_t)p * mask_words(ipad) + (j >> 5)]) >> (j & 31)) & 1u;
+          const int p = off + tg0 + t, j = s_list[c];
+          selected = (__ldcg(&ws.selmask[(size_t)p * nmw + (j >> 5)]) >> (j & 31)) & 1u;
         }
-        s_h[ci][n] = selected ? silu(gsum) * usum : 0.f;
+        h = selected ? silu(g) * uu * s_w[t] : 0.f;
       }
-      __syncthreads();
-#pragma unroll
-      for (int it = 0; it < IT; ++it) {
-        const int el = (it * kNT + threadIdx.x) * 8;
-        if (el < d) {
-          const uint4 dv = *reinterpret_cast<const uint4*>(drow + el);
-          const float dd[8] = {bf16_lo(dv.x), bf16_hi(dv.x), bf16_lo(dv.y), bf16_hi(dv.y),
-                               bf16_lo(dv.z), bf16_hi(dv.z), bf16_lo(dv.w), bf16_hi(dv.w)};
-#pragma unroll
-          for (int n = 0; n < TG; ++n)
-            if (n < ntg) {
-              const float h = s_h[ci][n];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) y[n][it * 8 + i] = fmaf(h, dd[i], y[n][it * 8 + i]);
-            }
-        }
+      s_h[t][c] = h;
+    }
+    __syncthreads();
+    // ---- down: A = [h_hi ; h_lo] (token rows), B = down columns, this warp's column tiles
+    const float2 hp = *reinterpret_cast<const float2*>(&s_h[g8][2 * c4]);
+    const uint32_t ahi = pack_bf16x2(hp.x, hp.y);
+    const float2 hhi = make_float2(__bfloat162float(__ushort_as_bfloat16((uint16_t)(ahi & 0xffffu))),
+                                   __bfloat162float(__ushort_as_bfloat16((uint16_t)(ahi >> 16))));
+    const uint32_t alo = pack_bf16x2(hp.x - hhi.x, hp.y - hhi.y);
+    float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
+    const bool tok_ok = g8 < ntg;
+    int nt = 0;
+    for (; nt + 2 <= NTW; nt += 2) {
+      const int m0 = (nt0 + nt) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
+      float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
+      mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
+      if (tok_ok) {
+        red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+        red_add_v2(yrow + m0 + 8 + 2 * c4, dB[0] + dB[2], dB[1] + dB[3]);
       }
     }
-    // weighted reduction into the FP32 accumulator
-#pragma unroll
-    for (int n = 0; n < TG; ++n)
-      if (n < ntg) {
-        const int p = off + tg0 + n;
-        const float w = ws.pair_w[p];
-        float* dst = ws.y_acc + (size_t)ws.pair_tok[p] * d;
-#pragma unroll
-        for (int it = 0; it < IT; ++it) {
-          const int el = (it * kNT + threadIdx.x) * 8;
-          if (el < d) {
-            red_add_v4(dst + el, w * y[n][it * 8 + 0], w * y[n][it * 8 + 1], w * y[n][it * 8 + 2],
-                       w * y[n][it * 8 + 3]);
-            red_add_v4(dst + el + 4, w * y[n][it * 8 + 4], w * y[n][it * 8 + 5],
-                       w * y[n][it * 8 + 6], w * y[n][it * 8 + 7]);
-          }
-        }
-      }
+    if (nt < NTW) {
+      const int m0 = (nt0 + nt) * 8;
+      uint32_t b0, b1;
+      ldsm_x2_t(b_base + 2u * m0, b0, b1);
+      float dA[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
+      if (tok_ok) red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+    }
   }
 }
 
@@ -648,20 +685,13 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   }
   if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
   GatherCfg cfg;
-  const int IT = (d + 2047) / 2048;
-  const int ITc = IT <= 1 ? 1 : IT <= 2 ? 2 : 4;
-  cfg.tg = 8 / ITc;
-  cfg.ch = max(1, min(64, (96 * 1024) / (6 * d)));
+  cfg.ch = max(1, min(kGCh, (200 * 1024) / (6 * d + 16)));
   cfg.nchunk = (D.inter + cfg.ch - 1) / cfg.ch;
   cfg.nlr = D.rank > 0 ? (d + kLrRows - 1) / kLrRows : 0;
   cfg.dense = dense;
-  const size_t gsmem = (size_t)cfg.ch * 6 * d + (size_t)cfg.tg * 2 * d;
+  const size_t gsmem = (size_t)cfg.ch * (6 * d + 16);
   dim3 ggrid(cfg.nchunk + cfg.nlr, maxslots);
-  switch (ITc) {
-    case 1: gather_kernel<1><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
-    case 2: gather_kernel<2><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
-    default: gather_kernel<4><<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg); break;
-  }
+  gather_kernel<<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
   {
     const size_t n8 = (size_t)B * d / 8;
     const size_t nb = (n8 + kNT - 1) / kNT;
@@ -676,11 +706,7 @@ int general_set_smem_limits() {
   cudaError_t e = cudaSuccess;
   e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-  if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-  if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 
