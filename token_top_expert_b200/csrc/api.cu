@@ -44,7 +44,7 @@ Dims to_dims(const msb_dims& m) {
 // Byte offsets of every workspace array for a batch of B tokens.
 struct Layout {
   size_t err, counters, y_acc, logits, ids, wts, slot_expert, slot_off, nused, pair_tok, pair_w,
-      pair_slot, pair_of, scores, selmask, sel, selcnt, umask, z, total;
+      pair_slot, pair_of, scores, selmask, sel, selcnt, umask, z, ulist, ucnt, coff, total;
 };
 
 Layout layout(const Dims& D, int B) {
@@ -70,6 +70,9 @@ Layout layout(const Dims& D, int B) {
   L.selcnt = o;        o = up(o + 4 * P);
   L.umask = o;         o = up(o + 4 * E * mask_words(D.ipad));
   L.z = o;             o = up(o + 4 * P * (size_t)(D.rank > 0 ? D.rank : 1));
+  L.ulist = o;         o = up(o + 2 * E * D.ipad);
+  L.ucnt = o;          o = up(o + 4 * E);
+  L.coff = o;          o = up(o + 4 * (E + 1));
   L.total = o;
   return L;
 }
@@ -96,6 +99,9 @@ Workspace bind(void* base, const Layout& L) {
   w.selcnt = reinterpret_cast<int32_t*>(b + L.selcnt);
   w.umask = reinterpret_cast<uint32_t*>(b + L.umask);
   w.z = reinterpret_cast<float*>(b + L.z);
+  w.ulist = reinterpret_cast<uint16_t*>(b + L.ulist);
+  w.ucnt = reinterpret_cast<int32_t*>(b + L.ucnt);
+  w.coff = reinterpret_cast<int32_t*>(b + L.coff);
   return w;
 }
 

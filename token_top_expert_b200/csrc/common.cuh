@@ -204,6 +204,9 @@ struct Workspace {
   int32_t* selcnt;      // [B*K]
   uint32_t* umask;      // [E][Ipad/32] union of the selections of each slot
   float* z;             // [B*K][r]  B_e x
+  uint16_t* ulist;      // [E][Ipad] ascending union list of each slot
+  int32_t* ucnt;        // [E] union size of each slot
+  int32_t* coff;        // [E+1] first gather work item (channel chunk) of each slot
 };
 
 constexpr int kCounters = 1024;
@@ -211,6 +214,9 @@ constexpr int kCounters = 1024;
 constexpr int kCntRouterAll = 1;      // router: token groups finished
 constexpr int kCntRouterGroup = 8;    // router: CTAs finished per token group (32 groups)
 constexpr int kCntFusedSlices = 64;   // single-launch path: contributions per output slice (16)
+constexpr int kCntGatherWork = 2;     // multi-kernel path: next gather work item
+constexpr int kCntUnion = 3;          // multi-kernel path: union CTAs finished
+constexpr int kCntGatherRun = 4;      // multi-kernel path: union channels per gather work item
 
 struct Dims {
   int d, inter, ipad, experts, top_e, rank, renorm;

@@ -21,7 +21,11 @@ constexpr int kNT = 256;          // threads per CTA in every general kernel
 constexpr int kRouterTok = 8;     // tokens per router CTA
 constexpr int kScoreRows = 64;    // sketch rows per score CTA (4 tensor-core row tiles)
 constexpr int kScoreTok = 8;      // tokens per MMA n-tile
-constexpr int kLrRows = 256;      // A_e rows per low-rank CTA
+constexpr int kLrRows = 256;      // A_e rows per low-rank work item
+constexpr int kGCh = 8;           // gather: channels per stage at most (one m-tile of gate/up rows)
+constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in flight)
+constexpr int kGRunStages = 8;    // gather: stages per work item at most
+constexpr int kGAccTiles = 32;    // gather: output column tiles per warp held in registers
 
 // =====================================================================================
 // router
@@ -388,6 +392,62 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
 }
 
 // =====================================================================================
+// union lists: the ascending list of each slot's union bitmap, and the prefix of the
+// slots' channel chunks (the gather kernel's work items)
+// =====================================================================================
+__global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch, int ngrid, int dense) {
+  __shared__ uint32_t s_tmp[kNT / 32 + 1];
+  __shared__ int s_last;
+  const int tid = threadIdx.x;
+  const int u = blockIdx.x, nu = *ws.nused;
+  if (u < nu) {
+    int n = D.inter;
+    if (!dense) {
+      const int nw = mask_words(D.ipad);  // <= 128 words, one per thread
+      const uint32_t w = tid < nw ? __ldcg(&ws.umask[(size_t)u * nw + tid]) : 0u;
+      uint32_t tot;
+      uint32_t rank = block_excl_scan<kNT>((uint32_t)__popc(w), s_tmp, &tot);
+      uint16_t* dst = ws.ulist + (size_t)u * D.ipad;
+      for (uint32_t b = w; b; b &= b - 1) dst[rank++] = (uint16_t)(tid * 32 + __ffs(b) - 1);
+      n = (int)tot;
+    }
+    if (tid == 0) ws.ucnt[u] = n;
+  }
+  // the last CTA: chunk prefix over the used slots, and a fresh work counter
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(&ws.counters[kCntUnion], 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // run length: a multiple of the stage size ch, about two runs per CTA of the grid,
+  // at most kGRunStages stages (longer runs mean fewer reduction-adds per output)
+  uint32_t n2[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+    if (2 * tid + i < nu) n2[i] = (uint32_t)__ldcg(&ws.ucnt[2 * tid + i]);
+  uint32_t all;
+  block_excl_scan<kNT>(n2[0] + n2[1], s_tmp, &all);
+  int run = (int)((all + 2u * ngrid - 1) / (2u * ngrid));
+  run = min(kGRunStages * ch, max(ch, (run + ch - 1) / ch * ch));
+  uint32_t c[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 2; ++i) c[i] = (n2[i] + run - 1) / run;
+  uint32_t tot;
+  const uint32_t pre = block_excl_scan<kNT>(c[0] + c[1], s_tmp, &tot);
+  if (2 * tid < nu) ws.coff[2 * tid] = (int)pre;
+  if (2 * tid + 1 < nu) ws.coff[2 * tid + 1] = (int)(pre + c[0]);
+  if (tid == 0) {
+    ws.coff[nu] = (int)tot;
+    ws.counters[kCntGatherRun] = (uint32_t)run;
+    ws.counters[kCntGatherWork] = 0u;
+    ws.counters[kCntUnion] = 0u;
+  }
+}
+
+// =====================================================================================
 // gathered channel records -> SwiGLU -> down; low-rank A_e z; weighted reduction
 // =====================================================================================
 // Each chunk CTA takes up to kGCh channels of one expert's union list and every token
@@ -403,12 +463,10 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
 //             FP32 accumulator of token t with 8-byte reduction-adds.
 // Dynamic shared memory: records [ch][3d + 8] bf16 (16 bytes of stagger per slot).
 struct GatherCfg {
-  int ch;       // channels per CTA (<= kGCh)
-  int nchunk;   // channel-chunk CTAs per slot
-  int nlr;      // low-rank CTAs per slot
+  int ch;       // channels per work item (<= kGCh)
+  int nlr;      // low-rank work items per slot
   int dense;    // 1: every channel is selected (no sketch)
 };
-constexpr int kGCh = 8;
 
 __device__ __forceinline__ void red_add_v2(float* dst, float a, float b) {
   asm volatile("red.global.add.v2.f32 [%0], {%1,%2};" ::"l"(dst), "f"(a), "f"(b) : "memory");
@@ -432,195 +490,294 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
 }
 
-__global__ void __launch_bounds__(kNT, 2) gather_kernel(const uint16_t* __restrict__ x,
+// Issue the bulk copies of channels run[c0 .. c0 + n) (shared memory) into a stage buffer.
+__device__ __forceinline__ void gather_issue(uint16_t* buf, const uint16_t* records, const int* run,
+                                             int e, int c0, int n, int d, int I, int* list,
+                                             uint64_t* bar) {
+  const int rs = 3 * d + 8;
+  fence_proxy_async();
+  mbar_arrive_expect_tx(bar, 6u * d * n);
+  for (int i = 0; i < n; ++i) {
+    const int j = run[c0 + i];
+    list[i] = j;
+    bulk_g2s(buf + (size_t)i * rs, records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
+  }
+}
+
+// REGACC: d <= 64 * kGAccTiles, outputs held in registers over a run.
+// KSW: the x B-fragments of this warp's k-steps held in registers per token group
+// (d <= 128 * KSW); 0: read through L1/L2 at every stage.
+// Stages of cfg.ch channels stream through kGBufs buffers, kGBufs - 1 of them in flight
+// while one is computed.
+template <bool REGACC, int KSW>
+__global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restrict__ x,
                                                         const uint16_t* __restrict__ records,
                                                         const uint16_t* __restrict__ lr_a, Dims D,
                                                         Workspace ws, GatherCfg cfg) {
   extern __shared__ __align__(128) uint8_t gsm[];
-  __shared__ __align__(8) uint64_t bar;
-  __shared__ int s_list[kGCh];
-  __shared__ int s_n;
+  __shared__ __align__(8) uint64_t bar[kGBufs];
+  __shared__ int s_item, s_u;
+  __shared__ int s_list[kGBufs][kGCh];
+  __shared__ int s_run[kGRunStages * kGCh];  // channel indices of the current run
   __shared__ int s_tok[8];
   __shared__ float s_w[8];
   __shared__ float s_red[kNT / 32][16][8];
-  __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels 8..15 zero
-  const int u = blockIdx.y;
-  if (u >= *ws.nused) return;
+  __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels >= ch zero
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = D.d, I = D.inter, ipad = D.ipad, r = D.rank;
-  const int e = ws.slot_expert[u];
-  const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
-
-  // ------------------------------------------------------------- low-rank CTAs
-  if ((int)blockIdx.x >= cfg.nchunk) {
-    const int row = ((int)blockIdx.x - cfg.nchunk) * kLrRows + tid;
-    if (row >= d || r == 0) return;
-    const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
-    for (int ti = 0; ti < cnt; ++ti) {
-      const int p = off + ti;
-      const float* z = ws.z + (size_t)p * r;
-      float acc = 0.f;
-      for (int q = 0; q < r; ++q) acc = fmaf(bf16_lo(arow[q]), __ldcg(z + q), acc);
-      atomicAdd(&ws.y_acc[(size_t)ws.pair_tok[p] * d + row], ws.pair_w[p] * acc);
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------- this chunk's channels
-  const int c0 = blockIdx.x * cfg.ch;
-  if (tid < 32) {
-    if (cfg.dense) {
-      if (lane == 0) s_n = max(0, min(cfg.ch, I - c0));
-      if (lane < cfg.ch) s_list[lane] = c0 + lane;
-    } else {
-      const int nw = mask_words(ipad);
-      const uint32_t* um = ws.umask + (size_t)u * nw;
-      const int per = (nw + 31) / 32;
-      uint32_t wv[4];
-      uint32_t pc = 0;
-      for (int i = 0; i < per; ++i) {
-        const int w = lane * per + i;
-        wv[i] = w < nw ? __ldcg(um + w) : 0u;
-        pc += __popc(wv[i]);
-      }
-      uint32_t inc = pc;
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
-      }
-      uint32_t rank = inc - pc;
-      const uint32_t total = __shfl_sync(0xffffffffu, inc, 31);
-      for (int i = 0; i < per; ++i) {
-        uint32_t b = wv[i];
-        while (b) {
-          const int bit = __ffs(b) - 1;
-          b &= b - 1;
-          if (rank >= (uint32_t)c0 && rank < (uint32_t)(c0 + cfg.ch))
-            s_list[rank - c0] = (lane * per + i) * 32 + bit;
-          ++rank;
-        }
-      }
-      if (lane == 0) s_n = max(0, min(cfg.ch, (int)total - c0));
-    }
-  }
-  __syncthreads();
-  const int nch = s_n;
-  if (nch == 0) return;
-
-  uint16_t* rec = reinterpret_cast<uint16_t*>(gsm);
+  const int nu = *ws.nused;
+  const int nchunks = __ldcg(&ws.coff[nu]);
+  const int run = (int)__ldcg(&ws.counters[kCntGatherRun]);
+  const int nitems = nchunks + nu * cfg.nlr;
   const int rs = 3 * d + 8;  // slot stride (elements)
-  const uint32_t rec_bytes = 6u * d;
+  const int CH = cfg.ch;
+  uint16_t* const buf0 = reinterpret_cast<uint16_t*>(gsm);
+  const size_t bstride = (size_t)CH * rs;  // stage buffer b at buf0 + b * bstride
   if (tid == 0) {
-    mbar_init(&bar, 1);
+#pragma unroll
+    for (int b = 0; b < kGBufs; ++b) mbar_init(&bar[b], 1);
     fence_mbar_init();
-    mbar_arrive_expect_tx(&bar, rec_bytes * nch);
-    for (int i = 0; i < nch; ++i)
-      bulk_g2s(rec + (size_t)i * rs, records + ((size_t)e * I + s_list[i]) * 3 * d, rec_bytes, &bar);
   }
   for (int i = tid; i < 8 * 2 * kGCh; i += kNT) (&s_h[0][0])[i] = 0.f;
-  __syncthreads();
-  if (!mbar_wait(&bar, 0, ws.err)) {
-    mbar_wait(&bar, 0, ws.err);
-    return;
-  }
-
+  uint32_t phases = 0;  // bit b: parity of buffer b's next completion
   const int c4 = lane & 3, g8 = lane >> 2;
   const int KS = d / 16;
   const int ks0 = warp * KS / (kNT / 32), ks1 = (warp + 1) * KS / (kNT / 32);
-  // gate/up ldmatrix row of this lane: channel lane % 8 (channels past nch repeat
-  // channel 0; their rows are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 (lane / 16)
-  const int gch = (lane & 7) < nch ? (lane & 7) : 0;
-  const uint32_t a_base =
-      smem_addr(rec + (size_t)gch * rs + ((lane >> 3) & 1) * d + 8 * (lane >> 4)) + 32u * ks0;
-  // down ldmatrix.trans row of this lane: channel lane % 8 (channels 8..15 of the k-step
-  // and channels past nch read channel 0; their h is zero), element block 8 (lane / 16)
-  const int dch = (lane & 7) < nch ? (lane & 7) : 0;
-  const uint32_t b_base = smem_addr(rec + (size_t)dch * rs + 2 * d + 8 * (lane >> 4));
   const int NTW = d / 64;  // 8-column output tiles per warp
   const int nt0 = warp * NTW;
   const int nmw = mask_words(ipad);
+  // h step ownership: thread tid < 8 * CH takes (token tid / CH, channel tid % CH)
+  const int hc = tid % CH, ht = tid / CH;
+  bool ok = true;
 
-  for (int tg0 = 0; tg0 < cnt; tg0 += 8) {
-    const int ntg = min(8, cnt - tg0);
-    __syncthreads();  // s_tok, s_w, s_h of the previous token group are free
-    if (tid < 8) {
-      const int p = off + tg0 + min(tid, ntg - 1);
-      s_tok[tid] = ws.pair_tok[p];
-      s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
-    }
-    __syncthreads();
-    // ---- gate/up partials over this warp's k-steps
-    {
-      const uint32_t* xrow = reinterpret_cast<const uint32_t*>(x + (size_t)s_tok[g8] * d);
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t a_addr = a_base;
-      int ks = ks0;
-      for (; ks + 2 <= ks1; ks += 2, a_addr += 64u) {
-        uint32_t a[2][4];
-        ldsm_x4(a_addr, a[0][0], a[0][1], a[0][2], a[0][3]);
-        ldsm_x4(a_addr + 32u, a[1][0], a[1][1], a[1][2], a[1][3]);
-        const uint32_t b00 = __ldg(xrow + ks * 8 + c4), b01 = __ldg(xrow + ks * 8 + 4 + c4);
-        const uint32_t b10 = __ldg(xrow + ks * 8 + 8 + c4), b11 = __ldg(xrow + ks * 8 + 12 + c4);
-        mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b00, b01);
-        mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b10, b11);
-      }
-      if (ks < ks1) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(a_addr, a0, a1, a2, a3);
-        mma_bf16(acc0, a0, a1, a2, a3, __ldg(xrow + ks * 8 + c4), __ldg(xrow + ks * 8 + 4 + c4));
-      }
-      s_red[warp][g8][2 * c4] = acc0[0] + acc1[0];
-      s_red[warp][g8][2 * c4 + 1] = acc0[1] + acc1[1];
-      s_red[warp][g8 + 8][2 * c4] = acc0[2] + acc1[2];
-      s_red[warp][g8 + 8][2 * c4 + 1] = acc0[3] + acc1[3];
-    }
-    __syncthreads();
-    // ---- h[token][channel] = silu(g) u, times the selection bit and the router weight
-    if (tid < 8 * kGCh) {
-      const int c = tid & (kGCh - 1), t = tid / kGCh;
-      float h = 0.f;
-      if (c < nch && t < ntg) {
-        float g = 0.f, uu = 0.f;
-#pragma unroll
-        for (int w = 0; w < kNT / 32; ++w) { g += s_red[w][c][t]; uu += s_red[w][8 + c][t]; }
-        bool selected = true;
-        if (!cfg.dense) {
-          const int p = off + tg0 + t, j = s_list[c];
-          selected = (__ldcg(&ws.selmask[(size_t)p * nmw + (j >> 5)]) >> (j & 31)) & 1u;
+#pragma unroll 1
+  for (;;) {
+    __syncthreads();  // the previous item's reads of shared memory are done
+    if (tid == 0) {
+      const int it = (int)atomicAdd(&ws.counters[kCntGatherWork], 1u);
+      int u = 0;
+      if (it < nchunks) {  // slot of run `it`: last u with coff[u] <= it
+        int lo = 0, hi = nu - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (__ldcg(&ws.coff[mid]) <= it) lo = mid; else hi = mid - 1;
         }
-        h = selected ? silu(g) * uu * s_w[t] : 0.f;
+        u = lo;
       }
-      s_h[t][c] = h;
+      s_item = it;
+      s_u = u;
     }
     __syncthreads();
-    // ---- down: A = [h_hi ; h_lo] (token rows), B = down columns, this warp's column tiles
-    const float2 hp = *reinterpret_cast<const float2*>(&s_h[g8][2 * c4]);
-    const uint32_t ahi = pack_bf16x2(hp.x, hp.y);
-    const float2 hhi = make_float2(__bfloat162float(__ushort_as_bfloat16((uint16_t)(ahi & 0xffffu))),
-                                   __bfloat162float(__ushort_as_bfloat16((uint16_t)(ahi >> 16))));
-    const uint32_t alo = pack_bf16x2(hp.x - hhi.x, hp.y - hhi.y);
-    float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
-    const bool tok_ok = g8 < ntg;
-    int nt = 0;
-    for (; nt + 2 <= NTW; nt += 2) {
-      const int m0 = (nt0 + nt) * 8;
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
-      float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
-      mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
-      if (tok_ok) {
-        red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
-        red_add_v2(yrow + m0 + 8 + 2 * c4, dB[0] + dB[2], dB[1] + dB[3]);
+    const int item = s_item;
+    if (item >= nitems || !ok) break;
+
+    // ----------------------------------------------------------- low-rank item
+    if (item >= nchunks) {
+      const int q = item - nchunks, u = q / cfg.nlr;
+      const int row = (q - u * cfg.nlr) * kLrRows + tid;
+      const int e = ws.slot_expert[u];
+      const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
+      if (row < d && r > 0) {
+        const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
+        for (int ti = 0; ti < cnt; ++ti) {
+          const int p = off + ti;
+          const float* z = ws.z + (size_t)p * r;
+          float acc = 0.f;
+          for (int qq = 0; qq < r; ++qq) acc = fmaf(bf16_lo(arow[qq]), __ldcg(z + qq), acc);
+          atomicAdd(&ws.y_acc[(size_t)ws.pair_tok[p] * d + row], ws.pair_w[p] * acc);
+        }
       }
+      continue;
     }
-    if (nt < NTW) {
-      const int m0 = (nt0 + nt) * 8;
-      uint32_t b0, b1;
-      ldsm_x2_t(b_base + 2u * m0, b0, b1);
-      float dA[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
-      if (tok_ok) red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+
+    // ----------------------------------------------------------- a run of union channels
+    const int u = s_u;
+    const int e = ws.slot_expert[u];
+    const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
+    const int rb = (item - __ldcg(&ws.coff[u])) * run;
+    const int nrun = min(run, __ldcg(&ws.ucnt[u]) - rb);
+    const int nst = (nrun + CH - 1) / CH;
+    for (int i = tid; i < nrun; i += kNT)
+      s_run[i] = cfg.dense ? rb + i : (int)__ldcg(&ws.ulist[(size_t)u * ipad + rb + i]);
+
+    for (int tg0 = 0; tg0 < cnt && ok; tg0 += 8) {  // (records are streamed again per 8 tokens)
+      const int ntg = min(8, cnt - tg0);
+      __syncthreads();  // s_run; s_tok, s_w, s_h and every stage buffer are free
+      if (tid < 8) {
+        const int p = off + tg0 + min(tid, ntg - 1);
+        s_tok[tid] = ws.pair_tok[p];
+        s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
+      }
+      if (tid == 0)  // fill: stages 0 .. kGBufs - 2
+        for (int st = 0; st < min(kGBufs - 1, nst); ++st)
+          gather_issue(buf0 + st * bstride, records, s_run, e, st * CH, min(CH, nrun - st * CH), d, I,
+                       s_list[st], &bar[st]);
+      __syncthreads();  // s_tok, the fill's lists
+      // B fragments (x of this lane's token g8) of this warp's k-steps
+      uint32_t xb[KSW > 0 ? KSW : 1][2];
+      const uint32_t* xrow = reinterpret_cast<const uint32_t*>(x + (size_t)s_tok[g8] * d);
+#pragma unroll
+      for (int i = 0; i < KSW; ++i)
+        if (ks0 + i < ks1) {
+          xb[i][0] = __ldg(xrow + (ks0 + i) * 8 + c4);
+          xb[i][1] = __ldg(xrow + (ks0 + i) * 8 + 4 + c4);
+        }
+      // selection bit of this thread's (token, channel) in stage 0
+      uint32_t selw = 1u;
+      if (!cfg.dense && tid < 8 * CH && ht < ntg && hc < min(CH, nrun)) {
+        const int j = s_list[0][hc];
+        selw = __ldcg(&ws.selmask[(size_t)(off + tg0 + ht) * nmw + (j >> 5)]) >> (j & 31);
+      }
+      float yacc[REGACC ? kGAccTiles : 1][2];
+#pragma unroll
+      for (int i = 0; i < (REGACC ? kGAccTiles : 1); ++i) { yacc[i][0] = 0.f; yacc[i][1] = 0.f; }
+
+#pragma unroll 1
+      for (int stg = 0; stg < nst; ++stg) {
+        const int b = stg % kGBufs;
+        const int nch = min(CH, nrun - stg * CH);
+        // keep kGBufs - 1 stages in flight: stage stg + kGBufs - 1 goes into the buffer
+        // that stage stg - 1 has just released
+        if (tid == 0 && stg + kGBufs - 1 < nst) {
+          const int sn = stg + kGBufs - 1, bn = sn % kGBufs;
+          gather_issue(buf0 + bn * bstride, records, s_run, e, sn * CH, min(CH, nrun - sn * CH), d, I,
+                       s_list[bn], &bar[bn]);
+        }
+        const bool okw = mbar_wait(&bar[b], (phases >> b) & 1u, ws.err);
+        if (!__syncthreads_and(okw)) {  // sticky error set; let copies in flight land
+          for (int q = stg; q < min(nst, stg + kGBufs); ++q)
+            mbar_wait(&bar[q % kGBufs], (phases >> (q % kGBufs)) & 1u, ws.err);
+          ok = false;
+          break;
+        }
+        phases ^= 1u << b;
+        const uint16_t* rec = buf0 + b * bstride;
+        // gate/up ldmatrix row: channel lane % 8 (channels past nch read channel 0;
+        // their rows are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 (lane / 16)
+        const int gch = (lane & 7) < nch ? (lane & 7) : 0;
+        uint32_t a_addr =
+            smem_addr(rec + (size_t)gch * rs + ((lane >> 3) & 1) * d + 8 * (lane >> 4)) + 32u * ks0;
+        // down ldmatrix.trans row: channel lane % 8 (channels past nch read channel 0;
+        // their h is zero), element block 8 (lane / 16)
+        const uint32_t b_base = smem_addr(rec + (size_t)gch * rs + 2 * d + 8 * (lane >> 4));
+        // ---- gate/up partials over this warp's k-steps
+        {
+          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+          int ks = ks0;
+          if (KSW > 0) {
+#pragma unroll
+            for (int i = 0; i < KSW; i += 2) {
+              if (ks0 + i + 1 < ks1) {
+                uint32_t a[2][4];
+                ldsm_x4(a_addr + 32u * i, a[0][0], a[0][1], a[0][2], a[0][3]);
+                ldsm_x4(a_addr + 32u * (i + 1), a[1][0], a[1][1], a[1][2], a[1][3]);
+                mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], xb[i][0], xb[i][1]);
+                mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], xb[i + 1][0], xb[i + 1][1]);
+              } else if (ks0 + i < ks1) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(a_addr + 32u * i, a0, a1, a2, a3);
+                mma_bf16(acc0, a0, a1, a2, a3, xb[i][0], xb[i][1]);
+              }
+            }
+            ks = ks1;
+          }
+          for (; ks + 2 <= ks1; ks += 2, a_addr += 64u) {
+            uint32_t a[2][4];
+            ldsm_x4(a_addr, a[0][0], a[0][1], a[0][2], a[0][3]);
+            ldsm_x4(a_addr + 32u, a[1][0], a[1][1], a[1][2], a[1][3]);
+            const uint32_t b00 = __ldg(xrow + ks * 8 + c4), b01 = __ldg(xrow + ks * 8 + 4 + c4);
+            const uint32_t b10 = __ldg(xrow + ks * 8 + 8 + c4), b11 = __ldg(xrow + ks * 8 + 12 + c4);
+            mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b00, b01);
+            mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b10, b11);
+          }
+          if (ks < ks1) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a_addr, a0, a1, a2, a3);
+            mma_bf16(acc0, a0, a1, a2, a3, __ldg(xrow + ks * 8 + c4), __ldg(xrow + ks * 8 + 4 + c4));
+          }
+          s_red[warp][g8][2 * c4] = acc0[0] + acc1[0];
+          s_red[warp][g8][2 * c4 + 1] = acc0[1] + acc1[1];
+          s_red[warp][g8 + 8][2 * c4] = acc0[2] + acc1[2];
+          s_red[warp][g8 + 8][2 * c4 + 1] = acc0[3] + acc1[3];
+        }
+        __syncthreads();
+        // ---- h[token][channel] = silu(g) u, times the selection bit and the router weight
+        if (tid < 8 * CH) {
+          float h = 0.f;
+          if (hc < nch && ht < ntg && (selw & 1u)) {
+            float g = 0.f, uu = 0.f;
+#pragma unroll
+            for (int w = 0; w < kNT / 32; ++w) { g += s_red[w][hc][ht]; uu += s_red[w][8 + hc][ht]; }
+            h = silu(g) * uu * s_w[ht];
+          }
+          s_h[ht][hc] = h;
+          // the next stage's selection bit (its list was written when it was issued)
+          selw = 1u;
+          if (!cfg.dense && stg + 1 < nst && ht < ntg && hc < min(CH, nrun - (stg + 1) * CH)) {
+            const int j = s_list[(stg + 1) % kGBufs][hc];
+            selw = __ldcg(&ws.selmask[(size_t)(off + tg0 + ht) * nmw + (j >> 5)]) >> (j & 31);
+          }
+        }
+        __syncthreads();
+        // ---- down: A = [h_hi ; h_lo] (token rows), B = down columns, this warp's column tiles
+        const float2 hp = *reinterpret_cast<const float2*>(&s_h[g8][2 * c4]);
+        const uint32_t ahi = pack_bf16x2(hp.x, hp.y);
+        const float hx = __uint_as_float(ahi << 16), hy = __uint_as_float(ahi & 0xffff0000u);
+        const uint32_t alo = pack_bf16x2(hp.x - hx, hp.y - hy);
+        if (REGACC) {
+#pragma unroll
+          for (int nt = 0; nt < kGAccTiles; nt += 2) {
+            if (nt < NTW) {
+              const int m0 = (nt0 + nt) * 8;
+              uint32_t b0, b1, b2, b3;
+              if (nt + 1 < NTW) {
+                ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
+              } else {
+                ldsm_x2_t(b_base + 2u * m0, b0, b1);
+                b2 = b0; b3 = b1;
+              }
+              float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
+              mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
+              yacc[nt][0] += dA[0] + dA[2];
+              yacc[nt][1] += dA[1] + dA[3];
+              yacc[nt + 1][0] += dB[0] + dB[2];
+              yacc[nt + 1][1] += dB[1] + dB[3];
+            }
+          }
+        } else {
+          float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
+          const bool tok_ok = g8 < ntg;
+          int nt = 0;
+          for (; nt + 2 <= NTW; nt += 2) {
+            const int m0 = (nt0 + nt) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
+            float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
+            mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
+            if (tok_ok) {
+              red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+              red_add_v2(yrow + m0 + 8 + 2 * c4, dB[0] + dB[2], dB[1] + dB[3]);
+            }
+          }
+          if (nt < NTW) {
+            const int m0 = (nt0 + nt) * 8;
+            uint32_t b0, b1;
+            ldsm_x2_t(b_base + 2u * m0, b0, b1);
+            float dA[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
+            if (tok_ok) red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+          }
+        }
+        __syncthreads();  // this stage's buffer, s_red and s_h are free
+      }
+      if (REGACC && ok && g8 < ntg) {  // one reduction-add per output of the run
+        float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
+#pragma unroll
+        for (int nt = 0; nt < kGAccTiles; ++nt)
+          if (nt < NTW) red_add_v2(yrow + (nt0 + nt) * 8 + 2 * c4, yacc[nt][0], yacc[nt][1]);
+      }
     }
   }
 }
@@ -666,6 +823,18 @@ __global__ void __launch_bounds__(kNT) finalize_kernel(uint16_t* __restrict__ ou
 // =====================================================================================
 // host-side launcher
 // =====================================================================================
+int sm_count() {
+  static int n[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (n[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    n[dev] = v;
+  }
+  return n[dev];
+}
+
 int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uint16_t* records,
                    const uint32_t* sketch, const float* alpha, int k, int mode, float tau,
                    const uint16_t* lr_a, const uint16_t* lr_b, uint16_t* out, const Dims& D,
@@ -685,13 +854,20 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   }
   if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
   GatherCfg cfg;
-  cfg.ch = max(1, min(kGCh, (200 * 1024) / (6 * d + 16)));
-  cfg.nchunk = (D.inter + cfg.ch - 1) / cfg.ch;
+  cfg.ch = max(1, min(kGCh, (196 * 1024 / kGBufs) / (6 * d + 16)));
   cfg.nlr = D.rank > 0 ? (d + kLrRows - 1) / kLrRows : 0;
   cfg.dense = dense;
-  const size_t gsmem = (size_t)cfg.ch * (6 * d + 16);
-  dim3 ggrid(cfg.nchunk + cfg.nlr, maxslots);
-  gather_kernel<<<ggrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+  // persistent CTAs, one per SM, taking work items (runs of union channels, then
+  // low-rank row blocks) off a counter
+  const int ngrid = sm_count();
+  union_kernel<<<maxslots, kNT, 0, st>>>(D, ws, cfg.ch, ngrid, dense);
+  const size_t gsmem = (size_t)kGBufs * cfg.ch * (6 * d + 16);
+  if (d <= 2048)
+    gather_kernel<true, 16><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+  else if (d <= 4096)
+    gather_kernel<false, 32><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+  else
+    gather_kernel<false, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
   {
     const size_t n8 = (size_t)B * d / 8;
     const size_t nb = (n8 + kNT - 1) / kNT;
@@ -706,7 +882,11 @@ int general_set_smem_limits() {
   cudaError_t e = cudaSuccess;
   e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  e = cudaFuncSetAttribute(gather_kernel<true, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (e != cudaSuccess) return MSB_ECUDA;
+  e = cudaFuncSetAttribute(gather_kernel<false, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  if (e != cudaSuccess) return MSB_ECUDA;
+  e = cudaFuncSetAttribute(gather_kernel<false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 
