@@ -85,7 +85,8 @@ struct Misc {
   float h[kRingMax];
   float red[kFW][2 * kRingMax];  // per-warp (gate . x, up . x) of a group's channels
   // channel select scratch
-  uint32_t wt[kFW], wt2[kFW];  // per-warp totals of the two block scans
+  uint32_t wt[kFW];            // per-warp totals of the bin scan
+  uint32_t wgt[kFW], weq[kFW]; // per warp range: keys above the k-th, keys equal to it
   uint32_t kb, rem, cnt, ccount, kth, need;
   uint32_t ck[kCandMax];       // keys of the bin holding the k-th key, and their indices
   uint32_t ci[kCandMax];
@@ -231,16 +232,33 @@ __device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, ui
   }
   __syncthreads();
   const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
+  // scatter layout: warp w owns the indices [w * span, (w + 1) * span)
+  const int span = 32 * ((n + kFT - 1) / kFT);
+  const int wb = warp * span, we = min(n, wb + span);
+  const uint32_t lt = (1u << lane) - 1u;
   uint32_t kth, need;
-  if (cnt > (uint32_t)kCandMax) {
+  if (cnt > (uint32_t)kCandMax) {  // heavy ties: radix descent, then count per warp range
     radix_kth_smem<kFT>(keys, n, k, hist, M.info, &kth, &need);
-  } else {
-    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t ngt = 0, neq = 0;
 #pragma unroll 4
-    for (int j0 = warp * 32; j0 < n; j0 += kFT) {  // warp-uniform trip count
+    for (int j0 = wb; j0 < we; j0 += 32) {
       const int j = j0 + lane;
-      const uint32_t key = j < n ? keys[j] : 0u;
-      const bool m = j < n && min((uint32_t)(kSelBins - 1), (maxkey - key) >> 15) == kb;
+      const uint32_t key = j < we ? keys[j] : 0u;
+      ngt += __popc(__ballot_sync(0xffffffffu, j < we && key > kth));
+      neq += __popc(__ballot_sync(0xffffffffu, j < we && key == kth));
+    }
+    if (lane == 0) { M.wgt[warp] = ngt; M.weq[warp] = neq; }
+    __syncthreads();
+  } else {
+    // gather the bin's keys; keys of higher bins (larger keys) are counted per warp range
+    uint32_t ngt = 0;
+#pragma unroll 4
+    for (int j0 = wb; j0 < we; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < we ? keys[j] : 0u;
+      const uint32_t bin = min((uint32_t)(kSelBins - 1), (maxkey - key) >> 15);
+      ngt += __popc(__ballot_sync(0xffffffffu, j < we && bin < kb));
+      const bool m = j < we && bin == kb;
       const uint32_t mb = __ballot_sync(0xffffffffu, m);
       if (mb) {
         const int leader = __ffs(mb) - 1;
@@ -254,42 +272,38 @@ __device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, ui
         }
       }
     }
+    if (lane == 0) { M.wgt[warp] = ngt; M.weq[warp] = 0u; }
     __syncthreads();
-    // rank inside the bin by (key desc, index asc): the k-th key has rank rem - 1
+    // rank inside the bin by (key desc, index asc); the k-th key sits at position rem - 1.
+    // A candidate whose equal keys occupy positions [gt, gt + eq) is above the k-th key
+    // if rem - 1 >= gt + eq, equal to it if gt <= rem - 1 < gt + eq.
     if (tid < (int)cnt) {
       const uint32_t mk = M.ck[tid], mi = M.ci[tid];
-      uint32_t rank = 0, gt = 0;
+      uint32_t gt = 0, eq = 0;
 #pragma unroll 4
       for (int i = 0; i < (int)cnt; ++i) {
-        const uint32_t ok_ = M.ck[i], oi = M.ci[i];
-        rank += (ok_ > mk) || (ok_ == mk && oi < mi);
+        const uint32_t ok_ = M.ck[i];
         gt += ok_ > mk;
+        eq += ok_ == mk;
       }
-      if (rank == rem - 1) { M.kth = mk; M.need = rem - gt; }
+      const uint32_t pk = rem - 1u, w = mi / (uint32_t)span;
+      if (pk >= gt + eq) {
+        atomicAdd(&M.wgt[w], 1u);
+      } else if (pk >= gt) {
+        atomicAdd(&M.weq[w], 1u);
+        M.kth = mk;
+        M.need = rem - gt;
+      }
     }
     __syncthreads();
     kth = M.kth;
     need = M.need;
   }
-  // scatter: warp w owns indices [w * span, (w + 1) * span); ballots give positions
-  const int span = 32 * ((n + kFT - 1) / kFT);
-  const int wb = warp * span, we = min(n, wb + span);
-  uint32_t ngt = 0, neq = 0;
-#pragma unroll 4
-  for (int j0 = wb; j0 < we; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < we ? keys[j] : 0u;
-    ngt += __popc(__ballot_sync(0xffffffffu, j < we && key > kth));
-    neq += __popc(__ballot_sync(0xffffffffu, j < we && key == kth));
-  }
-  if (lane == 0) M.wt2[warp] = ngt | (neq << 16);
-  __syncthreads();
   uint32_t gtb = 0, eqb = 0;
 #pragma unroll
   for (int w = 0; w < kFW; ++w) {
-    const uint32_t v = w < warp ? M.wt2[w] : 0u;
-    gtb += v & 0xffffu;
-    eqb += v >> 16;
+    gtb += w < warp ? M.wgt[w] : 0u;
+    eqb += w < warp ? M.weq[w] : 0u;
   }
   const uint32_t ltm = (1u << lane) - 1u;
 #pragma unroll 4
@@ -311,10 +325,8 @@ __device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, ui
 }
 
 // Sketch scores of this CTA's nt row tiles: warp w takes chunks [kc0, kc1) of every
-// tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B (every
-// column of B holds x; only column 0 of D is read).  Four accumulators, one per
-// 16-column step of a chunk, chain through the chunks.  Partial sums go to
-// part[warp][tile*16 + row].
+// tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B.
+// Partial sums go to part[warp][tile*16 + row].
 __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm, int nt, int KC,
                                          float* part_w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -323,12 +335,15 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
   const uint4* xp = xperm + c * 2;
 #pragma unroll 1
   for (int tl = 0; tl < nt; ++tl) {
-    float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
-    float m2[4] = {0.f, 0.f, 0.f, 0.f}, m3[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 2
     for (int kc = kc0; kc < kc1; ++kc) {
       const uint2 w = codes[((size_t)tl * KC + kc) * 32 + lane];
-      const uint4 xa = xp[kc * 8], xb = xp[kc * 8 + 1];
+      uint4 xa = make_uint4(0u, 0u, 0u, 0u), xb = xa;
+      if (g == 0) { xa = xp[kc * 8]; xb = xp[kc * 8 + 1]; }
+      // four independent 16-column steps (no accumulator chain between them)
+      float m0[4] = {0.f, 0.f, 0.f, 0.f}, m1[4] = {0.f, 0.f, 0.f, 0.f};
+      float m2[4] = {0.f, 0.f, 0.f, 0.f}, m3[4] = {0.f, 0.f, 0.f, 0.f};
       mma_bf16(m0, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
                (w.y << 2) & kSketchMask, xa.x, xa.y);
       mma_bf16(m1, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
@@ -337,10 +352,12 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
                (w.y << 10) & kSketchMask, xb.x, xb.y);
       mma_bf16(m3, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask, (w.x << 14) & kSketchMask,
                (w.y << 14) & kSketchMask, xb.z, xb.w);
+      acc0 += (m0[0] + m1[0]) + (m2[0] + m3[0]);
+      acc1 += (m0[2] + m1[2]) + (m2[2] + m3[2]);
     }
     if (c == 0) {
-      part_w[tl * kRowTile + g] = (m0[0] + m1[0]) + (m2[0] + m3[0]);
-      part_w[tl * kRowTile + g + 8] = (m0[2] + m1[2]) + (m2[2] + m3[2]);
+      part_w[tl * kRowTile + g] = acc0;
+      part_w[tl * kRowTile + g + 8] = acc1;
     }
   }
 }
@@ -602,13 +619,23 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
   }
 
   // Per group: gate . x and up . x of the group's channels on the tensor cores (A =
-  // the records' gate/up rows, bf16 straight from the ring via ldmatrix; B = x, read
-  // through L1; warp w takes k-steps [ks0, ks1) and the warps' partials meet in
+  // the records' gate/up rows, bf16 straight from the ring via ldmatrix; B = x; warp w
+  // takes k-steps [ks0, ks1) and the warps' partials meet in
   // M.red), then h, then y += h_i * down_i with every thread owning 8-element groups.
   const int KS = d / 16;
   const int ks0 = warp * KS / kFW, ks1 = (warp + 1) * KS / kFW;
   const uint32_t* x32 = reinterpret_cast<const uint32_t*>(P.x);
   const int c4 = lane & 3, g8 = lane >> 2;
+  // d <= 2048: the x B-fragments of this warp's k-steps sit in registers (loaded while
+  // the records are in flight); larger d reads them through L1 at each k-step
+  constexpr int KSW = IT == 1 ? 16 : 0;
+  uint32_t xb[KSW > 0 ? KSW : 1][2];
+#pragma unroll
+  for (int i = 0; i < KSW; ++i)
+    if (ks0 + i < ks1) {
+      xb[i][0] = __ldg(x32 + (ks0 + i) * 8 + c4);
+      xb[i][1] = __ldg(x32 + (ks0 + i) * 8 + 4 + c4);
+    }
   float y[IT][8];
 #pragma unroll
   for (int it = 0; it < IT; ++it)
@@ -636,7 +663,22 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
                                   8 * (lane >> 4)) + 32u * ks0;
       float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
       int ks = ks0;
-      if (ok) {
+      if (ok && KSW > 0) {
+#pragma unroll
+        for (int i = 0; i < KSW; i += 2) {
+          if (ks0 + i + 1 < ks1) {
+            uint32_t a[2][4];
+            ldsm_x4(a_addr + 32u * i, a[0][0], a[0][1], a[0][2], a[0][3]);
+            ldsm_x4(a_addr + 32u * (i + 1), a[1][0], a[1][1], a[1][2], a[1][3]);
+            mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], xb[i][0], xb[i][1]);
+            mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], xb[i + 1][0], xb[i + 1][1]);
+          } else if (ks0 + i < ks1) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(a_addr + 32u * i, a0, a1, a2, a3);
+            mma_bf16(acc0, a0, a1, a2, a3, xb[i][0], xb[i][1]);
+          }
+        }
+      } else if (ok) {
 #pragma unroll 1
         for (; ks + 4 <= ks1; ks += 4, a_addr += 128u) {
           uint32_t a[4][4], b[4][2];

@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
 #pragma unroll
     for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
     const uint4* wrow = reinterpret_cast<const uint4*>(router_t + (size_t)e * d);
+#pragma unroll 8
     for (int i = lane; i < d / 8; i += 32) {
       const uint4 wv = __ldg(wrow + i);
 #pragma unroll
@@ -243,6 +244,7 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
       const uint4* brow = reinterpret_cast<const uint4*>(lr_b + ((size_t)e * D.rank + rho) * d);
       const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
       float acc = 0.f;
+#pragma unroll 8
       for (int i = lane; i < d / 8; i += 32) acc = dot8(__ldg(brow + i), __ldg(xr + i), acc);
       acc = warp_sum(acc);
       if (lane == 0) ws.z[(size_t)p * D.rank + rho] = acc;
@@ -279,7 +281,7 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
     if (rt < ntiles) {
       const uint32_t* xp = xperm + g * xstride + c * 8;
-#pragma unroll 4
+#pragma unroll 8
       for (int kc = kc0; kc < kc1; ++kc) {
         const uint2 w = __ldg(codes + (size_t)kc * 32);
         const uint4 xa = *reinterpret_cast<const uint4*>(xp + kc * 32);
