@@ -260,22 +260,27 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
   const uint2* codes =
       reinterpret_cast<const uint2*>(sketch) + ((size_t)(e * (ipad / kRowTile) + tile0 + rt) * KC) * 32 + lane;
 
+  __shared__ int s_tk[kScoreTok];
   for (int tt = 0; tt < cnt; tt += kScoreTok) {
     const int ntok = min(kScoreTok, cnt - tt);
     __syncthreads();
-    // build xperm for tokens pair_tok[off + tt + n]
-    for (int i = threadIdx.x; i < kScoreTok * KC * 32; i += kNT) {
-      const int n = i / (KC * 32);
-      const int rem = i % (KC * 32);
-      const int kc = rem >> 5, cc = (rem >> 3) & 3, q = rem & 7;
-      const int s = q >> 1, p = q & 1;
-      uint32_t v = 0;
-      if (n < ntok) {
-        const int t = ws.pair_tok[off + tt + n];
-        const int col = kc * kColChunk + 16 * s + 2 * cc + 8 * p;
-        v = __ldg(reinterpret_cast<const uint32_t*>(x + (size_t)t * d + col));
+    if (threadIdx.x < kScoreTok)
+      s_tk[threadIdx.x] = threadIdx.x < ntok ? ws.pair_tok[off + tt + threadIdx.x] : -1;
+    __syncthreads();
+    // build xperm for tokens pair_tok[off + tt + n]: the 16-byte group v of a row holds
+    // columns 8v .. 8v+7 = the pairs cc = 0..3 of (chunk v / 8, step (v / 2) % 4, half v % 2)
+#pragma unroll
+    for (int n = 0; n < kScoreTok; ++n) {
+      const int t = s_tk[n];
+      for (int v = threadIdx.x; v < d / 8; v += kNT) {
+        uint4 q = make_uint4(0u, 0u, 0u, 0u);
+        if (t >= 0) q = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d) + v);
+        uint32_t* dst = xperm + n * xstride + (v >> 3) * 32 + ((v >> 1) & 3) * 2 + (v & 1);
+        dst[0] = q.x;
+        dst[8] = q.y;
+        dst[16] = q.z;
+        dst[24] = q.w;
       }
-      xperm[n * xstride + (kc * 4 + cc) * 8 + q] = v;
     }
     __syncthreads();
     float sum[4] = {0.f, 0.f, 0.f, 0.f};
@@ -525,9 +530,20 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   __shared__ float s_w[8];
   __shared__ float s_red[kNT / 32][16][8];
   __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels >= ch zero
+  // slot tables, copied once: run offsets, union sizes, experts, pair offsets
+  __shared__ int s_coff[MSB_MAX_EXPERTS + 1], s_ucnt[MSB_MAX_EXPERTS], s_se[MSB_MAX_EXPERTS],
+      s_so[MSB_MAX_EXPERTS + 1];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int d = D.d, I = D.inter, ipad = D.ipad, r = D.rank;
   const int nu = *ws.nused;
+  for (int i = tid; i <= nu; i += kNT) {
+    s_coff[i] = __ldcg(&ws.coff[i]);
+    s_so[i] = __ldcg(&ws.slot_off[i]);
+    if (i < nu) {
+      s_ucnt[i] = __ldcg(&ws.ucnt[i]);
+      s_se[i] = __ldcg(&ws.slot_expert[i]);
+    }
+  }
   const int nchunks = __ldcg(&ws.coff[nu]);
   const int run = (int)__ldcg(&ws.counters[kCntGatherRun]);
   const int nitems = nchunks + nu * cfg.nlr;
@@ -551,18 +567,22 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   // h step ownership: thread tid < 8 * CH takes (token tid / CH, channel tid % CH)
   const int hc = tid % CH, ht = tid / CH;
   bool ok = true;
+  // work items are claimed one ahead, so the counter's round trip overlaps an item
+  int next_item = 0;
+  if (tid == 0) next_item = (int)atomicAdd(&ws.counters[kCntGatherWork], 1u);
 
 #pragma unroll 1
   for (;;) {
-    __syncthreads();  // the previous item's reads of shared memory are done
+    __syncthreads();  // the previous item's reads of shared memory are done (and the tables)
     if (tid == 0) {
-      const int it = (int)atomicAdd(&ws.counters[kCntGatherWork], 1u);
+      const int it = next_item;
+      if (it < nitems) next_item = (int)atomicAdd(&ws.counters[kCntGatherWork], 1u);
       int u = 0;
       if (it < nchunks) {  // slot of run `it`: last u with coff[u] <= it
         int lo = 0, hi = nu - 1;
         while (lo < hi) {
           const int mid = (lo + hi + 1) >> 1;
-          if (__ldcg(&ws.coff[mid]) <= it) lo = mid; else hi = mid - 1;
+          if (s_coff[mid] <= it) lo = mid; else hi = mid - 1;
         }
         u = lo;
       }
@@ -577,8 +597,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
     if (item >= nchunks) {
       const int q = item - nchunks, u = q / cfg.nlr;
       const int row = (q - u * cfg.nlr) * kLrRows + tid;
-      const int e = ws.slot_expert[u];
-      const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
+      const int e = s_se[u];
+      const int off = s_so[u], cnt = s_so[u + 1] - off;
       if (row < d && r > 0) {
         const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
         for (int ti = 0; ti < cnt; ++ti) {
@@ -594,10 +614,10 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
 
     // ----------------------------------------------------------- a run of union channels
     const int u = s_u;
-    const int e = ws.slot_expert[u];
-    const int off = ws.slot_off[u], cnt = ws.slot_off[u + 1] - off;
-    const int rb = (item - __ldcg(&ws.coff[u])) * run;
-    const int nrun = min(run, __ldcg(&ws.ucnt[u]) - rb);
+    const int e = s_se[u];
+    const int off = s_so[u], cnt = s_so[u + 1] - off;
+    const int rb = (item - s_coff[u]) * run;
+    const int nrun = min(run, s_ucnt[u] - rb);
     const int nst = (nrun + CH - 1) / CH;
     for (int i = tid; i < nrun; i += kNT)
       s_run[i] = cfg.dense ? rb + i : (int)__ldcg(&ws.ulist[(size_t)u * ipad + rb + i]);
