@@ -157,7 +157,7 @@ def algorithmic_bytes(w, k, rank, union_sizes, dense):
     return total
 
 
-def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None):
+def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None):
     """Time the FP64 CPU oracle, as it stands, on the first tokens of the step
     sequence (a warm pass first fills its weight caches; the second pass is timed).
     Returns (tokens/s, tokens, seconds, threads)."""
@@ -173,14 +173,14 @@ def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None):
     t0 = time.time()
     n = 0
     while n < len(xs) and (max_tokens is None or n < max_tokens):
-        oracle.moe_block(xs[n], lay, w.top_e, k, rank=rank)   # warm: generate + sketch
+        oracle.moe_block(xs[n], lay, top_e or w.top_e, k, rank=rank)   # warm: generate + sketch
         toks.append(n)
         n += 1
         if time.time() - t0 > budget_s:
             break
     t1 = time.time()
     for i in toks:
-        oracle.moe_block(xs[i], lay, w.top_e, k, rank=rank)
+        oracle.moe_block(xs[i], lay, top_e or w.top_e, k, rank=rank)
     dt = time.time() - t1
     ntok = len(toks) * xs[0].shape[0]
     return ntok / dt, ntok, dt, threads
@@ -192,7 +192,7 @@ def run_reference(args, w, world, rank):
         return
     xs = [synth.activations(w, s, batch=args.batch) for s in range(max(min(args.steps, 1000), 1))]
     budget = 60.0
-    v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs, budget_s=budget / 4,
+    v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs, top_e=args.top_e, budget_s=budget / 4,
                                          max_tokens=args.steps)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus,
@@ -210,7 +210,8 @@ METRIC = "MoE-block decode tokens/s (achieved HBM GB/s vs peak) at B=1, 18% budg
 
 
 def config_of(w, args):
-    return {"workload": w.name, "d": w.d, "I": w.inter, "E": w.experts, "top_e": w.top_e,
+    return {"workload": w.name, "d": w.d, "I": w.inter, "E": w.experts,
+            "top_e": args.top_e or w.top_e, "trained_top_e": w.top_e,
             "k": args.k, "budget": round(args.k / w.inter, 4), "rank": args.rank,
             "global_batch": args.batch * args.gpus, "batch_per_gpu": args.batch,
             "decode_steps": w.steps, "replicas": args.replicas,
@@ -403,6 +404,8 @@ def main():
     ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--top-e", type=int, default=None,
+                    help="route each token to this many experts (at most the trained count)")
     ap.add_argument("--stack-grid", action="store_true",
                     help="stacked workload: run k in {13%%, 18%%, 100%%} x batch in {1, 32} on one set of layers")
     ap.add_argument("--threshold", action="store_true",
@@ -460,16 +463,17 @@ def main():
 
     def step(i, s):
         msb.moe_sparse_block(xs[i % nseq], layers[i % args.replicas], args.k, out=outs[i % nseq],
-                             workspace=ws, general=general, stream=s)
+                             workspace=ws, general=general, stream=s, top_e=args.top_e)
 
     # ---- union sizes of every step of the sequence (one traced pass) -> algorithmic bytes
     dense = args.k == w.inter
-    tr = msb.Trace(dims, B, args.k)
+    tr = msb.Trace(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B, args.k)
     bytes_per_step = []
     with torch.cuda.stream(stream):
         for i in range(nseq):
             msb.moe_sparse_block(xs[i], layers[i % args.replicas], args.k, out=outs[i],
-                                 workspace=ws, trace=tr, general=general, stream=stream)
+                                 workspace=ws, trace=tr, general=general, stream=stream,
+                                 top_e=args.top_e)
             if i < 64 or not (B == 1 and not dense):
                 stream.synchronize()
                 bytes_per_step.append(algorithmic_bytes(w, args.k, args.rank,
@@ -536,7 +540,7 @@ def main():
         for i in range(min(50, ne)):
             xd.copy_(xh[i % nseq], non_blocking=True)
             msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
-                                 general=general, stream=stream)
+                                 general=general, stream=stream, top_e=args.top_e)
             oh[i % nseq].copy_(od, non_blocking=True)
         stream.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
@@ -545,7 +549,7 @@ def main():
         for i in range(ne):
             xd.copy_(xh[i % nseq], non_blocking=True)
             msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
-                                 general=general, stream=stream)
+                                 general=general, stream=stream, top_e=args.top_e)
             oh[i % nseq].copy_(od, non_blocking=True)
         a1.record(stream)
         stream.synchronize()
@@ -558,7 +562,8 @@ def main():
 
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
-    plan = msb.path_info(dims, B, args.k, general=general)
+    plan = msb.path_info(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B,
+                         args.k, general=general)
     kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
     traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else ""))
     launches_per_step = 1 if plan["path"] == "single_launch" else (
@@ -582,7 +587,8 @@ def main():
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:
-        v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs_host, budget_s=6.0)
+        v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs_host, budget_s=6.0,
+                                             top_e=args.top_e)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": "%d tokens of the same decode sequence (FP64 numpy "
                                           "oracle, timed second pass), %.1f s" % (ntok, dt)}

@@ -181,6 +181,21 @@ int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, con
                          size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
                          void* stream);
 
+/* The block with the router's expert count overridden ("MoE top_k override
+ * (--moe-top-k)", section "Ce que ça fait"): each token is routed to its top_e
+ * highest-scoring experts instead of the dims->top_e the model was trained with.
+ * 1 <= top_e <= dims->top_e; a count above the trained one is rejected with
+ * MSB_EINVAL.  With dims->renorm the top_e weights are renormalised over the
+ * chosen experts; without it they are the softmax over all E.  The workspace is
+ * sized for the trained dims; the trace buffers hold top_e entries per token.
+ * Otherwise identical to moe_sparse_block (channel top-k with budget k). */
+int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_t,
+                               const void* records, const uint32_t* sketch, const float* alpha,
+                               int32_t k, int32_t top_e, const void* lr_a, const void* lr_b,
+                               void* out, const msb_dims* dims, void* workspace,
+                               size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
+                               void* stream);
+
 /* The calibrated-threshold selector that the pages compare top-k against
  * ("The threshold promises a budget but does not keep it"): identical to
  * moe_sparse_block except S_{t,e} = { j : score_j > tau }, so the number of

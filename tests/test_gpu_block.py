@@ -224,6 +224,35 @@ def test_nonfinite_input_is_flagged_then_recovers(msb, general):
     compare(x, g, oracle.SynthLayer(w), w.top_e, w.k)
 
 
+@pytest.mark.parametrize("top_e,batch", [(4, 1), (6, 1), (4, 4), (6, 16)])
+def test_expert_count_override(msb, top_e, batch):
+    """Routing to fewer experts than trained ("MoE top_k override (--moe-top-k)"),
+    combined with the channel top-k: the oracle with K = top_e."""
+    import torch
+    import token_top_expert_b200 as m
+    from parity import from_bf16_tensor, to_bf16_tensor
+    w = synth.QWEN30B_BLOCK
+    dev = device_layer(w)
+    lay = oracle.SynthLayer(w)
+    dims_k = m.Dims(w.d, w.inter, w.experts, top_e, w.rank, 1)
+    x = synth.activations(w, 21, batch=batch)
+    tr = m.Trace(dims_k, batch, w.k, scores=True)
+    ws = m.Workspace(dev.dims, batch)
+    out = m.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, trace=tr, top_e=top_e)
+    torch.cuda.synchronize()
+    ws.check()
+    if batch == 1:
+        assert msb.path_info(dims_k, 1, w.k)["path"] == "single_launch"
+    g = {"y": oracle.bf16_to_f64(from_bf16_tensor(out)), "ids": tr.expert_ids.cpu().numpy(),
+         "w": tr.expert_w.cpu().numpy(), "sel": tr.sel.cpu().numpy().view(np.uint16),
+         "sel_count": tr.sel_count.cpu().numpy(), "union": tr.union_count.cpu().numpy(),
+         "scores": tr.scores.cpu().numpy()}
+    compare(x, g, lay, top_e, w.k)
+    assert (g["union"] > 0).sum() <= top_e * batch
+    with pytest.raises(m.MsbError):
+        m.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, top_e=w.top_e + 1)
+
+
 def test_selection_is_deterministic(msb):
     w = synth.QWEN30B_BLOCK
     dev = device_layer(w)

@@ -139,5 +139,13 @@ def test_argument_checks_without_gpu(msb):
     assert call(d=bad) == _lib.MSB_EINVAL
     bad = _lib.MsbDims(2048, 8192, 128, 8, 32, 1)       # I beyond the compiled limit
     assert call(d=bad) == _lib.MSB_EUNSUPPORTED
+    # expert-count override: at most the trained top_e, at least 1
+    def call_top_e(top_e, x=fake):
+        return lib.moe_sparse_block_top_e(x, 1, fake, fake, fake, fake, 138, top_e, fake, fake,
+                                          fake * 2, ctypes.byref(dims), fake, ws, None, 0, None)
+
+    assert call_top_e(9) == _lib.MSB_EINVAL
+    assert call_top_e(0) == _lib.MSB_EINVAL
+    assert call_top_e(4, x=None) == _lib.MSB_EINVAL
     assert lib.msb_residual_rmsnorm(None, None, fake, 1, 2048, 1e-6, None) == _lib.MSB_EINVAL
     assert lib.msb_strerror(_lib.MSB_ETIMEOUT) == b"a kernel's bounded wait ran out"

@@ -30,7 +30,7 @@ SYMBOLS = (
     "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_workspace_size",
     "msb_workspace_init", "msb_check", "msb_strerror", "moe_sparse_block",
     "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
-    "moe_sparse_block_noalloc",
+    "moe_sparse_block_noalloc", "moe_sparse_block_top_e",
 )
 
 
@@ -81,6 +81,8 @@ def load() -> ctypes.CDLL:
         "msb_residual_rmsnorm": (I32, [P, P, P, I32, I32, F32, P]),
         "msb_path_info": (I32, [dims_p, I32, I32, U32, P]),
         "moe_sparse_block_noalloc": (I32, [P, P, P, P, P, I32, P, P, P, dims_p, trace_p, P]),
+        "moe_sparse_block_top_e": (I32, [P, I32, P, P, P, P, I32, I32, P, P, P, dims_p, P, SZ,
+                                         trace_p, U32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

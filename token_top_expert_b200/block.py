@@ -176,9 +176,11 @@ def _act(x, dims: Dims):
 # ------------------------------------------------------------------ the block
 
 def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspace | None = None,
-                     trace: Trace | None = None, general: bool = False, stream=None):
+                     trace: Trace | None = None, general: bool = False, stream=None,
+                     top_e: int | None = None):
     """One sparse-MoE block decode step: out[t] = sum_e w_te * (gathered SwiGLU over the
-    k top-scoring channels + A_e B_e x_t).  x: bf16 [B][d] on the GPU."""
+    k top-scoring channels + A_e B_e x_t).  x: bf16 [B][d] on the GPU.  top_e: route each
+    token to this many experts instead of the trained layer.dims.top_e (at most that)."""
     import torch
     dims = layer.dims
     _act(x, dims)
@@ -188,12 +190,15 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
     if workspace is None:
         workspace = Workspace(dims, B, x.device)
     tr = trace.c() if trace is not None else None
-    rc = _lib.load().moe_sparse_block(
-        _ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
-        _ptr(layer.alpha), k, _ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out),
-        ctypes.byref(dims.c()), workspace.ptr, workspace.nbytes,
-        ctypes.byref(tr) if tr is not None else None,
-        _lib.MSB_FLAG_GENERAL if general else 0, _stream(stream))
+    flags = _lib.MSB_FLAG_GENERAL if general else 0
+    args = (_ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
+            _ptr(layer.alpha), k)
+    rest = (_ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out), ctypes.byref(dims.c()), workspace.ptr,
+            workspace.nbytes, ctypes.byref(tr) if tr is not None else None, flags, _stream(stream))
+    if top_e is None:
+        rc = _lib.load().moe_sparse_block(*args, *rest)
+    else:
+        rc = _lib.load().moe_sparse_block_top_e(*args, top_e, *rest)
     _check(rc, "moe_sparse_block")
     return out
 

@@ -250,6 +250,20 @@ int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, con
                       workspace, workspace_bytes, trace, flags, stream);
 }
 
+int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_t,
+                               const void* records, const uint32_t* sketch, const float* alpha,
+                               int32_t k, int32_t top_e, const void* lr_a, const void* lr_b,
+                               void* out, const msb_dims* dims, void* workspace,
+                               size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
+                               void* stream) {
+  // "MoE top_k override (--moe-top-k)", "Ce que ça fait": fewer experts than trained only
+  if (!dims || top_e < 1 || top_e > dims->top_e) return MSB_EINVAL;
+  msb_dims m = *dims;
+  m.top_e = top_e;
+  return block_common(x, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out, &m,
+                      workspace, workspace_bytes, trace, flags, stream);
+}
+
 int32_t moe_sparse_block_threshold(const void* x, int32_t batch, const void* router_t,
                                    const void* records, const uint32_t* sketch,
                                    const float* alpha, float tau, const void* lr_a,

@@ -790,13 +790,16 @@ __global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_consta
     }
   }
   cluster.sync();  // no CTA leaves while its buffer may still be read
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K * P.cpe - 1));
+  // the barrier orders warp 0's reduction-adds before thread 0's fence, which makes them
+  // visible GPU-wide before the slice counter moves
+  if (tid == 0) {
+    __threadfence();
+    M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K * P.cpe - 1));
+    if (M.last) __threadfence();
+  }
   __syncthreads();
   if (M.last) {
     // every contribution to this slice has arrived: convert, re-zero, reset
-    __threadfence();
 #pragma unroll 1
     for (int i = tid; i < P.slice; i += kFT) {
       const float v = atomicExch(P.y_acc + q * P.slice + i, 0.f);
