@@ -157,9 +157,10 @@ def algorithmic_bytes(w, k, rank, union_sizes, dense):
     return total
 
 
-def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None):
+def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None, timed_s=12.0):
     """Time the FP64 CPU oracle, as it stands, on the first tokens of the step
-    sequence (a warm pass first fills its weight caches; the second pass is timed).
+    sequence: a warm pass (bounded by budget_s) fills its weight caches, then passes
+    over the same tokens are timed until at least timed_s seconds of oracle work.
     Returns (tokens/s, tokens, seconds, threads)."""
     import oracle
     try:
@@ -179,10 +180,15 @@ def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None):
         if time.time() - t0 > budget_s:
             break
     t1 = time.time()
-    for i in toks:
-        oracle.moe_block(xs[i], lay, top_e or w.top_e, k, rank=rank)
+    passes = 0
+    while True:
+        for i in toks:
+            oracle.moe_block(xs[i], lay, top_e or w.top_e, k, rank=rank)
+        passes += 1
+        if time.time() - t1 >= timed_s:
+            break
     dt = time.time() - t1
-    ntok = len(toks) * xs[0].shape[0]
+    ntok = passes * len(toks) * xs[0].shape[0]
     return ntok / dt, ntok, dt, threads
 
 
@@ -200,7 +206,8 @@ def run_reference(args, w, world, rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(w, args),
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": "%d tokens (first steps of the decode sequence), %.1f s" % (ntok, dt)},
+                         "sample": "%d token-blocks: passes over the first steps of the decode "
+                                   "sequence (weights cached by an untimed pass), %.1f s" % (ntok, dt)},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -590,8 +597,9 @@ def main():
         v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs_host, budget_s=6.0,
                                              top_e=args.top_e)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                "sample": "%d tokens of the same decode sequence (FP64 numpy "
-                                          "oracle, timed second pass), %.1f s" % (ntok, dt)}
+                                "sample": "%d token-blocks: passes over the first tokens of the "
+                                          "same decode sequence (FP64 numpy oracle, weights "
+                                          "cached by an untimed pass), %.1f s" % (ntok, dt)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, tail
