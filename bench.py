@@ -143,6 +143,21 @@ def dist_setup():
     return world, rank, local
 
 
+def replica_throughput(ms_local: float, units_per_rank: float, dist=None, device=None):
+    """Whole-job throughput of independent replicas (one per rank): the job takes the
+    slowest rank's device time (max over ranks) and processes every rank's units.
+    Returns (ms, units per second over all ranks).  Every rank takes the same
+    collective steps."""
+    import torch
+    ms, world = ms_local, 1
+    if dist is not None and dist.is_available() and dist.is_initialized():
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+        world = dist.get_world_size()
+    return ms, units_per_rank * world / (ms / 1e3)
+
+
 def algorithmic_bytes(w, k, rank, union_sizes, dense):
     """Bytes the method must read for one step: per used expert the sketch
     (I*d/4), row scales (4I), the union of selected channel records (6d each)
@@ -527,14 +542,10 @@ def main():
             e1.record(stream)
         stream.synchronize()
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
+    ms, value = replica_throughput(e0.elapsed_time(e1), args.steps * B, dist, dev)
     if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
         dist.barrier()
     ms_per_step = ms / args.steps
-    value = args.steps * B * world / (ms / 1e3)
     ws.check(stream)
 
     # ---- e2e: public call per step with pinned host x -> device -> host out
@@ -560,12 +571,7 @@ def main():
             oh[i % nseq].copy_(od, non_blocking=True)
         a1.record(stream)
         stream.synchronize()
-    e2e_ms = a0.elapsed_time(a1)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = ne * B * world / (e2e_ms / 1e3)
+    e2e_ms, e2e_value = replica_throughput(a0.elapsed_time(a1), ne * B, dist, dev)
 
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
