@@ -253,6 +253,23 @@ def test_expert_count_override(msb, top_e, batch):
         m.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, top_e=w.top_e + 1)
 
 
+@pytest.mark.parametrize("batch", [1, 4])
+def test_weight_derived_lowrank(msb, batch):
+    """The block with compensation factors derived from the weights alone (in place of
+    seeded ones): same kernels, same parity bar, against the oracle given the same factors."""
+    from token_top_expert_b200 import lowrank
+    w = synth.TINY
+    lw = synth.layer_weights(w)
+    a, b = lowrank.derive_lowrank(lw.gate, lw.up, lw.down, k=w.k, rank=w.rank, samples=1024)
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, w.rank, 1)
+    dev = msb.PackedLayer.from_host(dims, msb.pack(lw.gate, lw.up, lw.down, lw.router, dims), a, b)
+    lay = oracle.ArrayLayer(lw.gate, lw.up, lw.down, lw.router, a, b)
+    for step in range(3):
+        x = synth.activations(w, 300 + step, batch=batch)
+        g = run_gpu(x, dev, w.k)
+        compare(x, g, lay, w.top_e, w.k, rank=w.rank)
+
+
 def test_selection_is_deterministic(msb):
     w = synth.QWEN30B_BLOCK
     dev = device_layer(w)

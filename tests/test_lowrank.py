@@ -1,0 +1,108 @@
+"""Weight-derived low-rank compensation (host-side weight preparation).
+
+Pinned against the oracle's restatement of the selection (sketch, scores, top-k), against
+a closed form (orthogonal gate/up rows of channels that are always skipped: the map's
+coefficient is E[a sigmoid(a)] for a ~ N(0, |gate_j|^2), evaluated here by quadrature),
+and against the defining properties of the construction: nothing skipped gives a zero map;
+on fresh samples from the prior the compensated error is not larger than the uncompensated
+one; the factors are the leading singular directions of the map (Eckart-Young).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from token_top_expert_b200 import lowrank
+
+
+def _expert(d, inter, seed, scale):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(0, scale, (inter, d)), rng.normal(0, scale, (inter, d)),
+            rng.normal(0, scale, (d, inter)))
+
+
+def test_channel_moments_match_the_oracle_selection():
+    d, inter, k = 64, 48, 12
+    gate, up, down = _expert(d, inter, 1, 0.2)
+    x = np.random.default_rng(2).standard_normal((40, d)).astype(np.float32)
+    ma, mb = lowrank.channel_moments(gate, up, down, k, x)
+    t, alpha = oracle.ternary_sketch(gate)
+    ra, rb = np.zeros(inter), np.zeros(inter)
+    for xi in x.astype(np.float64):
+        keep = oracle.topk_channels(oracle.channel_scores(t, alpha, xi), k)
+        a, b = gate @ xi, up @ xi
+        h = a / (1.0 + np.exp(-a)) * b
+        h[keep] = 0.0
+        ra += h * a
+        rb += h * b
+    np.testing.assert_allclose(ma, ra / len(x), rtol=1e-3, atol=1e-6)
+    np.testing.assert_allclose(mb, rb / len(x), rtol=1e-3, atol=1e-6)
+
+
+def test_orthogonal_rows_closed_form():
+    """Channel 0 has a dominant gate row, so with k = 1 channels 1..3 are always skipped.
+    Their gate and up rows lie on distinct axes, so b is independent of a and of
+    the selection: E[h a] = 0 and E[h b] = E[silu(a)] |up|^2, hence c_a = 0 and
+    c_b = E[silu(a)] = E[a sigmoid(a)], a ~ N(0, |gate_j|^2)."""
+    d, inter = 16, 4
+    gate, up, down = np.zeros((inter, d)), np.zeros((inter, d)), np.zeros((d, inter))
+    gate[0, 0] = 50.0
+    up[0, 1] = 1.0
+    sig = [0.0, 0.7, 1.3, 2.0]
+    for j in range(1, inter):
+        gate[j, 2 * j] = sig[j]
+        up[j, 2 * j + 1] = 0.5
+        down[j, j] = 1.0
+    x = np.random.default_rng(5).standard_normal((400_000, d)).astype(np.float32)
+    ma, mb = lowrank.channel_moments(gate, up, down, 1, x)
+    m = lowrank.structured_map(gate, up, down, ma, mb)
+    z = np.linspace(-12, 12, 24001)
+    phi = np.exp(-z * z / 2) / np.sqrt(2 * np.pi)
+    for j in range(1, inter):
+        a = sig[j] * z
+        expect = np.trapezoid(a / (1 + np.exp(-a)) * phi, z)   # E[silu(a)]
+        # M[j] = c_a gate_j + c_b up_j with up_j = 0.5 e_(2j+1)
+        assert m[j, 2 * j + 1] == pytest.approx(0.5 * expect, rel=0.03)
+        assert abs(m[j, 2 * j]) < 0.03 * abs(expect)
+    assert np.all(m[0] == 0.0)  # channel 0 is never skipped
+
+
+def test_nothing_skipped_gives_a_zero_map():
+    d, inter = 32, 24
+    gate, up, down = _expert(d, inter, 3, 0.2)
+    a, b = lowrank.derive_lowrank(gate[None], up[None], down[None], k=inter, rank=4, samples=256)
+    assert not a.any() and not b.any()
+
+
+def test_compensation_does_not_add_error_on_fresh_samples():
+    d, inter, k, r = 64, 96, 18, 8
+    gate, up, down = _expert(d, inter, 5, 0.15)
+    a, b = lowrank.derive_lowrank(gate[None], up[None], down[None], k=k, rank=r, samples=8192,
+                                  seed=11)
+    af, bf = oracle.bf16_to_f64(a[0]), oracle.bf16_to_f64(b[0])
+    t, alpha = oracle.ternary_sketch(gate)
+    xs = np.random.default_rng(99).standard_normal((400, d))
+    e0 = e1 = 0.0
+    for x in xs:
+        keep = oracle.topk_channels(oracle.channel_scores(t, alpha, x), k)
+        skipped = np.setdiff1d(np.arange(inter), keep)
+        y = oracle.expert_output(x, gate, up, down, skipped)
+        e0 += float(y @ y)
+        res = y - af @ (bf @ x)
+        e1 += float(res @ res)
+    assert e1 < e0
+    print("skipped-channel error kept by the compensation: %.4f" % (e1 / e0))
+
+
+def test_factors_are_the_leading_singular_directions():
+    d, inter, k, r = 48, 40, 10, 6
+    gate, up, down = _expert(d, inter, 7, 0.2)
+    x = np.random.default_rng([4, 0]).standard_normal((1024, d), dtype=np.float32)
+    ma, mb = lowrank.channel_moments(gate, up, down, k, x)
+    m = lowrank.structured_map(gate, up, down, ma, mb)
+    a, b = lowrank.derive_lowrank(gate[None], up[None], down[None], k=k, rank=r, samples=1024,
+                                  seed=4, chunk=1024)
+    s = np.linalg.svd(m, compute_uv=False)
+    resid = np.linalg.norm(m - oracle.bf16_to_f64(a[0]) @ oracle.bf16_to_f64(b[0]))
+    tail = np.sqrt((s[r:] ** 2).sum())
+    # Eckart-Young, up to the BF16 rounding of the factors
+    assert resid == pytest.approx(tail, rel=0.05, abs=1e-2 * s[0])
