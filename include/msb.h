@@ -31,9 +31,12 @@
  *    means the legacy default stream) and returns after enqueueing.
  *  - Return value: MSB_OK (0) or a negative MSB_E* code.  Argument errors are
  *    detected on the host before anything is enqueued.  Kernel-side problems
- *    (a bounded wait that ran out) set a sticky word in the workspace that
- *    msb_check() reports after the stream has been synchronised.
- *  - Inputs must be finite (no NaN/Inf).
+ *    (a bounded wait that ran out, a non-finite router logit) set a sticky word
+ *    in the workspace that msb_check() reports after the stream has been
+ *    synchronised.
+ *  - Inputs must be finite (no NaN/Inf); a non-finite router logit makes that
+ *    call's output undefined (reported as MSB_ENONFINITE) and leaves the
+ *    workspace ready for the next call.
  */
 #ifndef MSB_H_
 #define MSB_H_
@@ -182,7 +185,7 @@ int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, con
                          void* stream);
 
 /* The block with the router's expert count overridden ("MoE top_k override
- * (--moe-top-k)", section "Ce que ça fait"): each token is routed to its top_e
+ * (--moe-top-k)", section "Ce que ca fait"): each token is routed to its top_e
  * highest-scoring experts instead of the dims->top_e the model was trained with.
  * 1 <= top_e <= dims->top_e; a count above the trained one is rejected with
  * MSB_EINVAL.  With dims->renorm the top_e weights are renormalised over the

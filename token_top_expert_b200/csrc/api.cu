@@ -256,7 +256,7 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
                                void* out, const msb_dims* dims, void* workspace,
                                size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
                                void* stream) {
-  // "MoE top_k override (--moe-top-k)", "Ce que ça fait": fewer experts than trained only
+  // "MoE top_k override (--moe-top-k)", "Ce que ca fait": fewer experts than trained only
   if (!dims || top_e < 1 || top_e > dims->top_e) return MSB_EINVAL;
   msb_dims m = *dims;
   m.top_e = top_e;
