@@ -248,6 +248,28 @@ def test_single_expert_dense_is_swiglu_ffn():
     np.testing.assert_allclose(y, ref.numpy(), rtol=1e-12, atol=1e-12)
 
 
+@pytest.mark.parametrize("renorm", [True, False])
+def test_all_experts_dense_is_softmax_weighted_ffns(renorm):
+    # K = E, k = I, no low-rank: every expert is used densely and the block is
+    # sum_e softmax(x W_router)_e * FFN_e(x) (with K = E renormalisation changes nothing);
+    # checked with torch's softmax and silu on CPU.
+    import torch
+    rng = np.random.default_rng(8)
+    d, I, E = 16, 10, 5
+    gate, up = rng.standard_normal((E, I, d)), rng.standard_normal((E, I, d))
+    down = rng.standard_normal((E, d, I))
+    router = rng.standard_normal((d, E))
+    x = rng.standard_normal((2, d))
+    lay = oracle.ArrayLayer(gate, up, down, router)
+    y = oracle.moe_block(x, lay, top_e=E, k=I, renorm=renorm, rank=0)["y"]
+    for t in range(2):
+        tx = torch.tensor(x[t])
+        p = torch.softmax(tx @ torch.tensor(router), dim=0)
+        ref = sum(p[e] * (torch.tensor(down[e]) @ (torch.nn.functional.silu(torch.tensor(gate[e]) @ tx)
+                                                  * (torch.tensor(up[e]) @ tx))) for e in range(E))
+        np.testing.assert_allclose(y[t], ref.numpy(), rtol=1e-11, atol=1e-11)
+
+
 # ----------------------------------------------------------------------------- numbers, glue
 
 def test_round_to_bf16():
