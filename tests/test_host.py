@@ -68,9 +68,9 @@ def decode_sketch(words, dims, e):
     return t
 
 
-@pytest.mark.parametrize("inter", [512, 33])
-def test_packer_matches_oracle_sketch(msb, inter):
-    w = synth.TINY.with_(inter=inter, experts=3, heavy_frac=0.05, heavy_scale=4.0)
+@pytest.mark.parametrize("d,inter", [(256, 512), (256, 33), (64, 33), (192, 48)])
+def test_packer_matches_oracle_sketch(msb, d, inter):
+    w = synth.TINY.with_(d=d, inter=inter, experts=3, heavy_frac=0.05, heavy_scale=4.0)
     lw = synth.layer_weights(w)
     dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, w.rank)
     pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
