@@ -19,7 +19,8 @@ and cites the passage it follows.  Sources (web pages, by title and section):
 * [SELECTOR] "Calibration-free top-k MoE selector saves tuning" (quotes the
   paper's abstract: BF16 weights, ternary sketch, low-rank recovery map).
 * [TOPK-OVR] "MoE top_k override (--moe-top-k)" -- "Ce que ca fait" (a token
-  picks 8 of 128 experts; the expert MLP is a gated "SwitchGLU").
+  picks 8 of 128 experts; the expert MLP is a gated "SwitchGLU"); "Combinaison
+  avec d'autres optimisations" (4-bit checkpoints; ``oracle.q4``).
 * [TWN] Li, Zhang and Liu, "Ternary Weight Networks" (2016): the ternarisation
   threshold 0.7*mean|W| and the scale alpha = mean |W| over the kept entries.
   The pages name a "ternary sketch" without its formula; TWN is the reading
@@ -50,3 +51,4 @@ from .moe_block import (  # noqa: F401
     SynthLayer,
     ArrayLayer,
 )
+from . import q4  # noqa: F401,E402
