@@ -26,7 +26,9 @@ def msb():
 
 
 def header_functions():
-    text = open(os.path.join(ROOT, "include", "msb.h")).read()
+    inc = os.path.join(ROOT, "include")
+    text = "".join(open(os.path.join(inc, f)).read() for f in sorted(os.listdir(inc))
+                   if f.endswith(".h"))
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
     return sorted(set(names))
@@ -106,6 +108,86 @@ def test_packer_exact_threshold_tie(msb):
     t = decode_sketch(pk["sketch"], dims, 0)
     np.testing.assert_array_equal(t[:I], t_ref)
     np.testing.assert_array_equal(pk["alpha"][0, :I], a_ref)
+
+
+def decode_q4_records(rec, d):
+    """Reference decoder of the 4-bit record format documented in include/msb_q4.h:
+    3d nibble codes (element 2i in bits 0-3 of byte i, element 2i+1 in bits 4-7), then
+    (scale, bias) BF16 pairs of the gate row's, the up row's and the down column's
+    groups of 64, then zero padding.  rec: [n][record bytes] u8.
+    Returns q [n][3][d], s [n][3][d/64], b [n][3][d/64] (float64), padding bytes."""
+    n, g = rec.shape[0], d // 64
+    nib = rec[:, :3 * d // 2]
+    q = np.empty((n, 3 * d), np.uint8)
+    q[:, 0::2] = nib & 0xF
+    q[:, 1::2] = nib >> 4
+    par = np.ascontiguousarray(rec[:, 3 * d // 2: 3 * d // 2 + 12 * g]).view(np.uint16)
+    par = par.reshape(n, 3, g, 2)
+    return (q.reshape(n, 3, d), oracle.bf16_to_f64(par[..., 0]), oracle.bf16_to_f64(par[..., 1]),
+            rec[:, 3 * d // 2 + 12 * g:])
+
+
+@pytest.mark.parametrize("d,inter", [(256, 40), (64, 33), (192, 17)])
+def test_q4_packer_matches_oracle(msb, d, inter):
+    """4-bit records, sketch and alpha against the oracle's quantiser (oracle.q4) and
+    its sketch of the dequantised gate rows, bit for bit; includes a zero gate row, a
+    constant group and heavy rows."""
+    w = synth.TINY.with_(d=d, inter=inter, experts=2, heavy_frac=0.1, heavy_scale=4.0)
+    lw = synth.layer_weights(w)
+    gate, up, down = lw.gate.copy(), lw.up.copy(), lw.down.copy()
+    gate[0, 1] = 0
+    up[1, 2, :64] = synth.f32_to_bf16_bits(np.full(64, -0.375, np.float32))
+    dims = msb.Dims(d, inter, w.experts, w.top_e, 0)
+    pk = msb.pack_q4(gate, up, down, lw.router, dims)
+    rb = oracle.q4.record_bytes(d)
+    assert pk["records"].shape == (w.experts, inter, rb)
+    for e in range(w.experts):
+        q, s, b, pad = decode_q4_records(pk["records"][e], d)
+        assert not pad.any()
+        for part, mat in enumerate((gate[e], up[e], down[e].T)):
+            q_ref, s_ref, b_ref = oracle.q4.quantize_groups(oracle.bf16_to_f64(mat))
+            np.testing.assert_array_equal(q[:, part], q_ref)
+            np.testing.assert_array_equal(s[:, part], s_ref)
+            np.testing.assert_array_equal(b[:, part], b_ref)
+        g_deq = oracle.q4.q4_weights(oracle.bf16_to_f64(gate[e]), oracle.bf16_to_f64(up[e]),
+                                     oracle.bf16_to_f64(down[e]))[0]
+        t_ref, a_ref = oracle.ternary_sketch(g_deq)
+        np.testing.assert_array_equal(decode_sketch(pk["sketch"], dims, e)[:inter], t_ref)
+        np.testing.assert_array_equal(pk["alpha"][e, :inter], a_ref)
+    np.testing.assert_array_equal(pk["router_t"], lw.router.T)
+
+
+def test_q4_argument_checks(msb):
+    from token_top_expert_b200 import _lib
+    lib = _lib.load()
+    for d, want in ((2048, 3456), (64, 112), (96, 0), (0, 0), (16384, 0)):
+        assert lib.msb_q4_record_bytes(ctypes.byref(msb.Dims(d, 8, 1, 1, 0).c())) == want
+    assert lib.msb_q4_record_bytes(None) == 0
+    z = np.zeros(64 * 8, np.uint16)
+    out = np.zeros(1 << 16, np.uint8)
+    for dims, want in ((msb.Dims(96, 8, 1, 1, 0), _lib.MSB_EINVAL),
+                       (msb.Dims(64, 0, 1, 1, 0), _lib.MSB_EINVAL),
+                       (msb.Dims(64, _lib.MSB_MAX_INTER + 1, 1, 1, 0), _lib.MSB_EUNSUPPORTED)):
+        rc = lib.msb_pack_q4(z.ctypes.data, z.ctypes.data, z.ctypes.data, z.ctypes.data,
+                             ctypes.byref(dims.c()), out.ctypes.data, out.ctypes.data,
+                             out.ctypes.data, out.ctypes.data, 1)
+        assert rc == want
+    # dims the size queries reject (more routed experts than experts) are rejected by
+    # both packers before anything is written, and by the bindings before allocating
+    bad = msb.Dims(64, 8, 2, 3, 0)
+    assert lib.msb_sketch_words(ctypes.byref(bad.c())) == 0
+    for fn in (lib.msb_pack, lib.msb_pack_q4):
+        rc = fn(z.ctypes.data, z.ctypes.data, z.ctypes.data, z.ctypes.data, ctypes.byref(bad.c()),
+                out.ctypes.data, out.ctypes.data, out.ctypes.data, out.ctypes.data, 1)
+        assert rc == _lib.MSB_EINVAL
+    g = np.zeros((2, 8, 64), np.uint16)
+    for fn in (msb.pack, msb.pack_q4):
+        with pytest.raises(msb.MsbError):
+            fn(g, g, np.zeros((2, 64, 8), np.uint16), np.zeros((64, 2), np.uint16), bad)
+    rc = lib.msb_pack_q4(None, z.ctypes.data, z.ctypes.data, z.ctypes.data,
+                         ctypes.byref(msb.Dims(64, 8, 1, 1, 0).c()), out.ctypes.data,
+                         out.ctypes.data, out.ctypes.data, out.ctypes.data, 1)
+    assert rc == _lib.MSB_EINVAL
 
 
 def test_argument_checks_without_gpu(msb):

@@ -14,6 +14,7 @@ from .block import (  # noqa: F401
     moe_sparse_block_noalloc,
     moe_sparse_block_threshold,
     pack,
+    pack_q4,
     path_info,
     residual_rmsnorm,
     sketch_words,

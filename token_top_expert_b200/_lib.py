@@ -1,4 +1,4 @@
-"""ctypes loader of libmsb.so (the C ABI declared in include/msb.h).
+"""ctypes loader of libmsb.so (the C ABI declared in include/msb.h and include/msb_q4.h).
 
 Loading fails loudly: there is no fallback implementation of any step.
 """
@@ -25,13 +25,15 @@ MSB_MAX_TOP_E = 16
 MSB_MAX_RANK = 128
 MSB_MAX_BATCH = 256
 
-# every function include/msb.h declares
+# every function include/msb.h and include/msb_q4.h declare
 SYMBOLS = (
     "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_workspace_size",
     "msb_workspace_init", "msb_check", "msb_strerror", "moe_sparse_block",
     "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
     "moe_sparse_block_noalloc", "moe_sparse_block_top_e",
+    "msb_q4_record_bytes", "msb_pack_q4",
 )
+MSB_Q4_GROUP = 64
 
 
 class MsbDims(ctypes.Structure):
@@ -71,6 +73,8 @@ def load() -> ctypes.CDLL:
         "msb_sketch_words": (SZ, [dims_p]),
         "msb_alpha_count": (SZ, [dims_p]),
         "msb_pack": (I32, [P, P, P, P, dims_p, P, P, P, P, I32]),
+        "msb_q4_record_bytes": (SZ, [dims_p]),
+        "msb_pack_q4": (I32, [P, P, P, P, dims_p, P, P, P, P, I32]),
         "msb_workspace_size": (SZ, [dims_p, I32]),
         "msb_workspace_init": (I32, [P, SZ, P]),
         "msb_check": (I32, [P, P]),

@@ -65,13 +65,46 @@ def pack(gate: np.ndarray, up: np.ndarray, down: np.ndarray, router: np.ndarray,
             raise ValueError("expected contiguous uint16 array of shape %s, got %s %s"
                              % (shape, a.dtype, a.shape))
     cd = dims.c()
+    words = lib.msb_sketch_words(ctypes.byref(cd))
+    if words == 0:
+        _check(_lib.MSB_EINVAL, "msb_sketch_words")
     records = np.empty((E, I, 3 * d), np.uint16)
-    sketch = np.empty(lib.msb_sketch_words(ctypes.byref(cd)), np.uint32)
+    sketch = np.empty(words, np.uint32)
     alpha = np.empty((E, dims.ipad), np.float32)
     router_t = np.empty((E, d), np.uint16)
     rc = lib.msb_pack(_ptr(gate), _ptr(up), _ptr(down), _ptr(router), ctypes.byref(cd),
                       _ptr(records), _ptr(sketch), _ptr(alpha), _ptr(router_t), threads)
     _check(rc, "msb_pack")
+    return {"records": records, "sketch": sketch, "alpha": alpha, "router_t": router_t}
+
+
+def pack_q4(gate: np.ndarray, up: np.ndarray, down: np.ndarray, router: np.ndarray, dims: Dims,
+            threads: int = 0) -> dict:
+    """Pack model-layout BF16 weights into 4-bit channel records (format in
+    include/msb_q4.h) with libmsb's host packer.
+
+    gate, up: [E][I][d]; down: [E][d][I]; router: [d][E] (uint16 BF16 bits).
+    Returns numpy arrays: records [E][I][msb_q4_record_bytes] u8, sketch u32 and
+    alpha [E][Ipad] f32 of the dequantised gate rows, router_t [E][d] u16.
+    """
+    lib = _lib.load()
+    E, I, d = dims.experts, dims.inter, dims.d
+    for a, shape in ((gate, (E, I, d)), (up, (E, I, d)), (down, (E, d, I)), (router, (d, E))):
+        if a.dtype != np.uint16 or a.shape != shape or not a.flags.c_contiguous:
+            raise ValueError("expected contiguous uint16 array of shape %s, got %s %s"
+                             % (shape, a.dtype, a.shape))
+    cd = dims.c()
+    rb = lib.msb_q4_record_bytes(ctypes.byref(cd))
+    words = lib.msb_sketch_words(ctypes.byref(cd))
+    if rb == 0 or words == 0:
+        _check(_lib.MSB_EINVAL, "msb_q4_record_bytes / msb_sketch_words")
+    records = np.empty((E, I, rb), np.uint8)
+    sketch = np.empty(words, np.uint32)
+    alpha = np.empty((E, dims.ipad), np.float32)
+    router_t = np.empty((E, d), np.uint16)
+    rc = lib.msb_pack_q4(_ptr(gate), _ptr(up), _ptr(down), _ptr(router), ctypes.byref(cd),
+                         _ptr(records), _ptr(sketch), _ptr(alpha), _ptr(router_t), threads)
+    _check(rc, "msb_pack_q4")
     return {"records": records, "sketch": sketch, "alpha": alpha, "router_t": router_t}
 
 

@@ -48,7 +48,7 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
     """Compile and link; returns the library path.  Raises on any compiler error."""
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
-    headers.append(os.path.join(INCLUDE, "msb.h"))
+    headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
     cc = nvcc()
     jobs = []
     objs = []
