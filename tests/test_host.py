@@ -231,3 +231,13 @@ def test_argument_checks_without_gpu(msb):
     assert call_top_e(4, x=None) == _lib.MSB_EINVAL
     assert lib.msb_residual_rmsnorm(None, None, fake, 1, 2048, 1e-6, None) == _lib.MSB_EINVAL
     assert lib.msb_strerror(_lib.MSB_ETIMEOUT) == b"a kernel's bounded wait ran out"
+
+
+def test_raw_stream_handle_needs_caller_buffers():
+    """Buffers the binding allocates live on torch's current stream; with a raw handle
+    it cannot order them, so it refuses instead of racing (checked before any CUDA call)."""
+    from token_top_expert_b200 import block
+    block._temporaries_on(None, [object()])       # default stream: nothing to order
+    block._temporaries_on(12345, [None, None])    # caller gave every buffer
+    with pytest.raises(ValueError):
+        block._temporaries_on(12345, [object()])

@@ -199,6 +199,24 @@ def _stream(stream):
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
+def _temporaries_on(stream, tensors):
+    """Buffers a call allocates for the caller (out, workspace) come from torch's current
+    stream.  When the call runs on another stream, order that stream after their
+    allocation and zero-fill, and tell the caching allocator that the stream uses them.
+    A raw stream handle cannot be ordered from here: the caller passes the buffers."""
+    tensors = [t for t in tensors if t is not None]
+    if stream is None or not tensors:
+        return
+    if isinstance(stream, int):
+        raise ValueError("with a raw stream handle, pass out= and workspace= allocated for it")
+    import torch
+    cur = torch.cuda.current_stream(stream.device)
+    if stream != cur:
+        stream.wait_stream(cur)
+        for t in tensors:
+            t.record_stream(stream)
+
+
 def _act(x, dims: Dims):
     import torch
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != dims.d or not x.is_contiguous():
@@ -213,15 +231,20 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
                      top_e: int | None = None):
     """One sparse-MoE block decode step: out[t] = sum_e w_te * (gathered SwiGLU over the
     k top-scoring channels + A_e B_e x_t).  x: bf16 [B][d] on the GPU.  top_e: route each
-    token to this many experts instead of the trained layer.dims.top_e (at most that)."""
+    token to this many experts instead of the trained layer.dims.top_e (at most that).
+    out and workspace are allocated when not given (pass both for repeated calls and for
+    a raw stream handle); the call is asynchronous on `stream` (default: torch's current
+    stream)."""
     import torch
     dims = layer.dims
     _act(x, dims)
     B = x.shape[0]
+    new_out = new_ws = None
     if out is None:
-        out = torch.empty_like(x)
+        out = new_out = torch.empty_like(x)
     if workspace is None:
-        workspace = Workspace(dims, B, x.device)
+        workspace = new_ws = Workspace(dims, B, x.device)
+    _temporaries_on(stream, [new_out, new_ws.buf if new_ws else None])
     tr = trace.c() if trace is not None else None
     flags = _lib.MSB_FLAG_GENERAL if general else 0
     args = (_ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
@@ -247,6 +270,7 @@ def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Tra
         raise ValueError("moe_sparse_block_noalloc takes one token")
     if out is None:
         out = torch.empty_like(x)
+        _temporaries_on(stream, [out])
     tr = trace.c() if trace is not None else None
     rc = _lib.load().moe_sparse_block_noalloc(
         _ptr(x), _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch), _ptr(layer.alpha),
@@ -264,10 +288,12 @@ def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
     dims = layer.dims
     _act(x, dims)
     B = x.shape[0]
+    new_out = new_ws = None
     if out is None:
-        out = torch.empty_like(x)
+        out = new_out = torch.empty_like(x)
     if workspace is None:
-        workspace = Workspace(dims, B, x.device)
+        workspace = new_ws = Workspace(dims, B, x.device)
+    _temporaries_on(stream, [new_out, new_ws.buf if new_ws else None])
     tr = trace.c() if trace is not None else None
     rc = _lib.load().moe_sparse_block_threshold(
         _ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
