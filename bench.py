@@ -228,7 +228,7 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
-METRIC = "MoE-block decode tokens/s (achieved HBM GB/s vs peak) at B=1, 18% budget"
+METRIC = "MoE-block decode tokens/s and achieved HBM GB/s vs peak at B=1, 18% budget"
 
 
 def config_of(w, args):
