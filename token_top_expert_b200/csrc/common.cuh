@@ -103,22 +103,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// Same with an L2 evict-first hint (streamed-once weights).
-__device__ __forceinline__ void bulk_g2s_stream(void* dst, const void* src, uint32_t bytes,
-                                                uint64_t* bar, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], "
-      "%2, [%3], %4;" ::"r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(policy)
-      : "memory");
-}
-
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-
 // D += A*B with A 16x16 bf16 (row), B 16x8 bf16 (col), D 16x8 fp32.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -158,19 +142,6 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b, float acc) {
   acc = fmaf(bf16_hi(a.z), bf16_hi(b.z), acc);
   acc = fmaf(bf16_lo(a.w), bf16_lo(b.w), acc);
   acc = fmaf(bf16_hi(a.w), bf16_hi(b.w), acc);
-  return acc;
-}
-
-// 8 bf16 dot 8 fp32
-__device__ __forceinline__ float dot8f(uint4 a, const float* x, float acc) {
-  acc = fmaf(bf16_lo(a.x), x[0], acc);
-  acc = fmaf(bf16_hi(a.x), x[1], acc);
-  acc = fmaf(bf16_lo(a.y), x[2], acc);
-  acc = fmaf(bf16_hi(a.y), x[3], acc);
-  acc = fmaf(bf16_lo(a.z), x[4], acc);
-  acc = fmaf(bf16_hi(a.z), x[5], acc);
-  acc = fmaf(bf16_lo(a.w), x[6], acc);
-  acc = fmaf(bf16_hi(a.w), x[7], acc);
   return acc;
 }
 
