@@ -420,6 +420,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=synth.QWEN30B_BLOCK.name, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--budget", type=float, default=None,
+                    help="read budget as a fraction of I (k = round(budget * I)); --k wins")
     ap.add_argument("--batch", type=int, default=None)
     ap.add_argument("--rank", type=int, default=None)
     ap.add_argument("--replicas", type=int, default=8)
@@ -434,6 +436,10 @@ def main():
                     help="measure the calibrated-threshold comparator instead of top-k")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
+    if args.k is None and args.budget is not None:
+        if not 0.0 < args.budget <= 1.0:
+            ap.error("--budget must lie in (0, 1]")
+        args.k = max(1, synth.budget_k(args.budget, w.inter))
     args.k = w.k if args.k is None else args.k
     args.batch = w.batch if args.batch is None else args.batch
     args.rank = w.rank if args.rank is None else args.rank

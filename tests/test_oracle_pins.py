@@ -324,6 +324,15 @@ def test_tiny_workload_budget_invariant():
 
 # ----------------------------------------------------------------------------- generator
 
+def test_budget_to_k_reproduces_every_stated_k():
+    """k = round(budget * I): the 18 % and 13 % budgets of I = 768 give the workloads'
+    k = 138 and 100, 18 % of I = 1536 gives 276; 100 % is every channel."""
+    assert synth.budget_k(0.18, 768) == 138 == synth.QWEN30B_BLOCK.k
+    assert synth.budget_k(0.13, 768) == 100 == synth.QWEN30B_BLOCK_13.k
+    assert synth.budget_k(0.18, 1536) == 276 == synth.LARGE_BLOCK.k
+    assert synth.budget_k(1.0, 768) == 768
+
+
 def test_generator_determinism_and_shapes():
     w = synth.TINY
     a = synth.expert_gate(w, 3)
