@@ -115,6 +115,8 @@ typedef struct msb_trace {
  *  lr_a      bf16  [E][d][r]     A_e, model layout (not repacked).
  *  lr_b      bf16  [E][r][d]     B_e, model layout (not repacked).
  */
+/* Sizes of the sketch (u32 words) and alpha (floats) outputs for these dims; 0 when
+ * the dims are invalid (any limit below, or top_e > experts). */
 size_t msb_sketch_words(const msb_dims* dims);
 size_t msb_alpha_count(const msb_dims* dims);
 
@@ -126,14 +128,16 @@ size_t msb_alpha_count(const msb_dims* dims);
  * (strict; evaluated exactly as 10*d*|W_i| > 7*sum|W| in double precision) and
  * alpha = mean |W_i| over the kept entries (0 if none), rounded to float.
  * Uses up to `threads` host threads (<= 0: all hardware threads).
- * Returns MSB_OK or MSB_EINVAL / MSB_EUNSUPPORTED. */
+ * Returns MSB_OK, or MSB_EINVAL / MSB_EUNSUPPORTED for a null pointer or dims that
+ * msb_sketch_words rejects (checked before anything is written). */
 int32_t msb_pack(const uint16_t* gate_host, const uint16_t* up_host, const uint16_t* down_host,
                  const uint16_t* router_host, const msb_dims* dims, uint16_t* records_host,
                  uint32_t* sketch_host, float* alpha_host, uint16_t* router_t_host,
                  int32_t threads);
 
 /* ------------------------------------------------------------------ workspace
- * Bytes of device workspace a call with up to max_batch tokens needs.  The
+ * Bytes of device workspace a call with up to max_batch tokens needs (0 for
+ * invalid dims or max_batch outside 1..MSB_MAX_BATCH).  The
  * workspace must be zero-filled once before its first use (msb_workspace_init);
  * every call leaves it ready for the next.  Calls that share a workspace must
  * not overlap on the GPU (same stream, or ordered by events). */
