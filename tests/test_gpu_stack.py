@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import synth
-from parity import OUT_RTOL, compare, from_bf16_tensor, require_gpu, to_bf16_tensor
+from parity import compare, from_bf16_tensor, require_gpu, to_bf16_tensor
 
 pytestmark = pytest.mark.gpu
 

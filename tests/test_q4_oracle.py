@@ -10,7 +10,6 @@ the degenerate constant group; the layer wrapper by a layer whose down columns l
 grid along d only (a wrapper that grouped down along I would change them).
 """
 import numpy as np
-import pytest
 
 import oracle
 import synth
