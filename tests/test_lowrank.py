@@ -106,3 +106,20 @@ def test_factors_are_the_leading_singular_directions():
     tail = np.sqrt((s[r:] ** 2).sum())
     # Eckart-Young, up to the BF16 rounding of the factors
     assert resid == pytest.approx(tail, rel=0.05, abs=1e-2 * s[0])
+
+
+def test_leading_factors_of_a_product():
+    """With n < d the SVD of the n x n QR core gives the singular values and the rank-r
+    truncation of p @ q that a direct SVD of the d x d product gives; asking for more
+    triplets than the product's rank pads with zeros."""
+    rng = np.random.default_rng(9)
+    d, n, r = 80, 24, 6
+    p, q = rng.normal(size=(d, n)), rng.normal(size=(n, d))
+    u, s, vt = lowrank.leading_factors(p, q, r)
+    u0, s0, vt0 = np.linalg.svd(p @ q)
+    np.testing.assert_allclose(s, s0[:r], rtol=1e-10)
+    np.testing.assert_allclose(u * s @ vt, u0[:, :r] * s0[:r] @ vt0[:r], atol=1e-9 * s0[0])
+    np.testing.assert_allclose(u.T @ u, np.eye(r), atol=1e-10)
+    u, s, vt = lowrank.leading_factors(p, q, n + 3)
+    assert s.shape == (n + 3,) and not s[n:].any() and not u[:, n:].any() and not vt[n:].any()
+    np.testing.assert_allclose(u * s @ vt, p @ q, atol=1e-9 * s0[0])
