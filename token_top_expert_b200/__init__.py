@@ -20,4 +20,4 @@ from .block import (  # noqa: F401
     sketch_words,
     workspace_size,
 )
-from . import lowrank, packfile  # noqa: F401,E402
+from . import checkpoint, lowrank, packfile  # noqa: F401,E402
