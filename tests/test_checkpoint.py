@@ -1,5 +1,7 @@
 """Weights in from safetensors checkpoints (host only): a small Qwen3-MoE-named model
 written with the safetensors library, read back by the package's own reader."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -115,3 +117,23 @@ def test_missing_or_malformed_tensors_are_reported(msb, tmp_path):
     open(p, "wb").write(raw[:20])
     with pytest.raises(checkpoint.CheckpointError):
         checkpoint.Shards(p)
+
+
+def test_prepare_writes_one_checked_file_per_moe_layer(msb, tmp_path):
+    from token_top_expert_b200 import checkpoint, packfile, prepare
+    w, lw, paths = _model(tmp_path)
+    out = tmp_path / "packed"
+    assert prepare.main(["--out", str(out), "--top-e", "2", "--rank", "4", "--k", "12",
+                         "--lowrank-samples", "256"] + paths) == 0
+    assert sorted(os.listdir(out)) == ["layer_001.msbpack"]
+    dims, rec, packed, a, b, meta = packfile.load(str(out / "layer_001.msbpack"))
+    assert meta == {"shards": [os.path.basename(p) for p in paths], "layer": 1, "k": 12}
+    d0, p0, a0, b0 = checkpoint.pack_layer(checkpoint.Shards(paths), 1, top_e=2, rank=4, k=12,
+                                           lowrank_samples=256)
+    assert dims == d0 and rec == "bf16"
+    for k in p0:
+        np.testing.assert_array_equal(packed[k], p0[k])
+    np.testing.assert_array_equal(a, a0)
+    np.testing.assert_array_equal(b, b0)
+    with pytest.raises(SystemExit):
+        prepare.main(["--out", str(out), "--top-e", "2", "--rank", "4"] + paths)   # no --k
