@@ -241,3 +241,39 @@ def test_raw_stream_handle_needs_caller_buffers():
     block._temporaries_on(12345, [None, None])    # caller gave every buffer
     with pytest.raises(ValueError):
         block._temporaries_on(12345, [object()])
+
+
+def test_binding_checks_buffers_before_launch(msb):
+    """The binding refuses buffers the kernels would overrun or misread -- out not
+    shaped like x, a trace laid out for another K or k, tensors on another device --
+    before it allocates or launches anything (CPU tensors stand in for device ones;
+    every case raises before the C call)."""
+    import torch
+    dims = msb.Dims(64, 40, 4, 2, 0)
+    z = lambda *s, dt=torch.int16, dev="cpu": torch.zeros(*s, dtype=dt, device=dev)  # noqa: E731
+    layer = msb.PackedLayer(dims, z(8), z(8, dt=torch.int32), z(4, 48, dt=torch.float32), z(4, 64))
+    x = z(3, 64, dt=torch.bfloat16)
+    with pytest.raises(ValueError, match="out"):
+        msb.moe_sparse_block(x, layer, 8, out=z(2, 64, dt=torch.bfloat16))
+    with pytest.raises(ValueError, match="out"):
+        msb.moe_sparse_block(x, layer, 8, out=z(3, 64))                       # int16, not bf16
+    with pytest.raises(ValueError, match="out"):
+        msb.moe_sparse_block(x, layer, 8, out=z(64, 3, dt=torch.bfloat16).t())
+    with pytest.raises(ValueError, match="trace.sel "):
+        msb.moe_sparse_block(x, layer, 8, trace=msb.Trace(dims, 3, 9, device="cpu"))
+    with pytest.raises(ValueError, match="trace.expert_ids"):
+        msb.moe_sparse_block(x, layer, 8, trace=msb.Trace(dims, 2, 8, device="cpu"))  # 2 < 3 rows
+    with pytest.raises(ValueError, match="trace.expert_ids"):
+        msb.moe_sparse_block(x, layer, 8, top_e=1, trace=msb.Trace(dims, 3, 8, device="cpu"))
+    with pytest.raises(ValueError, match="trace.sel "):                      # needs capacity I
+        msb.moe_sparse_block_threshold(x, layer, 0.5, trace=msb.Trace(dims, 3, 8, device="cpu"))
+    with pytest.raises(ValueError, match="trace.scores"):
+        tr = msb.Trace(dims, 3, 8, device="cpu")
+        tr.scores = z(3, 2, 40, dt=torch.float32)                            # I, not Ipad = 48
+        msb.moe_sparse_block(x, layer, 8, trace=tr)
+    meta = msb.PackedLayer(dims, z(8, dev="meta"), z(8, dt=torch.int32), z(4, 48, dt=torch.float32),
+                           z(4, 64))
+    with pytest.raises(ValueError, match="layer"):
+        msb.moe_sparse_block(x, meta, 8)
+    with pytest.raises(ValueError, match="layer"):
+        msb.moe_sparse_block_noalloc(x[:1], meta, 8)

@@ -217,6 +217,34 @@ def _temporaries_on(stream, tensors):
             t.record_stream(stream)
 
 
+def _check_call(x, layer: PackedLayer, out, trace, K: int, cap: int):
+    """Checks the C ABI cannot make (it sees raw pointers), done before anything is
+    allocated or launched: layer, out and trace on x's device; out shaped like x; the
+    trace laid out for this call (K routed experts per token, `cap` channels per
+    (token, expert) in sel, at least x's batch of rows)."""
+    dev = x.device
+    if layer.records.device != dev:
+        raise ValueError("the layer is on %s, x on %s" % (layer.records.device, dev))
+    if out is not None and (out.shape != x.shape or out.dtype != x.dtype or
+                            not out.is_contiguous() or out.device != dev):
+        raise ValueError("out must be a contiguous bf16 tensor shaped like x, on x's device")
+    if trace is None:
+        return
+    B, dims = x.shape[0], layer.dims
+    want = {"expert_ids": (K,), "expert_w": (K,), "sel_count": (K,), "sel": (K, cap)}
+    if trace.scores is not None:
+        want["scores"] = (K, dims.ipad)
+    for name, tail in want.items():
+        t = getattr(trace, name)
+        if (t.dim() != 1 + len(tail) or t.shape[0] < B or tuple(t.shape[1:]) != tail or
+                not t.is_contiguous() or t.device != dev):
+            raise ValueError("trace.%s is %s on %s; this call needs [>= %d]%s on %s"
+                             % (name, tuple(t.shape), t.device, B, list(tail), dev))
+    u = trace.union_count
+    if u.dim() != 1 or u.shape[0] < dims.experts or u.device != dev:
+        raise ValueError("trace.union_count needs >= %d entries on %s" % (dims.experts, dev))
+
+
 def _act(x, dims: Dims):
     import torch
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != dims.d or not x.is_contiguous():
@@ -238,6 +266,7 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
     import torch
     dims = layer.dims
     _act(x, dims)
+    _check_call(x, layer, out, trace, dims.top_e if top_e is None else top_e, k)
     B = x.shape[0]
     new_out = new_ws = None
     if out is None:
@@ -268,6 +297,7 @@ def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Tra
     _act(x, dims)
     if x.shape[0] != 1:
         raise ValueError("moe_sparse_block_noalloc takes one token")
+    _check_call(x, layer, out, trace, dims.top_e, k)
     if out is None:
         out = torch.empty_like(x)
         _temporaries_on(stream, [out])
@@ -287,6 +317,7 @@ def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
     import torch
     dims = layer.dims
     _act(x, dims)
+    _check_call(x, layer, out, trace, dims.top_e, dims.inter)
     B = x.shape[0]
     new_out = new_ws = None
     if out is None:
