@@ -277,3 +277,10 @@ def test_binding_checks_buffers_before_launch(msb):
         msb.moe_sparse_block(x, meta, 8)
     with pytest.raises(ValueError, match="layer"):
         msb.moe_sparse_block_noalloc(x[:1], meta, 8)
+    h = z(3, 64, dt=torch.float32)
+    with pytest.raises(ValueError, match="h must"):
+        msb.residual_rmsnorm(h.double(), None, x)
+    with pytest.raises(ValueError, match="x_next"):
+        msb.residual_rmsnorm(h, None, z(3, 32, dt=torch.bfloat16))
+    with pytest.raises(ValueError, match="y must"):
+        msb.residual_rmsnorm(h, z(3, 64, dt=torch.float32), x)

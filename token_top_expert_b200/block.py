@@ -349,6 +349,13 @@ def path_info(dims: Dims, batch: int, k: int, general: bool = False) -> dict:
 
 def residual_rmsnorm(h, y, x_next, eps: float = 1e-6, stream=None):
     """h += y (FP32 residual, y bf16 or None); x_next = BF16(RMSNorm(h))."""
+    import torch
+    if h.dtype != torch.float32 or h.dim() != 2 or not h.is_contiguous():
+        raise ValueError("h must be a contiguous float32 [batch][d] tensor")
+    for name, t in (("y", y), ("x_next", x_next)):
+        if t is not None and (t.shape != h.shape or t.dtype != torch.bfloat16 or
+                              not t.is_contiguous() or t.device != h.device):
+            raise ValueError("%s must be a contiguous bf16 tensor shaped like h, on h's device" % name)
     B, d = h.shape
     rc = _lib.load().msb_residual_rmsnorm(_ptr(h), _ptr(y), _ptr(x_next), B, d, float(eps),
                                           _stream(stream))
