@@ -251,7 +251,13 @@ def test_binding_checks_buffers_before_launch(msb):
     import torch
     dims = msb.Dims(64, 40, 4, 2, 0)
     z = lambda *s, dt=torch.int16, dev="cpu": torch.zeros(*s, dtype=dt, device=dev)  # noqa: E731
-    layer = msb.PackedLayer(dims, z(8), z(8, dt=torch.int32), z(4, 48, dt=torch.float32), z(4, 64))
+    words = msb.sketch_words(dims)
+
+    def fake_layer(dev="cpu"):
+        return msb.PackedLayer(dims, z(4, 40, 3 * 64, dev=dev), z(words, dt=torch.int32, dev=dev),
+                               z(4, 48, dt=torch.float32, dev=dev), z(4, 64, dev=dev))
+
+    layer = fake_layer()
     x = z(3, 64, dt=torch.bfloat16)
     with pytest.raises(ValueError, match="out"):
         msb.moe_sparse_block(x, layer, 8, out=z(2, 64, dt=torch.bfloat16))
@@ -271,8 +277,7 @@ def test_binding_checks_buffers_before_launch(msb):
         tr = msb.Trace(dims, 3, 8, device="cpu")
         tr.scores = z(3, 2, 40, dt=torch.float32)                            # I, not Ipad = 48
         msb.moe_sparse_block(x, layer, 8, trace=tr)
-    meta = msb.PackedLayer(dims, z(8, dev="meta"), z(8, dt=torch.int32), z(4, 48, dt=torch.float32),
-                           z(4, 64))
+    meta = fake_layer("meta")
     with pytest.raises(ValueError, match="layer"):
         msb.moe_sparse_block(x, meta, 8)
     with pytest.raises(ValueError, match="layer"):
@@ -284,3 +289,34 @@ def test_binding_checks_buffers_before_launch(msb):
         msb.residual_rmsnorm(h, None, z(3, 32, dt=torch.bfloat16))
     with pytest.raises(ValueError, match="y must"):
         msb.residual_rmsnorm(h, z(3, 64, dt=torch.float32), x)
+
+
+def test_packed_layer_checks_its_tensors(msb):
+    import torch
+    dims = msb.Dims(64, 40, 4, 2, 2)
+    z = lambda *s, dt=torch.int16: torch.zeros(*s, dtype=dt)  # noqa: E731
+    ok = dict(records=z(4, 40, 192), sketch=z(msb.sketch_words(dims), dt=torch.int32),
+              alpha=z(4, 48, dt=torch.float32), router_t=z(4, 64), lr_a=z(4, 64, 2), lr_b=z(4, 2, 64))
+    msb.PackedLayer(dims, **ok)
+    for name, bad in (("records", z(4, 40, 191)), ("sketch", z(7, dt=torch.int32)),
+                      ("alpha", z(4, 40, dt=torch.float32)), ("alpha", z(4, 48, dt=torch.int32)),
+                      ("router_t", z(64, 4).t()), ("lr_a", None), ("lr_b", z(4, 2, 64, dt=torch.int32))):
+        with pytest.raises(ValueError, match=name):
+            msb.PackedLayer(dims, **dict(ok, **{name: bad}))
+    with pytest.raises(ValueError, match="dims"):
+        msb.PackedLayer(msb.Dims(64, 40, 4, 5, 0), **dict(ok, lr_a=None, lr_b=None))
+
+
+def test_from_host_takes_the_leading_factors_of_a_lower_rank(msb):
+    dims = msb.Dims(64, 40, 4, 2, 2)
+    rng = np.random.default_rng(1)
+    packed = {"records": np.zeros((4, 40, 192), np.uint16),
+              "sketch": np.zeros(msb.sketch_words(dims), np.uint32),
+              "alpha": np.zeros((4, 48), np.float32), "router_t": np.zeros((4, 64), np.uint16)}
+    a = rng.integers(0, 2**15, (4, 64, 5)).astype(np.uint16)
+    b = rng.integers(0, 2**15, (4, 5, 64)).astype(np.uint16)
+    lay = msb.PackedLayer.from_host(dims, packed, a, b, device="cpu")
+    np.testing.assert_array_equal(lay.lr_a.numpy().view(np.uint16), a[:, :, :2])
+    np.testing.assert_array_equal(lay.lr_b.numpy().view(np.uint16), b[:, :2, :])
+    with pytest.raises(ValueError, match="lr_a"):
+        msb.PackedLayer.from_host(msb.Dims(64, 40, 4, 2, 8), packed, a, b, device="cpu")

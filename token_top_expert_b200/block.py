@@ -117,19 +117,46 @@ class PackedLayer:
         self.dims = dims
         self.records, self.sketch, self.alpha, self.router_t = records, sketch, alpha, router_t
         self.lr_a, self.lr_b = lr_a, lr_b
+        self._check()
+
+    def _check(self):
+        """Sizes, element types and device of every tensor against the dims, so that the
+        kernels never read past a buffer (done once, at construction)."""
+        d, I, E, r = self.dims.d, self.dims.inter, self.dims.experts, self.dims.rank
+        words = sketch_words(self.dims)
+        if words == 0:
+            raise ValueError("dims rejected by the library: %s" % (self.dims,))
+        want = [("records", self.records, E * I * 3 * d, 2), ("sketch", self.sketch, words, 4),
+                ("alpha", self.alpha, E * self.dims.ipad, 4), ("router_t", self.router_t, E * d, 2)]
+        if r > 0:
+            want += [("lr_a", self.lr_a, E * d * r, 2), ("lr_b", self.lr_b, E * r * d, 2)]
+        dev = self.records.device
+        for name, t, numel, size in want:
+            if t is None:
+                raise ValueError("%s is required (rank %d)" % (name, r))
+            if (t.numel() != numel or t.element_size() != size or not t.is_contiguous() or
+                    t.device != dev or (name == "alpha" and not t.dtype.is_floating_point)):
+                raise ValueError("%s: expected %d contiguous %d-byte elements on %s, got %s %s on %s"
+                                 % (name, numel, size, dev, t.dtype, tuple(t.shape), t.device))
 
     @classmethod
     def from_host(cls, dims: Dims, packed: dict, lr_a: np.ndarray | None, lr_b: np.ndarray | None,
                   device="cuda"):
+        """Upload host arrays (``pack`` output, BF16 factor bits).  Factors of a rank above
+        dims.rank contribute their first dims.rank columns of A_e and rows of B_e."""
         import torch
 
         def t(a):
             return torch.from_numpy(np.ascontiguousarray(a)).to(device)
 
+        r = dims.rank
+        if r > 0 and lr_a is not None and lr_b is not None:
+            # factors of a higher rank: the first r columns of A_e and rows of B_e
+            lr_a, lr_b = lr_a[:, :, :r], lr_b[:, :r, :]
         return cls(dims, t(packed["records"].view(np.int16)), t(packed["sketch"].view(np.int32)),
                    t(packed["alpha"]), t(packed["router_t"].view(np.int16)),
-                   None if lr_a is None or dims.rank == 0 else t(lr_a.view(np.int16)),
-                   None if lr_b is None or dims.rank == 0 else t(lr_b.view(np.int16)))
+                   None if lr_a is None or r == 0 else t(lr_a.view(np.int16)),
+                   None if lr_b is None or r == 0 else t(lr_b.view(np.int16)))
 
     def clone(self) -> "PackedLayer":
         """A copy at different addresses (same values)."""
