@@ -246,10 +246,16 @@ def _temporaries_on(stream, tensors):
 
 def _check_call(x, layer: PackedLayer, out, trace, K: int, cap: int):
     """Checks the C ABI cannot make (it sees raw pointers), done before anything is
-    allocated or launched: layer, out and trace on x's device; out shaped like x; the
+    allocated or launched: x on the current device; layer, out and trace on x's device;
+    out shaped like x; the
     trace laid out for this call (K routed experts per token, `cap` channels per
     (token, expert) in sel, at least x's batch of rows)."""
     dev = x.device
+    if dev.type == "cuda":
+        import torch
+        if dev.index != torch.cuda.current_device():
+            raise ValueError("x is on %s but the current device is cuda:%d (the library "
+                             "launches on the current device)" % (dev, torch.cuda.current_device()))
     if layer.records.device != dev:
         raise ValueError("the layer is on %s, x on %s" % (layer.records.device, dev))
     if out is not None and (out.shape != x.shape or out.dtype != x.dtype or
