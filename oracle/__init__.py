@@ -26,6 +26,9 @@ and cites the passage it follows.  Sources (web pages, by title and section):
   The pages name a "ternary sketch" without its formula; TWN is the reading
   adopted for it.
 
+A second restatement in plain C99 (``oracle/c/msb_oracle.c``, loaded through
+``oracle.c_oracle``) is held against this one by ``tests/test_oracle_c.py``.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 against closed forms, hand-worked examples (``tests/golden/``), brute force or
 library routines -- except the exact GPU outputs at k < I, which have no worked
