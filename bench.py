@@ -161,14 +161,15 @@ def replica_throughput(ms_local: float, units_per_rank: float, dist=None, device
 def algorithmic_bytes(w, k, rank, union_sizes, dense):
     """Bytes the method must read for one step: per used expert the sketch
     (I*d/4), row scales (4I), the union of selected channel records (6d each)
-    and A_e, B_e (4dr).  The dense path reads only channel records."""
+    and A_e, B_e (4dr).  The dense path (k = I) reads no sketch or scales; it still
+    adds the low-rank term when rank > 0."""
     total = 0
     for u in union_sizes:
         if u == 0:
             continue
-        total += 6 * w.d * int(u)
+        total += 6 * w.d * int(u) + 4 * w.d * rank
         if not dense:
-            total += w.inter * w.d // 4 + 4 * w.inter + 4 * w.d * rank
+            total += w.inter * w.d // 4 + 4 * w.inter
     return total
 
 
