@@ -158,6 +158,15 @@ def replica_throughput(ms_local: float, units_per_rank: float, dist=None, device
     return ms, units_per_rank * world / (ms / 1e3)
 
 
+def block_launches(path, dense, rank):
+    """Kernels one block call launches: the single-launch kernel, or the multi-kernel
+    path's router, score (not for a dense block without compensation), select (not
+    dense), union, gather and finalize."""
+    if path == "single_launch":
+        return 1
+    return 4 + (1 if (not dense or rank > 0) else 0) + (0 if dense else 1)
+
+
 def algorithmic_bytes(w, k, rank, union_sizes, dense):
     """Bytes the method must read for one step: per used expert the sketch
     (I*d/4), row scales (4I), the union of selected channel records (6d each)
@@ -340,7 +349,8 @@ def run_stack_one(args, w, local, dev, layers, k, B, rank, setup_s):
         "us_per_layer": ms_per_step * 1e3 / L, "bytes_per_step": byts,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None},
-        "gpu_launches": steps * (2 * L + 1) * (1 if plan["path"] == "single_launch" else 5),
+        # per step: L blocks and L + 1 residual/RMSNorm launches
+        "gpu_launches": steps * (L * block_launches(plan["path"], dense, rank) + L + 1),
         "clocks": clk.summary(), "setup_s": setup_s,
     }
     print(json.dumps(line), flush=True)
@@ -586,8 +596,7 @@ def main():
                          args.k, general=general)
     kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
     traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else ""))
-    launches_per_step = 1 if plan["path"] == "single_launch" else (
-        (3 if args.rank == 0 else 4) if dense else 5)
+    launches_per_step = block_launches(plan["path"], dense, args.rank)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world if world > 1 else 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -42,3 +42,15 @@ def test_large_block_and_budget_totals():
     bench = _bench()
     w = synth.LARGE_BLOCK
     assert bench.algorithmic_bytes(w, 276, 64, [276] * 8, False) == 75_284_480
+
+
+def test_launch_counts_follow_the_launch_sequence():
+    """One launch on the single-launch path; on the multi-kernel path router, score
+    (skipped for a dense block without compensation), select (skipped when dense),
+    union, gather, finalize."""
+    bench = _bench()
+    assert bench.block_launches("single_launch", False, 32) == 1
+    assert bench.block_launches("multi_kernel", False, 32) == 6
+    assert bench.block_launches("multi_kernel", False, 0) == 6
+    assert bench.block_launches("multi_kernel", True, 0) == 4
+    assert bench.block_launches("multi_kernel", True, 32) == 5
