@@ -424,21 +424,24 @@ def run_threshold(args, w, world, rank, local):
 
 
 def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one process each, under torchrun)")
+    ap.add_argument("--steps", type=int, default=100000, help="timed decode steps")
+    ap.add_argument("--warmup", type=int, default=20, help="untimed warm-up steps")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
+                    help="ours: the CUDA library; reference: the FP64 CPU oracle on a bounded sample")
     ap.add_argument("--workload", default=synth.QWEN30B_BLOCK.name, choices=sorted(synth.WORKLOADS))
-    ap.add_argument("--k", type=int, default=None)
+    ap.add_argument("--k", type=int, default=None, help="channels kept per (token, expert)")
     ap.add_argument("--budget", type=float, default=None,
                     help="read budget as a fraction of I (k = round(budget * I)); --k wins")
-    ap.add_argument("--batch", type=int, default=None)
-    ap.add_argument("--rank", type=int, default=None)
-    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--batch", type=int, default=None, help="tokens per step")
+    ap.add_argument("--rank", type=int, default=None, help="compensation rank r (0: none)")
+    ap.add_argument("--replicas", type=int, default=8,
+                    help="weight copies rotated per step so that every step reads HBM")
     ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle timing")
+    ap.add_argument("--e2e-steps", type=int, default=2000,
+                    help="steps of the end-to-end measurement (host copies in the timed region)")
     ap.add_argument("--top-e", type=int, default=None,
                     help="route each token to this many experts (at most the trained count)")
     ap.add_argument("--stack-grid", action="store_true",
