@@ -240,6 +240,86 @@ def run_reference(args, w, world, rank):
 
 METRIC = "MoE-block decode tokens/s and achieved HBM GB/s vs peak at B=1, 18% budget"
 
+# %globaltimer marks of the single-launch kernel (instrumented build), in kernel order
+PHASE_MARKS = ("start", "x and router rows in", "logits in", "experts ranked", "sketch tiles in",
+               "sketch scored", "scores and z pushed", "scores in", "top-k selected",
+               "positions found", "records issued, A_e z done", "first record pair used",
+               "records done", "partial outputs in", "end")
+
+
+def run_phase_marks(args, w, local):
+    """Per-phase timeline of the single-launch kernel from its instrumented build
+    (libmsb_instr.so): `steps` launches captured back to back in one CUDA graph (weight
+    replicas rotated, as in the timed bench), each CTA's %globaltimer at every phase
+    boundary.  Times are relative to the moment the step's last CTA had x and its router
+    rows (the end of the wait for the previous launch).  Prints one JSON line."""
+    import torch
+    import token_top_expert_b200 as msb
+    from token_top_expert_b200 import _lib
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lw = synth.layer_weights(w)
+    dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
+    pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
+    base = msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev)
+    del lw, pk
+    layers = [base] + [base.clone() for _ in range(args.replicas - 1)]
+    plan = msb.path_info(dims, 1, args.k)
+    if plan["path"] != "single_launch":
+        raise SystemExit("phase marks need the single-launch path, got %s" % plan)
+    n = max(8, min(args.steps, 400))
+    grid = plan["cluster_size"] * w.top_e
+    nseq = min(w.steps, 1000)
+    xs = torch.from_numpy(np.stack([synth.activations(w, s) for s in range(nseq)]).view(np.int16)).to(dev).view(torch.bfloat16)
+    outs = torch.empty_like(xs)
+    ws = msb.Workspace(dims, 1, dev)
+    marks = torch.zeros((n, grid, 16), dtype=torch.int64, device=dev)
+    stream = torch.cuda.Stream(dev)
+    lib = _lib.load()
+
+    def launch(i, mk):
+        lib.msb_debug_set_marks(mk)
+        msb.moe_sparse_block(xs[i % nseq], layers[i % args.replicas], args.k, out=outs[i % nseq],
+                             workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            launch(i, None)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(n):
+            launch(i, marks[i].data_ptr())
+    lib.msb_debug_set_marks(None)
+    graph.replay()
+    graph.replay()
+    stream.synchronize()
+    ws.check(stream)
+    m = marks.cpu().numpy().astype(np.float64)
+    t = m[:, :, :len(PHASE_MARKS)]
+    t0 = t[:, :, 1].max(axis=1)[:, None, None]  # every CTA has x: the step's work starts
+    rel = (t - t0) / 1e3  # us
+    skip = min(4, n // 4)
+    rel = rel[skip:]
+    ends = t[skip:, :, len(PHASE_MARKS) - 1].max(axis=1)
+    period = float(np.median(np.diff(ends))) / 1e3
+    phases = []
+    for i, name in enumerate(PHASE_MARKS):
+        v = rel[:, :, i]
+        phases.append({"mark": name, "median_us": round(float(np.median(v)), 3),
+                       "max_us": round(float(np.median(v.max(axis=1))), 3)})
+    smids = m[skip, :, 15].astype(int)
+    per_sm = np.bincount(smids, minlength=148)
+    line = {"metric": "single-launch kernel phase timeline (median over launches)",
+            "workload": w.name, "k": args.k, "rank": args.rank, "launches": int(rel.shape[0]),
+            "ctas": grid, "plan": plan, "period_us": round(period, 3),
+            "sms_used": int((per_sm > 0).sum()), "sms_with_two_ctas": int((per_sm > 1).sum()),
+            "phases": phases, "source_hash": kernel_source_hash(),
+            "note": "times relative to the moment the step's last CTA had x and its router rows; "
+                    "median = median over CTAs, max = slowest CTA (both medians over launches)"}
+    print(json.dumps(line), flush=True)
+    del graph
+
 
 def config_of(w, args):
     return {"workload": w.name, "d": w.d, "I": w.inter, "E": w.experts,
@@ -448,6 +528,8 @@ def main():
                     help="stacked workload: run k in {13%%, 18%%, 100%%} x batch in {1, 32} on one set of layers")
     ap.add_argument("--threshold", action="store_true",
                     help="measure the calibrated-threshold comparator instead of top-k")
+    ap.add_argument("--phase-marks", action="store_true",
+                    help="per-phase timeline of the single-launch kernel (instrumented build)")
     args = ap.parse_args()
     w = synth.WORKLOADS[args.workload]
     if args.k is None and args.budget is not None:
@@ -464,6 +546,12 @@ def main():
 
     if args.impl == "reference":
         run_reference(args, w, world, rank)
+        return
+    if args.phase_marks:
+        os.environ["MSB_VARIANT"] = "instr"
+        from token_top_expert_b200 import build as _bm
+        _bm.build(variant="instr")
+        run_phase_marks(args, w, local)
         return
     if w.layers > 1 or args.threshold:
         from token_top_expert_b200 import build as _bld
@@ -568,30 +656,46 @@ def main():
     ms_per_step = ms / args.steps
     ws.check(stream)
 
-    # ---- e2e: public call per step with pinned host x -> device -> host out
+    # ---- e2e: the C-ABI call on host buffers, per step: pinned host x -> device, the
+    # block, device -> pinned host out (moe_sparse_block_host through HostCall; with
+    # --top-e, the device call between two torch copies)
     xh = torch.from_numpy(np.stack(xs_host).view(np.int16)).view(torch.bfloat16).pin_memory()
     oh = torch.empty_like(xh).pin_memory()
-    xd = torch.empty((B, w.d), dtype=torch.bfloat16, device=dev)
-    od = torch.empty_like(xd)
     ne = min(args.e2e_steps, args.steps)
-    with torch.cuda.stream(stream):
-        for i in range(min(50, ne)):
+    if args.top_e is None:
+        calls = [msb.HostCall(lay, args.k, B, stream=stream, general=general) for lay in layers]
+        xp = [xh[i].data_ptr() for i in range(nseq)]
+        op = [oh[i].data_ptr() for i in range(nseq)]
+
+        def e2e_step(i):
+            calls[i % args.replicas](xp[i % nseq], op[i % nseq])
+    else:
+        xd = torch.empty((B, w.d), dtype=torch.bfloat16, device=dev)
+        od = torch.empty_like(xd)
+
+        def e2e_step(i):
             xd.copy_(xh[i % nseq], non_blocking=True)
             msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
                                  general=general, stream=stream, top_e=args.top_e)
             oh[i % nseq].copy_(od, non_blocking=True)
+    with torch.cuda.stream(stream):
+        for i in range(min(50, ne)):
+            e2e_step(i)
         stream.synchronize()
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         for i in range(ne):
-            xd.copy_(xh[i % nseq], non_blocking=True)
-            msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
-                                 general=general, stream=stream, top_e=args.top_e)
-            oh[i % nseq].copy_(od, non_blocking=True)
+            e2e_step(i)
         a1.record(stream)
         stream.synchronize()
     e2e_ms, e2e_value = replica_throughput(a0.elapsed_time(a1), ne * B, dist, dev)
+    # the host results of the last steps match the device results of the same steps (up to
+    # the order of the FP32 reduction-adds across experts)
+    for i in range(max(0, ne - 8), ne):
+        a_, b_ = oh[i % nseq].float(), outs[i % nseq].float().cpu()
+        if float((a_ - b_).norm()) > 1e-2 * float(b_.norm()):
+            raise SystemExit("e2e output of step %d differs from the device-timed run" % i)
 
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9

@@ -57,6 +57,9 @@ extern "C" {
 #define MSB_ETIMEOUT (-4)      /* (msb_check) a kernel's bounded wait ran out */
 #define MSB_ENONFINITE (-5)    /* (msb_check) the router met NaN/Inf logits: x or W_router
                                   is not finite (invalid input; the output is undefined) */
+#define MSB_EINTERNAL (-6)     /* (msb_check) a kernel's internal consistency check failed
+                                  (e.g. a channel selection of the wrong size); the access
+                                  it guarded was skipped and the output is undefined */
 
 /* ------------------------------------------------------------------ limits */
 #define MSB_MAX_D 8192         /* hidden size d: multiple of 64, 64..8192 */
@@ -145,8 +148,8 @@ size_t msb_workspace_size(const msb_dims* dims, int32_t max_batch);
 int32_t msb_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, reads and clears the workspace's sticky error word.
- * Returns MSB_OK, MSB_ETIMEOUT, MSB_ENONFINITE, or MSB_ECUDA if the stream
- * itself failed. */
+ * Returns MSB_OK, MSB_EINTERNAL, MSB_ETIMEOUT, MSB_ENONFINITE (in that order of
+ * precedence when several were flagged), or MSB_ECUDA if the stream itself failed. */
 int32_t msb_check(void* workspace, void* stream);
 
 const char* msb_strerror(int32_t status);
@@ -203,6 +206,22 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
                                size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
                                void* stream);
 
+/* The block on activations in host memory: copies x_host to x_dev, runs
+ * moe_sparse_block(x_dev -> out_dev) and copies out_dev to out_host, all enqueued on
+ * `stream` with cudaMemcpyAsync (no synchronisation: the host buffers must stay
+ * valid, and out_host unread, until the stream has passed the copies).  Use pinned
+ * host memory (cudaHostAlloc / torch pin_memory) for asynchronous copies.
+ *  x_host, out_host  bf16 [batch][d] host memory, not overlapping each other.
+ *  x_dev, out_dev    bf16 [batch][d] device staging buffers (as x and out of
+ *                    moe_sparse_block: 16-byte aligned, not overlapping).
+ * The other arguments are those of moe_sparse_block (no trace).  Every argument is
+ * checked before anything is enqueued; on an error nothing is copied. */
+int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, const void* router_t,
+                              const void* records, const uint32_t* sketch, const float* alpha,
+                              int32_t k, const void* lr_a, const void* lr_b, void* out_dev,
+                              void* out_host, const msb_dims* dims, void* workspace,
+                              size_t workspace_bytes, uint32_t flags, void* stream);
+
 /* The calibrated-threshold selector that the pages compare top-k against
  * ("The threshold promises a budget but does not keep it"): identical to
  * moe_sparse_block except S_{t,e} = { j : score_j > tau }, so the number of
@@ -230,14 +249,22 @@ int32_t moe_sparse_block_threshold(const void* x, int32_t batch, const void* rou
  * The first call on a device looks up the array's device address (do that
  * first call before any stream capture).  Every call clears the part of the
  * array it uses on `stream` and then launches; all calls share the array, so
- * calls that overlap on the GPU (unordered streams) race.  A bounded wait that
- * ran out inside the kernel is not reported by this entry point (there is no
- * workspace for msb_check to read); the output of such a call is undefined. */
+ * calls that overlap on the GPU (unordered streams) race.  What the kernel
+ * flags (a non-finite router logit, a bounded wait that ran out, a failed
+ * consistency check; the output of such a call is undefined) stays in the
+ * array's error word until the next call clears it: read it with
+ * msb_noalloc_check before that next call. */
 #define MSB_NOALLOC_MAX_D 8192
 int32_t moe_sparse_block_noalloc(const void* x, const void* router_t, const void* records,
                                  const uint32_t* sketch, const float* alpha, int32_t k,
                                  const void* lr_a, const void* lr_b, void* out,
                                  const msb_dims* dims, const msb_trace* trace, void* stream);
+
+/* Status of the last moe_sparse_block_noalloc call on the current device: synchronises
+ * `stream`, reads the static array's error word and clears it.  Returns MSB_OK,
+ * MSB_EINTERNAL, MSB_ETIMEOUT, MSB_ENONFINITE (as msb_check), or MSB_ECUDA.  Call it
+ * after the call whose status is wanted and before the next allocation-free call. */
+int32_t msb_noalloc_check(void* stream);
 
 /* Stack glue between decode layers (attention omitted):
  *   h[t] += y[t]            (h float [batch][d], y bf16 [batch][d]; y may be NULL: no add)

@@ -25,10 +25,14 @@ def msb():
     return m
 
 
-def header_functions():
+INSTR_HEADER = "msb_instr.h"  # entry points of the instrumented build only
+
+
+def header_functions(instrumented=False):
     inc = os.path.join(ROOT, "include")
-    text = "".join(open(os.path.join(inc, f)).read() for f in sorted(os.listdir(inc))
-                   if f.endswith(".h"))
+    names = [f for f in sorted(os.listdir(inc)) if f.endswith(".h")]
+    names = [f for f in names if (f == INSTR_HEADER) == instrumented]
+    text = "".join(open(os.path.join(inc, f)).read() for f in names)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)
     return sorted(set(names))
@@ -42,6 +46,23 @@ def test_library_exports_every_declared_symbol(msb):
     lib = ctypes.CDLL(_lib.LIB_PATH)
     for name in declared:
         assert hasattr(lib, name), name
+    # the product library carries none of the instrumented build's entry points
+    for name in header_functions(instrumented=True):
+        assert not hasattr(lib, name), name
+
+
+def test_instrumented_library_exports_its_entry_points():
+    from token_top_expert_b200 import build
+    path = build.build(variant="instr")
+    lib = ctypes.CDLL(path)
+    extra = header_functions(instrumented=True)
+    assert extra == ["msb_debug_inject", "msb_debug_set_marks"]
+    for name in header_functions() + extra:
+        assert hasattr(lib, name), name
+    lib.msb_debug_inject.restype = ctypes.c_int32
+    lib.msb_debug_inject.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
+    assert lib.msb_debug_inject(3, 0) == -1   # MSB_EINVAL: no such injection
+    assert lib.msb_debug_inject(0, 0) == 0
 
 
 def decode_sketch(words, dims, e):

@@ -6,6 +6,7 @@ include/msb.h); this package only marshals arguments to it.
 from ._lib import MsbError, load as load_library  # noqa: F401
 from .block import (  # noqa: F401
     Dims,
+    HostCall,
     PackedLayer,
     Trace,
     Workspace,
@@ -13,6 +14,7 @@ from .block import (  # noqa: F401
     moe_sparse_block,
     moe_sparse_block_noalloc,
     moe_sparse_block_threshold,
+    noalloc_check,
     pack,
     pack_q4,
     path_info,

@@ -8,7 +8,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmsb.so")
+# MSB_VARIANT=instr selects the instrumented build (phase marks, wait-expiry injection)
+VARIANT = os.environ.get("MSB_VARIANT") or None
+LIB_PATH = os.path.join(_HERE, "libmsb_instr.so" if VARIANT == "instr" else "libmsb.so")
 
 MSB_OK = 0
 MSB_EINVAL = -1
@@ -16,6 +18,7 @@ MSB_EUNSUPPORTED = -2
 MSB_ECUDA = -3
 MSB_ETIMEOUT = -4
 MSB_ENONFINITE = -5
+MSB_EINTERNAL = -6
 MSB_FLAG_GENERAL = 1
 
 MSB_MAX_D = 8192
@@ -30,7 +33,8 @@ SYMBOLS = (
     "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_workspace_size",
     "msb_workspace_init", "msb_check", "msb_strerror", "moe_sparse_block",
     "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
-    "moe_sparse_block_noalloc", "moe_sparse_block_top_e",
+    "moe_sparse_block_noalloc", "msb_noalloc_check", "moe_sparse_block_top_e",
+    "moe_sparse_block_host",
     "msb_q4_record_bytes", "msb_pack_q4",
 )
 MSB_Q4_GROUP = 64
@@ -63,8 +67,8 @@ def load() -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libmsb.so is not built (%s); run `python -m token_top_expert_b200.build`"
-                          % LIB_PATH)
+        raise ImportError("%s is not built; run `python -m token_top_expert_b200.build%s`"
+                          % (LIB_PATH, " --instrumented" if VARIANT == "instr" else ""))
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, U32, SZ, F32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_float
     dims_p = ctypes.POINTER(MsbDims)
@@ -85,9 +89,15 @@ def load() -> ctypes.CDLL:
         "msb_residual_rmsnorm": (I32, [P, P, P, I32, I32, F32, P]),
         "msb_path_info": (I32, [dims_p, I32, I32, U32, P]),
         "moe_sparse_block_noalloc": (I32, [P, P, P, P, P, I32, P, P, P, dims_p, trace_p, P]),
+        "msb_noalloc_check": (I32, [P]),
         "moe_sparse_block_top_e": (I32, [P, I32, P, P, P, P, I32, I32, P, P, P, dims_p, P, SZ,
                                          trace_p, U32, P]),
+        "moe_sparse_block_host": (I32, [P, P, I32, P, P, P, P, I32, P, P, P, P, dims_p, P, SZ,
+                                        U32, P]),
     }
+    if VARIANT == "instr":
+        sig["msb_debug_set_marks"] = (I32, [P])
+        sig["msb_debug_inject"] = (I32, [U32, ctypes.c_uint64])
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
         fn.restype = res

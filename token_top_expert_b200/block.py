@@ -321,10 +321,17 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
     return out
 
 
+def noalloc_check(stream=None):
+    """Raise MsbError if the last moe_sparse_block_noalloc call on the current device
+    was flagged by its kernel (synchronises the stream; clears the flag)."""
+    _check(_lib.load().msb_noalloc_check(_stream(stream)), "moe_sparse_block_noalloc kernel")
+
+
 def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Trace | None = None,
                              stream=None):
     """The batch-1 block without a workspace (scratch is a static device array of
-    the library), for callers that cannot allocate device memory."""
+    the library), for callers that cannot allocate device memory.  Read the call's
+    kernel status with noalloc_check() before the next such call."""
     import torch
     dims = layer.dims
     _act(x, dims)
@@ -341,6 +348,55 @@ def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Tra
         ctypes.byref(tr) if tr is not None else None, _stream(stream))
     _check(rc, "moe_sparse_block_noalloc")
     return out
+
+
+class HostCall:
+    """Repeated block calls on activations in host memory (moe_sparse_block_host): each
+    call copies one [batch][d] bf16 host tensor to the device, runs the block and copies
+    the result back into a host tensor, all enqueued on `stream`.
+
+    The layer, k, batch, device staging buffers, workspace and stream are fixed and
+    checked once, here; a call passes only the two host buffers (pinned host tensors of
+    shape [batch][d], bf16), so the per-step cost on the host is one C call.  The call is
+    asynchronous: synchronise the stream before reading `out_host` or reusing `x_host`."""
+
+    def __init__(self, layer: PackedLayer, k: int, batch: int, stream=None, general: bool = False):
+        import torch
+        dims = layer.dims
+        if not 1 <= k <= dims.inter:
+            raise ValueError("k must lie in 1..%d" % dims.inter)
+        dev = layer.records.device
+        self.batch, self.d = batch, dims.d
+        self.x_dev = torch.empty((batch, dims.d), dtype=torch.bfloat16, device=dev)
+        self.out_dev = torch.empty_like(self.x_dev)
+        self.workspace = Workspace(dims, batch, dev)
+        self._dims = dims.c()
+        self.stream = stream if stream is not None else torch.cuda.current_stream(dev)
+        _temporaries_on(self.stream, [self.x_dev, self.out_dev, self.workspace.buf])
+        self._fn = _lib.load().moe_sparse_block_host
+        self._head = (_ptr(self.x_dev), batch, _ptr(layer.router_t), _ptr(layer.records),
+                      _ptr(layer.sketch), _ptr(layer.alpha), k, _ptr(layer.lr_a), _ptr(layer.lr_b),
+                      _ptr(self.out_dev))
+        self._tail = (ctypes.byref(self._dims), self.workspace.ptr, self.workspace.nbytes,
+                      _lib.MSB_FLAG_GENERAL if general else 0, _stream(self.stream))
+        self._layer = layer  # keep the weights alive
+
+    def check_host(self, t):
+        """A host tensor this call can take (shape, dtype, pinned, contiguous)."""
+        import torch
+        if (t.device.type != "cpu" or t.dtype != torch.bfloat16 or tuple(t.shape) != (self.batch, self.d)
+                or not t.is_contiguous() or not t.is_pinned()):
+            raise ValueError("expected a pinned contiguous bf16 host tensor of shape [%d][%d]"
+                             % (self.batch, self.d))
+        return t
+
+    def __call__(self, x_host, out_host):
+        """x_host, out_host: host tensors accepted by check_host, or their data pointers."""
+        xp = x_host if isinstance(x_host, int) else x_host.data_ptr()
+        op = out_host if isinstance(out_host, int) else out_host.data_ptr()
+        rc = self._fn(xp, *self._head, op, *self._tail)
+        if rc != _lib.MSB_OK:
+            raise MsbError(rc, "moe_sparse_block_host")
 
 
 def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,

@@ -6,6 +6,14 @@ Every .cu / .cpp file under csrc/ is compiled to an object in _build/ (in
 parallel) and linked into token_top_expert_b200/libmsb.so.  The CUDA runtime is
 linked statically, so the library loads on a machine without a GPU (the host
 packer and the argument checks work there).
+
+    python -m token_top_expert_b200.build --instrumented
+
+builds the instrumented variant libmsb_instr.so (objects in _build_instr/): the same
+sources with MSB_INSTRUMENTED defined.  Its single-launch kernel records a
+%globaltimer mark per phase and CTA (read by `bench.py --phase-marks`), and a test can
+make one bounded wait run out on purpose (`msb_debug_inject`; tests/instrumented_check.py).
+The product library is built without either.
 """
 from __future__ import annotations
 
@@ -21,6 +29,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libmsb.so")
+VARIANTS = {None: (BUILD, LIB, []),
+            "instr": (os.path.join(PKG, "_build_instr"), os.path.join(PKG, "libmsb_instr.so"),
+                      ["-DMSB_INSTRUMENTED"])}
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
@@ -44,8 +55,9 @@ def _newer(target: str, deps) -> bool:
     return all(os.path.getmtime(d) <= t for d in deps)
 
 
-def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
+def build(verbose: bool = False, ptxas_verbose: bool = False, variant: str | None = None) -> str:
     """Compile and link; returns the library path.  Raises on any compiler error."""
+    BUILD, LIB, defs = VARIANTS[variant]
     os.makedirs(BUILD, exist_ok=True)
     headers = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
     headers += [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
@@ -58,7 +70,7 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
         objs.append(obj)
         if _newer(obj, [path] + headers):
             continue
-        cmd = [cc] + ARCH + COMMON + ["-c", path, "-o", obj]
+        cmd = [cc] + ARCH + COMMON + defs + ["-c", path, "-o", obj]
         if ptxas_verbose and src.endswith(".cu"):
             cmd += ["-Xptxas", "-v"]
         jobs.append(cmd)
@@ -84,4 +96,5 @@ def build(verbose: bool = False, ptxas_verbose: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv, ptxas_verbose="--ptxas" in sys.argv))
+    print(build(verbose="-v" in sys.argv, ptxas_verbose="--ptxas" in sys.argv,
+                variant="instr" if "--instrumented" in sys.argv else None))

@@ -10,6 +10,14 @@
 #include "msb.h"
 
 namespace msb {
+
+#ifdef MSB_INSTRUMENTED
+DebugCtl& debug_ctl() {
+  static DebugCtl ctl = {nullptr, 0u, 0u};
+  return ctl;
+}
+#endif
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -140,6 +148,32 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+// Argument checks of a block call (no CUDA call): MSB_OK or the error to return.
+int block_check(const void* x, int32_t batch, const void* router_t, const void* records,
+                const uint32_t* sketch, const float* alpha, int32_t k, int mode, float tau,
+                const void* lr_a, const void* lr_b, const void* out, const msb_dims* dims,
+                const void* workspace, size_t workspace_bytes) {
+  int rc = check_dims(dims);
+  if (rc != MSB_OK) return rc;
+  if (batch < 1) return MSB_EINVAL;
+  if (batch > MSB_MAX_BATCH) return MSB_EUNSUPPORTED;
+  const Dims D = to_dims(*dims);
+  const bool dense = (mode == 0 && k == D.inter);
+  if (mode == 0 && (k < 1 || k > D.inter)) return MSB_EINVAL;
+  if (mode == 1 && !(tau == tau)) return MSB_EINVAL;
+  if (!x || !router_t || !records || !out || !workspace) return MSB_EINVAL;
+  if (!dense && (!sketch || !alpha)) return MSB_EINVAL;
+  if (D.rank > 0 && (!lr_a || !lr_b)) return MSB_EINVAL;
+  if (!aligned16(x) || !aligned16(router_t) || !aligned16(records) || !aligned16(out) ||
+      !aligned16(workspace) || (sketch && !aligned16(sketch)) || (alpha && !aligned16(alpha)))
+    return MSB_EINVAL;
+  if ((lr_a && !aligned16(lr_a)) || (lr_b && !aligned16(lr_b))) return MSB_EINVAL;
+  const size_t act_bytes = (size_t)batch * D.d * 2;
+  if (overlaps(x, act_bytes, out, act_bytes)) return MSB_EINVAL;
+  if (workspace_bytes < layout(D, batch).total) return MSB_EINVAL;
+  return MSB_OK;
+}
+
 int block_common(const void* x, int32_t batch, const void* router_t, const void* records,
                  const uint32_t* sketch, const float* alpha, int32_t k, int mode, float tau,
                  const void* lr_a, const void* lr_b, void* out, const msb_dims* dims,
@@ -225,6 +259,7 @@ int32_t msb_check(void* workspace, void* stream) {
   if (cudaMemcpyAsync(workspace, &zero, 4, cudaMemcpyHostToDevice, st) != cudaSuccess)
     return MSB_ECUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return MSB_ECUDA;
+  if (err & kErrInternal) return MSB_EINTERNAL;
   return (err & kErrTimeout) ? MSB_ETIMEOUT : MSB_ENONFINITE;
 }
 
@@ -237,6 +272,7 @@ const char* msb_strerror(int32_t status) {
     case MSB_ECUDA: return "CUDA launch or runtime error";
     case MSB_ETIMEOUT: return "a kernel's bounded wait ran out";
     case MSB_ENONFINITE: return "non-finite router logits (x or W_router has NaN/Inf)";
+    case MSB_EINTERNAL: return "a kernel's internal consistency check failed";
     default: return "unknown status";
   }
 }
@@ -262,6 +298,28 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
   m.top_e = top_e;
   return block_common(x, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out, &m,
                       workspace, workspace_bytes, trace, flags, stream);
+}
+
+int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, const void* router_t,
+                              const void* records, const uint32_t* sketch, const float* alpha,
+                              int32_t k, const void* lr_a, const void* lr_b, void* out_dev,
+                              void* out_host, const msb_dims* dims, void* workspace,
+                              size_t workspace_bytes, uint32_t flags, void* stream) {
+  // every check before the first copy, so that a rejected call enqueues nothing
+  int rc = block_check(x_dev, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out_dev,
+                       dims, workspace, workspace_bytes);
+  if (rc != MSB_OK) return rc;
+  if (!x_host || !out_host) return MSB_EINVAL;
+  const size_t bytes = (size_t)batch * dims->d * 2;
+  if (overlaps(x_host, bytes, out_host, bytes)) return MSB_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MSB_ECUDA;
+  rc = block_common(x_dev, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out_dev,
+                    dims, workspace, workspace_bytes, nullptr, flags, stream);
+  if (rc != MSB_OK) return rc;
+  if (cudaMemcpyAsync(out_host, out_dev, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MSB_ECUDA;
+  return MSB_OK;
 }
 
 int32_t moe_sparse_block_threshold(const void* x, int32_t batch, const void* router_t,
@@ -292,6 +350,28 @@ int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t f
   info[7] = 0;
   return MSB_OK;
 }
+
+#ifdef MSB_INSTRUMENTED
+// Instrumented build only (libmsb_instr.so): per-CTA %globaltimer marks of the
+// single-launch kernel's phases go to `marks` (device, [grid][16] u64; slot 15 = the
+// SM the CTA ran on), or nowhere when NULL.
+int32_t msb_debug_set_marks(void* marks) {
+  debug_ctl().marks = static_cast<unsigned long long*>(marks);
+  return MSB_OK;
+}
+
+// Instrumented build only: skip = 1 makes the single-launch kernel's first CTA withhold
+// its first record copy, skip = 2 makes the gather CTA of work item 0 withhold its first stage
+// (0: neither); wait_ns replaces the 2-second limit of the bounded waits (0: restore it).
+// A withheld copy is never issued, so the wait for it runs out: the call is flagged
+// (msb_check: MSB_ETIMEOUT) and its output is undefined.
+int32_t msb_debug_inject(uint32_t skip, uint64_t wait_ns) {
+  if (skip > 2u) return MSB_EINVAL;
+  debug_ctl().skip = skip;
+  debug_ctl().wait_ns = wait_ns;
+  return MSB_OK;
+}
+#endif
 
 int32_t msb_residual_rmsnorm(float* h, const void* y, void* x_next, int32_t batch, int32_t d,
                              float eps, void* stream) {

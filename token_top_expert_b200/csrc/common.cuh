@@ -35,6 +35,8 @@ __host__ __device__ inline int mask_words(int ipad) { return (ipad + 31) / 32; }
 // ---------------------------------------------------------------- device error word
 constexpr uint32_t kErrTimeout = 1u;
 constexpr uint32_t kErrNonFinite = 2u;  // router saw NaN/Inf logits (invalid input)
+constexpr uint32_t kErrInternal = 4u;   // a kernel's consistency check failed (a selection of
+                                        // the wrong size); the offending access was skipped
 constexpr uint32_t kSpinLimit = 1u << 22;            // polls before a wait gives up ...
 constexpr uint64_t kWaitLimitNs = 2000ull * 1000000;  // ... or 2 s of wall time, whichever first
 
@@ -74,20 +76,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete may sleep for up to
+// `hint_ns` before the call returns false (it wakes as soon as the phase completes), so
+// that a waiting warp takes no issue slots from the warps that work meanwhile.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
-// Wait for phase `parity` of the barrier, bounded by a poll count and by wall time.
-// On expiry sets the sticky error word and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+// Wait for phase `parity` of the barrier, bounded by a poll count and by wall time
+// (limit_ns).  On expiry sets the sticky error word and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1; i < kSpinLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) break;
+    if (mbar_try_wait_sleep(bar, parity, 2000u)) return true;
+    if ((i & 15u) == 0 && globaltimer_ns() - t0 > limit_ns) break;
   }
   atomicOr(err, kErrTimeout);
   return false;
@@ -101,6 +118,11 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
           smem_addr(dst)),
       "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
+}
+
+// Prefetch `bytes` (multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 // D += A*B with A 16x16 bf16 (row), B 16x8 bf16 (col), D 16x8 fp32.

@@ -1,49 +1,61 @@
 // Single-launch batch-1 sparse-MoE block (the decode hot path).
 //
-// One thread-block cluster per routed expert (or two smaller clusters per
-// expert).  Exchange inside a cluster goes through distributed shared memory and
-// hardware cluster barriers; across clusters only through FP32 atomics into a
-// small accumulator whose last contributor (per output slice) writes BF16.
+// One 16-CTA thread-block cluster per routed expert.  Every exchange inside a
+// cluster is a one-way push: the producer writes into the consumers' shared memory
+// with st.async / red.async, and each consumer waits on its own mbarrier for the
+// exact byte count it expects, so no exchange costs a cluster-wide barrier.
+// Across clusters only FP32 reduction-adds into a small accumulator meet; the last
+// contribution to an output slice writes it as BF16.
 //
-//  A  router: the cluster's CTAs each score E/CS experts (x . W_router rows
-//     staged by 1-D bulk copies), broadcast the logits over DSMEM; every CTA then
-//     runs softmax + top-K and cluster c takes the c-th ranked expert.
+//  A  router: each CTA computes E/16 logits x . W_router[e] (rows staged by a
+//     bulk copy before the grid dependency wait) and pushes them to every CTA of
+//     the cluster; every CTA ranks the E logits and cluster c takes the c-th expert.
 //  B  sketch scores: each CTA stages its 16-row tiles of the packed 2-bit sketch,
-//     scores them on the tensor cores (the packed codes are the bf16 A fragment),
-//     broadcasts alpha*|T.x| to the cluster; z = B_e x rows alongside.
-//  C  exact top-k: every CTA selects the same k channels (radix select, ties to the
-//     lower index); each CTA streams its share of the 6d-byte channel records
-//     through a shared-memory ring and accumulates SwiGLU(gate.x, up.x) * down.
-//  D  partial outputs are reduce-added into the owning CTA's slice over DSMEM;
-//     the owner adds A_e z, scales by the router weight and adds into the FP32
-//     accumulator; the last contribution to a slice converts it to BF16.
+//     scores them on the tensor cores (the packed codes are the bf16 A fragment)
+//     and pushes alpha*|T.x| and its largest key to every CTA of the cluster.
+//  C  exact top-k: every CTA selects the same k channels (histogram below the
+//     cluster's largest score, the k-th key's bin ranked directly; ties to the
+//     lower index) and issues bulk copies of its share of the channel records.
+//  D  records: as each 6d-byte record lands, its gate.x and up.x are reduced over
+//     the CTA, h = silu(gate.x) * up.x, and every thread adds h * down over its
+//     8-element groups of the output; z = B_e x (pushed like the scores) and
+//     A_e z on this CTA's output slice run while the records stream.
+//  E  combine: each CTA pushes its partial output, slice by slice, to the slice's
+//     owner; the owner sums the 16 partials, adds A_e z, scales by the router
+//     weight and reduction-adds into the FP32 accumulator; the last of the K
+//     contributions to a slice converts it to BF16 and re-zeroes it.
 //
-// The kernel is launched with programmatic stream serialisation: everything that
-// reads only weights (barrier set-up, router rows) runs before
-// griddepcontrol.wait, so it overlaps the previous launch's tail.
+// The kernel's code is kept small (rolled loops, rare paths out of line): on B200
+// a kernel whose executed code fits the SM's instruction cache stays warm from one
+// launch to the next, while one that does not pays instruction fetches every launch.
+//
+// The launch uses programmatic stream serialisation: barrier set-up and the router
+// rows' copy run before griddepcontrol.wait, overlapping the previous launch.
 //
 // "KAIST drops calibration from MoE decoding ...": "Top-k instead of a threshold"
 // (fixed read budget), "A reader built from weights alone" (ternary sketch filter
 // + low-rank compensation).  No TMA multicast and no peer memory is used.
-#include <cooperative_groups.h>
-
 #include "block_scan.cuh"
 #include "common.cuh"
 #include "fused.h"
-
-namespace cg = cooperative_groups;
+#include "launch.h"
 
 namespace msb {
 
-constexpr int kFT = 256;        // threads per CTA
-constexpr int kFW = kFT / 32;   // warps per CTA
-constexpr int kRingMax = 16;    // record slots
+constexpr int kFT = 256;       // threads per CTA
+constexpr int kFW = kFT / 32;  // warps per CTA
+constexpr int kRingMax = 16;   // record slots
 constexpr int kSmemMax = 227 * 1024;
-constexpr int kSmemPair = 110 * 1024;  // fallback pairing limit if the device cannot be queried
-constexpr int kAregs = 8;              // register quads for the slice's A_e rows (8 bf16 each)
-constexpr int kMyselMax = 256;         // channels one CTA reads at most
-constexpr int kSelBins = 2048;         // select histogram bins (256 per octave below the largest key)
-constexpr int kCandMax = 64;           // keys ranked directly in the k-th key's bin
+constexpr int kSmemPair = 113 * 1024;  // fallback pairing limit if the device cannot be queried
+constexpr int kSelBins = 2048;         // select histogram: 256 bins per octave below the largest key
+constexpr int kSelShift = 15;
+constexpr int kCandMax = 64;           // keys of the k-th key's bin ranked directly
+constexpr int kWordsMax = (MSB_MAX_INTER + 31) / 32;
+constexpr int kMyselMax = 512;         // channels one CTA reads at most
+constexpr int kMarks = 16;             // phase marks per CTA (instrumented builds)
+
+// mbarriers: fixed ones, then one per record slot
+enum { kBarRows = 0, kBarX, kBarLogits, kBarSketch, kBarLow, kBarScores, kBarZ, kBarY, kBarRing };
 
 struct FusedParams {
   const uint16_t* x;
@@ -56,123 +68,184 @@ struct FusedParams {
   uint16_t* out;
   uint32_t* err;
   uint32_t* slice_cnt;  // [cs] arrival counters, one per output slice
-  float* y_acc;
+  float* y_acc;         // [d] FP32 accumulator, zero between calls
+#ifdef MSB_INSTRUMENTED
+  unsigned long long* marks;  // [grid][kMarks] phase timestamps, or null
+  uint32_t skip;              // 1: CTA 0 never issues its first record copy
+  uint64_t wait_ns;           // bounded-wait limit
+#endif
   TraceDev tr;
   Dims D;
-  int k, dense, cs, cpe;
-  int epad;    // router logits padded to a multiple of 64 (with -inf)
+  int k, dense, cs;
   int rpc;     // router rows per CTA
   int tpc;     // sketch row tiles per CTA
-  int zpc;     // z rows per CTA (max)
   int slice;   // output elements owned per CTA (d / cs)
   int ring;    // record slots
-  int rs;      // ring slot stride in bf16 elements: 3d + 8 (16 bytes of stagger between
-               // slots, so rows of consecutive slots fall in different banks)
-  int group;   // channels per reduction group (<= ring)
-  // shared-memory carve-up (byte offsets)
-  int o_z, o_ylr, o_misc, o_big;  // shared-memory offsets
-  int o_logits, o_xperm, o_keys, o_alpha, o_part, o_hist, o_xbig;  // offsets in big
-  int o_aslice_off;  // A_e rows: byte offset inside big, past every other use of big
-  int aslice_regs;   // 1: A_e rows of the slice are held in registers instead
+  int rs;      // ring slot stride (elements): 3d + 8, so that the rows of consecutive slots
+               // fall 16 bytes apart in the shared-memory banks (conflict-free ldmatrix)
+  int rrs;     // router row stride in shared memory (elements): d + 8, for the same reason
+  int epad;    // logits padded to a multiple of 64 (with -inf)
+  // shared-memory carve-up (byte offsets from the dynamic base)
+  int o_misc, o_lr, o_rbuf, o_mysel, o_big;
+  int o_x, o_xperm, o_logits, o_keys, o_hist, o_part;  // inside big (phases A-C)
+  int o_alpha, o_brows;                                  // inside big (phase B)
   int smem;
+  uint32_t x1_bytes, sc_bytes, z_bytes, y_bytes;  // bytes each CTA expects per exchange
 };
 
 struct Misc {
-  uint64_t bar[2 + kRingMax];
+  uint64_t bar[kBarRing + kRingMax];
   int ids[MSB_MAX_TOP_E];
   float lv[MSB_MAX_TOP_E];  // routed logits in rank order
+  float wk[MSB_MAX_TOP_E];  // combine weights of the routed experts, rank order
+  uint32_t tie, cmax, kb, rem, cnt, ccount, kth, need;
   uint32_t info[2];
-  float h[kRingMax];
-  float red[kFW][2 * kRingMax];  // per-warp (gate . x, up . x) of a group's channels
-  // channel select scratch
-  uint32_t wt[kFW];            // per-warp totals of the bin scan
-  uint32_t wgt[kFW], weq[kFW]; // per warp range: keys above the k-th, keys equal to it
-  uint32_t kb, rem, cnt, ccount, kth, need;
-  uint32_t ck[kCandMax];       // keys of the bin holding the k-th key, and their indices
-  uint32_t ci[kCandMax];
-  uint32_t cmax[16];           // largest score key of each CTA of the cluster
-  uint32_t lmax;               // largest score key of this CTA
-  uint32_t tie;                // router: a rank slot was claimed twice
-  uint16_t mysel[kMyselMax];  // this CTA's share of the selected channels
+  uint32_t wt[kFW];
+  float red8[kFW][8];    // per-warp sums of up to 8 dot products (logits; gate/up of a batch)
+  float h[8];            // h of a batch's records
+  uint32_t ck[kCandMax], ci[kCandMax];
+  uint32_t csel[kWordsMax];  // selected keys of the k-th key's bin
+  uint32_t selw[kWordsMax];  // selection bitmap over the channels
+  uint32_t pref[kWordsMax];  // exclusive prefix of popc(selw)
+  float z[MSB_MAX_RANK];     // B_e x
   int last;
 };
 
+// the kernel's dynamic shared memory (carved up by the offsets in FusedParams)
+extern __shared__ __align__(128) uint8_t g_sm[];
+// this CTA's share of the selected channels (positions [c0, c1) of the ascending list)
+#define MYSEL(P) reinterpret_cast<uint16_t*>(g_sm + (P).o_mysel)
+
+// ---------------------------------------------------------------- cluster PTX
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// address of the same shared-memory location in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t mapa(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+// remote store of one word, completion counted (4 bytes) on the remote mbarrier
+__device__ __forceinline__ void st_async(uint32_t ra, uint32_t v, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(ra),
+               "r"(v), "r"(rbar)
+               : "memory");
+}
+__device__ __forceinline__ void st_async4(uint32_t ra, float a, float b, float c, float d, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(ra),
+      "f"(a), "f"(b), "f"(c), "f"(d), "r"(rbar)
+      : "memory");
+}
+// remote max of one word, completion counted (4 bytes) on the remote mbarrier
+__device__ __forceinline__ void red_async_max(uint32_t ra, uint32_t v, uint32_t rbar) {
+  asm volatile(
+      "red.async.relaxed.cluster.shared::cluster.mbarrier::complete_tx::bytes.max.u32 [%0], %1, [%2];" ::"r"(
+          ra),
+      "r"(v), "r"(rbar)
+      : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// The kernel runs once per CTA per launch, so its code is fetched cold every time
-// (on B200, cold straight-line code costs ~0.4 us per KB per SM).  It is written
-// for a small footprint: loops with short bodies, shared helpers kept out of line,
-// fast intrinsics for the few transcendental steps.
+#ifdef MSB_INSTRUMENTED
+#define MARK(i)                                                                \
+  do {                                                                         \
+    if (P.marks && threadIdx.x == 0) P.marks[blockIdx.x * kMarks + (i)] = globaltimer_ns(); \
+  } while (0)
+#define WAIT_LIMIT (P.wait_ns)
+#else
+#define MARK(i) \
+  do {          \
+  } while (0)
+#define WAIT_LIMIT kWaitLimitNs
+#endif
 
-// Bounded wait on an mbarrier phase (shared by every wait site).
-__device__ __noinline__ bool wait_phase(uint64_t* bar, uint32_t parity, uint32_t* err) {
-  return mbar_wait(bar, parity, err);
+// Bounded wait: the common case (phase already complete) inline, the spin out of line.
+__device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, uint32_t* err, uint64_t limit) {
+  return mbar_wait(bar, parity, err, limit);
+}
+#define wait_phase(bar, parity, err) \
+  (mbar_try_wait((bar), (parity)) || wait_slow((bar), (parity), (err), WAIT_LIMIT))
+
+// Router top-K, exact pass: rank = #{e' : l_e' > l_e} + #{e' < e : l_e' == l_e} (ties
+// to the lower index), one thread per logit.  Rare (taken after a tie among the top K).
+// Ends with a barrier.
+__device__ __noinline__ void router_rank_exact(const float* logits, int E, int K, Misc& M) {
+  if (threadIdx.x < K) M.ids[threadIdx.x] = -1;
+  __syncthreads();
+#pragma unroll 1
+  for (int ee = threadIdx.x; ee < E; ee += kFT) {
+    const float v = logits[ee];
+    int r = 0;
+#pragma unroll 1
+    for (int j = 0; j < E; ++j) {
+      const float u = logits[j];
+      r += (u > v) || (u == v && j < ee);
+    }
+    if (r < K) {
+      M.ids[r] = ee;
+      M.lv[r] = v;
+    }
+  }
+  __syncthreads();
 }
 
 // Router top-K over the E logits in shared memory (padded with -inf to Epad, a
 // multiple of 64), by rank counting, P = 256/E threads per logit (at most 4) on
-// 16-value vector steps.  Fast pass: rank = #{e' : l_e' > l_e}; the owner of rank
-// j < K claims slot j.  Without ties among the top K every claim lands in its own
-// slot and these ranks are exact; two logits with the same value have the same
-// count, so a tie shows as a second claim on one slot, and then the exact pass
-// ranks by #{e' : l_e' > l_e} + #{e' < e : l_e' == l_e} (ties to the lower index).
-// M.ids must be -1 and M.tie 0 on entry.  Ends with a barrier.
+// 16-value vector steps: rank = #{e' : l_e' > l_e}; the owner of rank j < K claims
+// slot j.  Without ties among the top K every claim lands in its own slot and these
+// ranks are exact; two logits with the same value have the same count, so a tie shows
+// as a second claim on one slot, and then the exact pass runs.  M.ids must be -1 and
+// M.tie 0 on entry.  Ends with a barrier.
 __device__ __noinline__ void router_rank(const float* logits, int E, int Epad, int K, Misc& M,
                                          uint32_t* err) {
   const int tid = threadIdx.x;
   const int lgP = E <= 64 ? 2 : (E <= 128 ? 1 : 0);
   const int span = Epad >> lgP;
 #pragma unroll 1
-  for (int pass = 0; pass < 2; ++pass) {
-#pragma unroll 1
-    for (int base = 0; base < (E << lgP); base += kFT) {
-      const int item = base + tid, ee = item >> lgP, h = item & ((1 << lgP) - 1);
-      float gt = 0.f;
-      float v = 0.f;
-      if (ee < E) {
-        v = logits[ee];
-        if (pass == 0) {
-          if (!isfinite(v)) atomicOr(err, kErrNonFinite);
-          const float4* lp = reinterpret_cast<const float4*>(logits + h * span);
+  for (int base = 0; base < (E << lgP); base += kFT) {
+    const int item = base + tid, ee = item >> lgP, h = item & ((1 << lgP) - 1);
+    float gt = 0.f;
+    float v = 0.f;
+    if (ee < E) {
+      v = logits[ee];
+      if (!isfinite(v)) atomicOr(err, kErrNonFinite);
+      const float4* lp = reinterpret_cast<const float4*>(logits + h * span);
 #pragma unroll 4
-          for (int c = 0; c < span / 4; ++c) {
-            const float4 u = lp[c];
-            gt += (u.x > v ? 1.f : 0.f) + (u.y > v ? 1.f : 0.f);
-            gt += (u.z > v ? 1.f : 0.f) + (u.w > v ? 1.f : 0.f);
-          }
-        } else {
-          int r = 0;
-#pragma unroll 1
-          for (int j = h * span; j < (h + 1) * span; ++j) {
-            const float u = logits[j];
-            r += (u > v) || (u == v && j < ee);
-          }
-          gt = (float)r;
-        }
-      }
-      if (lgP >= 1) gt += __shfl_xor_sync(0xffffffffu, gt, 1);
-      if (lgP >= 2) gt += __shfl_xor_sync(0xffffffffu, gt, 2);
-      const int rank = (int)gt;
-      if (ee < E && h == 0 && rank < K) {
-        if (atomicCAS(&M.ids[rank], -1, ee) != -1) M.tie = 1u;
-        M.lv[rank] = v;
+      for (int c = 0; c < span / 4; ++c) {
+        const float4 u = lp[c];
+        gt += (u.x > v ? 1.f : 0.f) + (u.y > v ? 1.f : 0.f);
+        gt += (u.z > v ? 1.f : 0.f) + (u.w > v ? 1.f : 0.f);
       }
     }
-    __syncthreads();
-    if (pass == 1 || M.tie == 0u) break;
-    if (tid < K) M.ids[tid] = -1;
-    __syncthreads();
+    if (lgP >= 1) gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+    if (lgP >= 2) gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+    const int rank = (int)gt;
+    if (ee < E && h == 0 && rank < K) {
+      if (atomicCAS(&M.ids[rank], -1, ee) != -1) M.tie = 1u;
+      M.lv[rank] = v;
+    }
   }
+  __syncthreads();
+  if (M.tie) router_rank_exact(logits, E, K, M);
 }
 
-// Combine weight of the routed expert of rank j (every lane of the warp calls it,
-// after router_rank): softmax over the K routed logits (renorm) or over all E
-// logits.  lv[0] is the largest logit.
-__device__ __forceinline__ float router_weight(const float* logits, int E, int K, int renorm,
-                                               const Misc& M, int j) {
+// Warp 0, after router_rank: the combine weights of the K routed experts into M.wk
+// (rank order): softmax over the K routed logits (renorm) or over all E logits.
+// lv[0] is the largest logit.
+__device__ __noinline__ void router_weights(const float* logits, int E, int K, int renorm, Misc& M) {
   const int lane = threadIdx.x & 31;
   const float mx = M.lv[0];
   const float pl = lane < K ? __expf(M.lv[lane] - mx) : 0.f;
@@ -184,149 +257,27 @@ __device__ __forceinline__ float router_weight(const float* logits, int E, int K
     for (int i = lane; i < E; i += 32) denom += __expf(logits[i] - mx);
   }
   denom = warp_sum(denom);
-  return __fdividef(__shfl_sync(0xffffffffu, pl, j), denom);
+  if (lane < K) M.wk[lane] = __fdividef(pl, denom);
 }
 
-// Exact top-k of the n channel scores (keys = float bits, so integer order is value
-// order), ties to the lower index; writes this CTA's share, positions [c0, c1) of
-// the ascending selected list, to M.mysel and (when trace is set) the whole list to
-// trace.  Keys are binned by (maxkey - key) >> 15 (256 bins per octave below the
-// largest key, bin 0 the largest, the last bin catching the rest): one counting
-// pass and one scan find the bin of the k-th key, whose keys are then ranked
-// directly; a bin with more than kCandMax keys falls back to a radix descent.
-// hist: kSelBins zeroed words.  M.ccount must be 0 on entry.
-__device__ __noinline__ void select_share(const uint32_t* keys, int n, int k, uint32_t maxkey,
-                                          uint32_t* hist, Misc& M, int c0, int c1, uint16_t* trace) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-#pragma unroll 4
-  for (int j = tid; j < n; j += kFT) atomicAdd(&hist[min((uint32_t)(kSelBins - 1), (maxkey - keys[j]) >> 15)], 1u);
-  __syncthreads();
-  // thread t owns bins [8t, 8t + 8)
-  uint32_t c[8];
-  {
-    const uint4 a = reinterpret_cast<const uint4*>(hist)[2 * tid];
-    const uint4 b = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
-    c[0] = a.x; c[1] = a.y; c[2] = a.z; c[3] = a.w; c[4] = b.x; c[5] = b.y; c[6] = b.z; c[7] = b.w;
-  }
-  uint32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) local += c[i];
-  uint32_t incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) M.wt[warp] = incl;
-  __syncthreads();
-  uint32_t above = incl - local;
-#pragma unroll
-  for (int w = 0; w < kFW; ++w) above += w < warp ? M.wt[w] : 0u;
-  const uint32_t kk = (uint32_t)k;
-  if (above < kk && kk <= above + local) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (above < kk && kk <= above + c[i]) { M.kb = 8 * tid + i; M.rem = kk - above; M.cnt = c[i]; }
-      above += c[i];
+// Trace of the routing (one CTA): expert ids, weights, and the channels read per expert.
+__device__ __noinline__ void trace_routing(const TraceDev& tr, const Misc& M, int E, int K, int k) {
+  const int tid = threadIdx.x;
+  if (tid < K && tr.expert_ids) tr.expert_ids[tid] = M.ids[tid] < 0 ? tid : M.ids[tid];
+  if (tid < K && tr.expert_w) tr.expert_w[tid] = M.wk[tid];
+  if (tr.union_count)
+#pragma unroll 1
+    for (int i = tid; i < E; i += kFT) {
+      int c = 0;
+#pragma unroll 1
+      for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? k : c;  // (-1 never matches)
+      tr.union_count[i] = c;
     }
-  }
-  __syncthreads();
-  const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
-  // scatter layout: warp w owns the indices [w * span, (w + 1) * span)
-  const int span = 32 * ((n + kFT - 1) / kFT);
-  const int wb = warp * span, we = min(n, wb + span);
-  const uint32_t lt = (1u << lane) - 1u;
-  uint32_t kth, need;
-  if (cnt > (uint32_t)kCandMax) {  // heavy ties: radix descent, then count per warp range
-    radix_kth_smem<kFT>(keys, n, k, hist, M.info, &kth, &need);
-    uint32_t ngt = 0, neq = 0;
-#pragma unroll 4
-    for (int j0 = wb; j0 < we; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t key = j < we ? keys[j] : 0u;
-      ngt += __popc(__ballot_sync(0xffffffffu, j < we && key > kth));
-      neq += __popc(__ballot_sync(0xffffffffu, j < we && key == kth));
-    }
-    if (lane == 0) { M.wgt[warp] = ngt; M.weq[warp] = neq; }
-    __syncthreads();
-  } else {
-    // gather the bin's keys; keys of higher bins (larger keys) are counted per warp range
-    uint32_t ngt = 0;
-#pragma unroll 4
-    for (int j0 = wb; j0 < we; j0 += 32) {
-      const int j = j0 + lane;
-      const uint32_t key = j < we ? keys[j] : 0u;
-      const uint32_t bin = min((uint32_t)(kSelBins - 1), (maxkey - key) >> 15);
-      ngt += __popc(__ballot_sync(0xffffffffu, j < we && bin < kb));
-      const bool m = j < we && bin == kb;
-      const uint32_t mb = __ballot_sync(0xffffffffu, m);
-      if (mb) {
-        const int leader = __ffs(mb) - 1;
-        uint32_t slot0 = 0;
-        if (lane == leader) slot0 = atomicAdd(&M.ccount, (uint32_t)__popc(mb));
-        slot0 = __shfl_sync(0xffffffffu, slot0, leader);
-        if (m) {
-          const uint32_t slot = slot0 + __popc(mb & lt);
-          M.ck[slot] = key;
-          M.ci[slot] = (uint32_t)j;
-        }
-      }
-    }
-    if (lane == 0) { M.wgt[warp] = ngt; M.weq[warp] = 0u; }
-    __syncthreads();
-    // rank inside the bin by (key desc, index asc); the k-th key sits at position rem - 1.
-    // A candidate whose equal keys occupy positions [gt, gt + eq) is above the k-th key
-    // if rem - 1 >= gt + eq, equal to it if gt <= rem - 1 < gt + eq.
-    if (tid < (int)cnt) {
-      const uint32_t mk = M.ck[tid], mi = M.ci[tid];
-      uint32_t gt = 0, eq = 0;
-#pragma unroll 4
-      for (int i = 0; i < (int)cnt; ++i) {
-        const uint32_t ok_ = M.ck[i];
-        gt += ok_ > mk;
-        eq += ok_ == mk;
-      }
-      const uint32_t pk = rem - 1u, w = mi / (uint32_t)span;
-      if (pk >= gt + eq) {
-        atomicAdd(&M.wgt[w], 1u);
-      } else if (pk >= gt) {
-        atomicAdd(&M.weq[w], 1u);
-        M.kth = mk;
-        M.need = rem - gt;
-      }
-    }
-    __syncthreads();
-    kth = M.kth;
-    need = M.need;
-  }
-  uint32_t gtb = 0, eqb = 0;
-#pragma unroll
-  for (int w = 0; w < kFW; ++w) {
-    gtb += w < warp ? M.wgt[w] : 0u;
-    eqb += w < warp ? M.weq[w] : 0u;
-  }
-  const uint32_t ltm = (1u << lane) - 1u;
-#pragma unroll 4
-  for (int j0 = wb; j0 < we; j0 += 32) {
-    const int j = j0 + lane;
-    const uint32_t key = j < we ? keys[j] : 0u;
-    const uint32_t bg = __ballot_sync(0xffffffffu, j < we && key > kth);
-    const uint32_t be = __ballot_sync(0xffffffffu, j < we && key == kth);
-    const uint32_t eqr = eqb + __popc(be & ltm);
-    if (((bg >> lane) & 1u) || (((be >> lane) & 1u) && eqr < need)) {
-      const int pos = (int)(gtb + __popc(bg & ltm) + min(eqr, need));
-      if (pos >= c0 && pos < c1) M.mysel[pos - c0] = (uint16_t)j;
-      if (trace) trace[pos] = (uint16_t)j;
-    }
-    gtb += __popc(bg);
-    eqb += __popc(be);
-  }
-  __syncthreads();
 }
 
 // Sketch scores of this CTA's nt row tiles: warp w takes chunks [kc0, kc1) of every
 // tile; the packed 2-bit codes are the bf16 A fragments (+-2 or 0), x is B.
-// Partial sums go to part[warp][tile*16 + row].
+// Partial sums go to part_w[tile*16 + row].
 __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm, int nt, int KC,
                                          float* part_w) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -362,451 +313,799 @@ __device__ __noinline__ void score_tiles(const uint2* codes, const uint4* xperm,
   }
 }
 
-template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
-__global__ void __launch_bounds__(kFT, 1) fused_block_kernel(const __grid_constant__ FusedParams P) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CS = P.cs;
-  const int q = (int)cluster.block_rank();
-  const int cid = blockIdx.x / CS;
-  const int rc = cid / P.cpe;     // which routed expert (rank order)
-  const int half = cid % P.cpe;   // which cluster of that expert
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const Dims D = P.D;
-  const int d = D.d, E = D.experts, I = D.inter, ipad = D.ipad, r = D.rank, K = D.top_e;
-  const int KC = d / kColChunk;
+__device__ __forceinline__ uint32_t sel_bin(uint32_t maxkey, uint32_t key) {
+  return min((uint32_t)(kSelBins - 1), (maxkey - key) >> kSelShift);
+}
 
-  float* zs = reinterpret_cast<float*>(sm + P.o_z);
-  float* ylr = reinterpret_cast<float*>(sm + P.o_ylr);     // A_e z on this CTA's slice
-  Misc& M = *reinterpret_cast<Misc*>(sm + P.o_misc);
-  uint8_t* big = sm + P.o_big;
-  // `big` is reused phase by phase (offsets from the plan):
-  //   A: router rows at 0, logits (remote-written) after them
-  //   B: sketch tiles at 0, B_e rows, alpha, partial sums, x fragments, scores (remote-written)
-  //   C: the record ring at 0          D: the partial output at 0
-  //   A_e rows sit past all of these (loaded in B, read after the ring drains)
-  uint16_t* xs = reinterpret_cast<uint16_t*>(big + P.o_xbig);  // phases A-B (C reads x from L1/L2)
-  float* logits = reinterpret_cast<float*>(big + P.o_logits);
-  uint32_t* xperm = reinterpret_cast<uint32_t*>(big + P.o_xperm);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(big + P.o_keys);  // channel scores (float bits)
-  float* alpha_s = reinterpret_cast<float*>(big + P.o_alpha);
-  float* part = reinterpret_cast<float*>(big + P.o_part);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(big + P.o_hist);  // phase C select
-  float* ybuf = reinterpret_cast<float*>(big);             // phase D: partial output (over the ring)
-
-  // Every CTA of the cluster must be running before any DSMEM access targets it:
-  // arrive now, wait just before the first remote access.
-  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
-
-  // ------------------------------------------------------------------ prologue (weights only)
-  const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
-  const uint32_t rbytes = (uint32_t)(e_hi - e_lo) * 2u * d;
-  if (tid == 0) {
+// Heavy ties in the k-th key's bin (more than kCandMax keys): exact radix descent
+// over all keys, then warp 0 walks the words in index order and takes the equal
+// keys lowest index first.  Writes M.selw.  Ends with a barrier.
+__device__ __noinline__ void select_fallback(const uint32_t* keys, int n, int k, uint32_t* hist,
+                                             Misc& M) {
+  uint32_t kth, need;
+  radix_kth_smem<kFT>(keys, n, k, hist, M.info, &kth, &need);
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t taken = 0;
 #pragma unroll 1
-    for (int i = 0; i < 2 + P.ring; ++i) mbar_init(&M.bar[i], 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(&M.bar[0], rbytes);
-    if (rbytes) bulk_g2s(big, P.router_t + (size_t)e_lo * d, rbytes, &M.bar[0]);
-  }
-#pragma unroll 1
-  for (int i = tid; i < P.slice; i += kFT) ylr[i] = 0.f;
-  for (int i = E + tid; i < P.epad; i += kFT) logits[i] = -INFINITY;
-  if (tid < K) M.ids[tid] = -1;
-  if (tid == 0) { M.lmax = 0u; M.ccount = 0u; M.tie = 0u; }
-  // x and the workspace may be written by the previous launch: wait for it here.
-  pdl_wait();
-#pragma unroll 1
-  for (int i = tid; i < d / 8; i += kFT)
-    reinterpret_cast<uint4*>(xs)[i] = __ldg(reinterpret_cast<const uint4*>(P.x) + i);
-  __syncthreads();
-
-  // ------------------------------------------------------------------ phase A: router
-  bool ok = wait_phase(&M.bar[0], 0, P.err);
-  ok = __syncthreads_and(ok);
-  asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-  if (ok) {
-    const uint16_t* rows = reinterpret_cast<const uint16_t*>(big);
-#pragma unroll 1
-    for (int row = warp; row < e_hi - e_lo; row += kFW) {
-      const uint4* wr = reinterpret_cast<const uint4*>(rows + (size_t)row * d);
-      const uint4* xr = reinterpret_cast<const uint4*>(xs);
-      float acc = 0.f;
-#pragma unroll 2
-      for (int i = lane; i < d / 8; i += 32) acc = dot8(wr[i], xr[i], acc);
-      acc = warp_sum(acc);
-      if (lane < CS) cluster.map_shared_rank(logits, lane)[e_lo + row] = acc;
-    }
-  }
-  cluster.sync();
-  router_rank(logits, E, P.epad, K, M, P.err);
-  int e = M.ids[rc];
-  if (e < 0) {  // a rank left empty (non-finite logits): keep a valid index, the call is flagged
-    e = rc;
-    if (tid == 0) atomicOr(P.err, kErrNonFinite);
-  }
-  const float we = router_weight(logits, E, K, D.renorm, M, rc);
-  if (blockIdx.x == 0) {
-    if (warp == 0) {  // (the weight of a non-renormalised softmax is a warp-wide sum)
-      const float wl = router_weight(logits, E, K, D.renorm, M, lane < K ? lane : 0);
-
-      if (lane < K && P.tr.expert_ids) P.tr.expert_ids[lane] = M.ids[lane] < 0 ? lane : M.ids[lane];
-      if (lane < K && P.tr.expert_w) P.tr.expert_w[lane] = wl;
-    }
-    if (P.tr.union_count)
-#pragma unroll 1
-      for (int i = tid; i < E; i += kFT) {
-        int c = 0;
-        for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? P.k : c;  // (-1 never matches)
-        P.tr.union_count[i] = c;
-      }
-  }
-
-  // ------------------------------------------------------------------ phase B: scores, z
-  const int ntile_all = ipad / kRowTile;
-  const int lt0 = min(ntile_all, q * P.tpc), lt1 = min(ntile_all, lt0 + P.tpc);
-  const int nt = lt1 - lt0;
-  const uint32_t code_bytes = P.dense ? 0u : (uint32_t)nt * KC * kChunkWords * 4u;
-  const int nz = r > q ? (r - q + CS - 1) / CS : 0;  // z rows q, q+CS, ... below r
-  const bool lr_out = (half == 0 && r > 0);
-  uint16_t* brows = reinterpret_cast<uint16_t*>(big + code_bytes);
-  uint16_t* aslice = reinterpret_cast<uint16_t*>(big + P.o_aslice_off);
-  const bool lr_smem = lr_out && !P.aslice_regs;
-  if (tid == 0 && ok) {
-    uint32_t bytes = code_bytes + (P.dense ? 0u : (uint32_t)nt * kRowTile * 4u) + (uint32_t)nz * 2u * d;
-    if (lr_smem) bytes += (uint32_t)P.slice * r * 2u;
-    fence_proxy_async();
-    mbar_arrive_expect_tx(&M.bar[1], bytes);
-    if (code_bytes) {
-      bulk_g2s(big, P.sketch + ((size_t)e * ntile_all + lt0) * KC * kChunkWords, code_bytes, &M.bar[1]);
-      bulk_g2s(alpha_s, P.alpha + (size_t)e * ipad + (size_t)lt0 * kRowTile, nt * kRowTile * 4u,
-               &M.bar[1]);
-    }
-#pragma unroll 1
-    for (int i = 0; i < nz; ++i)
-      bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[1]);
-    if (lr_smem)
-      bulk_g2s(aslice, P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, (uint32_t)P.slice * r * 2u,
-               &M.bar[1]);
-  }
-  // A_e rows of this CTA's output slice into registers (8 bf16 per quad), when they fit
-  uint4 areg[kAregs];
-  const int nachunk = (lr_out && P.aslice_regs) ? P.slice * r / 8 : 0;
-#pragma unroll
-  for (int u = 0; u < kAregs; ++u) {
-    const int j = tid + u * kFT;
-    areg[u] = make_uint4(0u, 0u, 0u, 0u);
-    if (ok && j < nachunk)
-      areg[u] = __ldg(reinterpret_cast<const uint4*>(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r) + j);
-  }
-  // phase-B scratch in big (past the tiles and B_e rows, which are still landing)
-#pragma unroll 1
-  for (int i = tid; i < kFW * P.tpc * kRowTile; i += kFT) part[i] = 0.f;
-  if (!P.dense)
-#pragma unroll 1
-    for (int i = tid; i < kSelBins / 4; i += kFT) reinterpret_cast<uint4*>(hist)[i] = make_uint4(0u, 0u, 0u, 0u);
-  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
-#pragma unroll 1
-  for (int i = tid; i < d / 2; i += kFT) {
-    const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
-    xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
-  }
-  ok = ok && wait_phase(&M.bar[1], 0, P.err);
-  ok = __syncthreads_and(ok);
-  if (ok && !P.dense && nt > 0)
-    score_tiles(reinterpret_cast<const uint2*>(big), reinterpret_cast<const uint4*>(xperm), nt, KC,
-                part + warp * P.tpc * kRowTile);
-  // z rows: z[rho] = B_e[rho] . x, broadcast to the cluster
-  if (ok && r > 0) {
-#pragma unroll 1
-    for (int i = warp; i < nz; i += kFW) {
-      const uint4* br = reinterpret_cast<const uint4*>(brows + (size_t)i * d);
-      const uint4* xr = reinterpret_cast<const uint4*>(xs);
-      float acc = 0.f;
-#pragma unroll 2
-      for (int j = lane; j < d / 8; j += 32) acc = dot8(br[j], xr[j], acc);
-      acc = warp_sum(acc);
-      if (lane < CS) cluster.map_shared_rank(zs, lane)[q + i * CS] = acc;
-    }
-  }
-  __syncthreads();
-  const int nrows = (ok && !P.dense) ? nt * kRowTile : 0;
-  // score = alpha * |sum of the 8 warps' partials| / 2 (into part's first row) ...
-  uint32_t lmax = 0;
-#pragma unroll 1
-  for (int lr = tid; lr < nrows; lr += kFT) {
-    float sc = 0.f;
-#pragma unroll
-    for (int w = 1; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + lr];
-    sc = alpha_s[lr] * fabsf(sc + part[lr]) * 0.5f;
-    part[lr] = sc;
-    lmax = max(lmax, __float_as_uint(sc));
-    if (half == 0 && P.tr.scores) P.tr.scores[(size_t)rc * ipad + lt0 * kRowTile + lr] = sc;
-  }
-  lmax = __reduce_max_sync(0xffffffffu, lmax);
-  if (lane == 0 && lmax) atomicMax(&M.lmax, lmax);
-  __syncthreads();
-  // ... then broadcast to every CTA of the cluster: item i -> (row i / CS, CTA i % CS),
-  // with this CTA's largest key
-  if (tid < CS) cluster.map_shared_rank(M.cmax, tid)[q] = M.lmax;
-  const int lg = CS == 16 ? 4 : 3;
-#pragma unroll 1
-  for (int i = tid; i < nrows * CS; i += kFT)
-    cluster.map_shared_rank(keys, i & (CS - 1))[lt0 * kRowTile + (i >> lg)] =
-        __float_as_uint(part[i >> lg]);
-  cluster.sync();
-  pdl_trigger();  // the next launch may start its weight-only prologue
-
-  // ------------------------------------------------------------------ phase C: top-k, records
-  // this CTA's share of the k channels: positions [c0, c1) of the ascending list
-  const int NQ = CS * P.cpe, gq = half * CS + q;
-  const int c0 = gq * P.k / NQ, c1 = (gq + 1) * P.k / NQ;
-  const int nmine = c1 - c0;
-  if (!P.dense) {
-    uint32_t maxkey = 0;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) maxkey = i < CS ? max(maxkey, M.cmax[i]) : maxkey;
-    uint16_t* trace = (half == 0 && q == 0 && P.tr.sel) ? P.tr.sel + (size_t)rc * P.k : nullptr;
-    select_share(keys, I, P.k, maxkey, hist, M, c0, c1, trace);
-    if (half == 0 && q == 0 && tid == 0 && P.tr.sel_count) P.tr.sel_count[rc] = P.k;
-  } else {
-#pragma unroll 1
-    for (int i = tid; i < nmine; i += kFT) M.mysel[i] = (uint16_t)(c0 + i);
-    __syncthreads();
-  }
-  const uint32_t rec_bytes = 6u * d;
-  uint16_t* ring = reinterpret_cast<uint16_t*>(big);
-  if (warp == 0 && ok) {  // lane i issues the copy into slot i
-    fence_proxy_async();
-    const int first = min(P.ring, nmine);
-    if (lane < first) {
-      const int ch = M.mysel[lane];
-      mbar_arrive_expect_tx(&M.bar[2 + lane], rec_bytes);
-      bulk_g2s(ring + (size_t)lane * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
-               &M.bar[2 + lane]);
-    }
-  }
-  // A_e z on this CTA's output slice, while the records are in flight
-  if (ok && lr_out) {
-    if (P.aslice_regs) {
-      const int cpr = r / 8;  // register quads per A_e row
-#pragma unroll
-      for (int u = 0; u < kAregs; ++u) {
-        const int j = tid + u * kFT;
-        if (j < nachunk) {
-          const int row = j / cpr, rho0 = (j - row * cpr) * 8;
-          const float* zz = zs + rho0;
-          float acc = bf16_lo(areg[u].x) * zz[0];
-          acc = fmaf(bf16_hi(areg[u].x), zz[1], acc);
-          acc = fmaf(bf16_lo(areg[u].y), zz[2], acc);
-          acc = fmaf(bf16_hi(areg[u].y), zz[3], acc);
-          acc = fmaf(bf16_lo(areg[u].z), zz[4], acc);
-          acc = fmaf(bf16_hi(areg[u].z), zz[5], acc);
-          acc = fmaf(bf16_lo(areg[u].w), zz[6], acc);
-          acc = fmaf(bf16_hi(areg[u].w), zz[7], acc);
-          atomicAdd(&ylr[row], acc);
+    for (int c = 0; c < (n + 31) / 32; ++c) {
+      const int j = 32 * c + lane;
+      const uint32_t key = j < n ? keys[j] : 0u;
+      const uint32_t gtb = __ballot_sync(0xffffffffu, j < n && key > kth);
+      const uint32_t eqb = __ballot_sync(0xffffffffu, j < n && key == kth);
+      uint32_t take = 0;
+      if (taken < need) {
+        const uint32_t left = need - taken;
+        if ((uint32_t)__popc(eqb) <= left) {
+          take = eqb;
+        } else {  // the `left` lowest set bits of eqb
+          const uint32_t top = __fns(eqb, 0, (int)left);
+          take = eqb & (top >= 31 ? 0xffffffffu : ((2u << top) - 1u));
         }
+      }
+      taken += (uint32_t)__popc(take);
+      if (lane == 0) M.selw[c] = gtb | take;
+    }
+  }
+  __syncthreads();
+}
+
+// Exact top-k of the n channel keys (float bits of non-negative scores, so integer
+// order is value order), ties to the lower index, as a bitmap M.selw over the
+// channels.  Keys are binned by (maxkey - key) >> 15 (256 bins per octave below the
+// largest key, bin 0 the largest, the last bin catching the rest): one counting
+// pass and one scan find the bin of the k-th key, whose keys are then ranked
+// directly.  hist (kSelBins words), M.csel and M.ccount must be zero on entry.
+__device__ __noinline__ void select_topk(const uint32_t* keys, int n, int k, uint32_t maxkey,
+                                         uint32_t* hist, Misc& M) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+#pragma unroll 1
+  for (int j = tid; j < n; j += kFT) atomicAdd(&hist[sel_bin(maxkey, keys[j])], 1u);
+  __syncthreads();
+  // thread t owns bins [8t, 8t + 8): find the bin holding the k-th largest key
+  const uint4 h0 = reinterpret_cast<const uint4*>(hist)[2 * tid];
+  const uint4 h1 = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
+  const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) local += c[i];
+  uint32_t incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += t;
+  }
+  if (lane == 31) M.wt[warp] = incl;
+  __syncthreads();
+  uint32_t above = incl - local;
+#pragma unroll
+  for (int w = 0; w < kFW; ++w) above += w < warp ? M.wt[w] : 0u;
+  const uint32_t kk = (uint32_t)k;
+  if (above < kk && kk <= above + local) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (above < kk && kk <= above + c[i]) { M.kb = 8 * tid + i; M.rem = kk - above; M.cnt = c[i]; }
+      above += c[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
+  if (cnt > (uint32_t)kCandMax) {
+    select_fallback(keys, n, k, hist, M);
+    return;
+  }
+  // gather the keys of bin kb with their indices (warp-aggregated slots)
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 1
+  for (int j0 = warp * 32; j0 < n; j0 += kFT) {
+    const int j = j0 + lane;
+    const uint32_t key = j < n ? keys[j] : 0u;
+    const bool m = j < n && sel_bin(maxkey, key) == kb;
+    const uint32_t mb = __ballot_sync(0xffffffffu, m);
+    if (mb) {
+      const int leader = __ffs(mb) - 1;
+      uint32_t slot0 = 0;
+      if (lane == leader) slot0 = atomicAdd(&M.ccount, (uint32_t)__popc(mb));
+      slot0 = __shfl_sync(0xffffffffu, slot0, leader) + __popc(mb & lt);
+      if (m) {
+        M.ck[slot0] = key;
+        M.ci[slot0] = (uint32_t)j;
+      }
+    }
+  }
+  __syncthreads();
+  // rank inside the bin by (key desc, index asc); the first `rem` are selected
+  if (tid < (int)cnt) {
+    const uint32_t mk = M.ck[tid], mi = M.ci[tid];
+    uint32_t rank = 0;
+#pragma unroll 4
+    for (int i = 0; i < (int)cnt; ++i) {
+      const uint32_t ok_ = M.ck[i];
+      rank += (ok_ > mk) || (ok_ == mk && M.ci[i] < mi);
+    }
+    if (rank < rem) atomicOr(&M.csel[mi >> 5], 1u << (mi & 31));
+  }
+  __syncthreads();
+  // selection bitmap: keys of higher bins, plus the selected keys of bin kb
+#pragma unroll 1
+  for (int cw = warp; cw < (n + 31) / 32; cw += kFW) {
+    const int j = 32 * cw + lane;
+    const uint32_t key = j < n ? keys[j] : 0u;
+    const uint32_t w = __ballot_sync(0xffffffffu, j < n && sel_bin(maxkey, key) < kb);
+    if (lane == 0) M.selw[cw] = w | M.csel[cw];
+  }
+  __syncthreads();
+}
+
+// Warp 0: exclusive prefix of the selection words' popcounts into M.pref, then the
+// channels at positions [c0, c0 + nmine) of the ascending selected list into
+// M.mysel.  nw <= 128 words.  A position the bitmap does not hold (a selection of
+// the wrong size) reads channel 0 and flags the call.
+__device__ __noinline__ void positions(int nw, int n, int c0, int nmine, Misc& M, uint16_t* mysel,
+                                      uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  // exclusive prefix over the words, 32 at a time (nw <= 128)
+  uint32_t carry = 0;
+#pragma unroll 1
+  for (int c0w = 0; c0w < nw; c0w += 32) {
+    const int c = c0w + lane;
+    const uint32_t cnt = c < nw ? (uint32_t)__popc(M.selw[c]) : 0u;
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    if (c < nw) M.pref[c] = carry + incl - cnt;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+#pragma unroll 1
+  for (int t = lane; t < nmine; t += 32) {
+    const uint32_t p = (uint32_t)(c0 + t);
+    int lo = 0, hi = nw - 1;  // largest c with pref[c] <= p
+#pragma unroll 1
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (M.pref[mid] <= p) lo = mid; else hi = mid - 1;
+    }
+    // the (p - pref + 1)-th set bit of the word
+    uint32_t w = M.selw[lo];
+#pragma unroll 1
+    for (uint32_t i = M.pref[lo]; i < p; ++i) w &= w - 1u;
+    const uint32_t bit = w ? (uint32_t)(__ffs(w) - 1) : 32u;
+    int ch = 32 * lo + (int)bit;
+    if (bit > 31u || ch >= n) {
+      ch = 0;
+      atomicOr(err, kErrInternal);
+    }
+    mysel[t] = (uint16_t)ch;
+  }
+  __syncwarp();
+}
+
+// Warp 0 of one CTA per cluster: the expert's whole ascending selected list (k entries)
+// and its size into the trace (dense: every channel).
+__device__ __noinline__ void trace_selection(const FusedParams& P, const Misc& M, int nw, int rc) {
+  const int lane = threadIdx.x & 31, k = P.k;
+  if (lane == 0 && P.tr.sel_count) P.tr.sel_count[rc] = k;
+  if (!P.tr.sel) return;
+  uint16_t* out = P.tr.sel + (size_t)rc * k;
+  if (P.dense) {
+#pragma unroll 1
+    for (int j = lane; j < k; j += 32) out[j] = (uint16_t)j;
+    return;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+#pragma unroll 1
+  for (int c = 0; c < nw; ++c) {
+    const uint32_t w = M.selw[c];
+    const uint32_t pos = M.pref[c] + __popc(w & lt);
+    if (((w >> lane) & 1u) && pos < (uint32_t)k) out[pos] = (uint16_t)(32 * c + lane);
+  }
+}
+
+// acc + (8 bf16 of a) . z[0..8)
+__device__ __forceinline__ float dot8f(uint4 a, const float* z, float acc) {
+  acc = fmaf(bf16_lo(a.x), z[0], acc);
+  acc = fmaf(bf16_hi(a.x), z[1], acc);
+  acc = fmaf(bf16_lo(a.y), z[2], acc);
+  acc = fmaf(bf16_hi(a.y), z[3], acc);
+  acc = fmaf(bf16_lo(a.z), z[4], acc);
+  acc = fmaf(bf16_hi(a.z), z[5], acc);
+  acc = fmaf(bf16_lo(a.w), z[6], acc);
+  acc = fmaf(bf16_hi(a.w), z[7], acc);
+  return acc;
+}
+
+// A_e z on this CTA's output slice: lr[i] = sum_rho A[i][rho] * z[rho] (A: the slice's
+// rows, global, [slice][r] bf16).  Rows of r % 8 == 0 go by 16-byte loads.
+__device__ __noinline__ void lowrank_slice(const uint16_t* A, int slice, int r, const float* z, float* lr) {
+#pragma unroll 1
+  for (int i = threadIdx.x; i < slice; i += kFT) {
+    const uint16_t* arow = A + (size_t)i * r;
+    float acc = 0.f;
+    if ((r & 7) == 0) {
+      // up to 8 16-byte loads of the row in flight at once, then their products
+#pragma unroll 1
+      for (int c0 = 0; c0 < r; c0 += 64) {
+        uint4 a[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          a[u] = c0 + 8 * u < r ? __ldg(reinterpret_cast<const uint4*>(arow + c0 + 8 * u)) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (c0 + 8 * u < r) acc = dot8f(a[u], z + c0 + 8 * u, acc);
       }
     } else {
 #pragma unroll 1
-      for (int i = tid; i < P.slice; i += kFT) {
-        const uint16_t* arow = aslice + (size_t)i * r;
-        float acc = 0.f;
+      for (int rho = 0; rho < r; ++rho) acc = fmaf(__uint_as_float((uint32_t)__ldg(arow + rho) << 16), z[rho], acc);
+    }
+    lr[i] = acc;
+  }
+}
+
+// y[0..8) += h * (8 bf16 of v)
+__device__ __forceinline__ void axpy8(float (&y)[8], float h, uint4 v) {
+  y[0] = fmaf(h, bf16_lo(v.x), y[0]);
+  y[1] = fmaf(h, bf16_hi(v.x), y[1]);
+  y[2] = fmaf(h, bf16_lo(v.y), y[2]);
+  y[3] = fmaf(h, bf16_hi(v.y), y[3]);
+  y[4] = fmaf(h, bf16_lo(v.z), y[4]);
+  y[5] = fmaf(h, bf16_hi(v.z), y[5]);
+  y[6] = fmaf(h, bf16_lo(v.w), y[6]);
+  y[7] = fmaf(h, bf16_hi(v.w), y[7]);
+}
+
+
+// score = alpha * |sum of the 8 warps' partials| / 2 for this CTA's nrows rows, pushed
+// to every CTA of the cluster (keys at rows lt0*16 ...), with one max per warp of rows
+// into each CTA's cmax.
+__device__ __forceinline__ void push_scores(const FusedParams& P, Misc& M, const float* part,
+                                         const float* alpha_s, uint32_t* keys, int nrows, int lt0,
+                                         int rc, int q) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, CS = P.cs;
+  const uint32_t rbar_s = smem_addr(&M.bar[kBarScores]);
 #pragma unroll 1
-        for (int rho = 0; rho < r; ++rho) acc = fmaf(bf16_lo(arow[rho]), zs[rho], acc);
-        ylr[i] = acc;
+  for (int lr0 = 0; lr0 < nrows; lr0 += kFT) {
+    const int row = lr0 + tid;
+    uint32_t key = 0;
+    if (row < nrows) {
+      float sc = 0.f;
+#pragma unroll
+      for (int w = 1; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + row];
+      sc = alpha_s[row] * fabsf(sc + part[row]) * 0.5f;
+      key = __float_as_uint(sc);
+      if (P.tr.scores) P.tr.scores[(size_t)rc * P.D.ipad + lt0 * kRowTile + row] = sc;
+      const uint32_t la = smem_addr(keys + lt0 * kRowTile + row);
+#pragma unroll 1
+      for (int dst = 0; dst < CS; ++dst) st_async(mapa(la, dst), key, mapa(rbar_s, dst));
+    }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, key);
+    if (lr0 + warp * 32 < nrows && lane < CS)
+      red_async_max(mapa(smem_addr(&M.cmax), lane), m, mapa(rbar_s, lane));
+  }
+}
+
+// z rows of this CTA: z[q + i*CS] = B_e[q + i*CS] . x (rows staged in shared memory,
+// one warp per row), pushed to every CTA of the cluster.
+__device__ __forceinline__ void push_z(const FusedParams& P, Misc& M, const uint16_t* brows,
+                                    const uint16_t* xs, int q, int nz) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, CS = P.cs;
+  const int d = P.D.d;
+  const uint32_t rbar_z = smem_addr(&M.bar[kBarZ]);
+#pragma unroll 1
+  for (int i = warp; i < nz; i += kFW) {
+    const uint4* br = reinterpret_cast<const uint4*>(brows + (size_t)i * d);
+    const uint4* xv = reinterpret_cast<const uint4*>(xs);
+    float acc = 0.f;
+#pragma unroll 2
+    for (int j = lane; j < d / 8; j += 32) acc = dot8(br[j], xv[j], acc);
+    acc = warp_sum(acc);
+    if (lane < CS) st_async(mapa(smem_addr(&M.z[q + i * CS]), lane), __float_as_uint(acc), mapa(rbar_z, lane));
+  }
+}
+
+// After a wait of this CTA ran out: wait (bounded) for every barrier whose bytes may
+// still be landing -- the copies into this CTA and the other CTAs' pushes -- so that
+// nothing lands in its shared memory after it has exited.
+__device__ __noinline__ void quiesce(Misc& M, int dense, uint32_t* err, uint64_t limit) {
+  if (threadIdx.x != 0) return;
+#pragma unroll 1
+  for (int b = kBarRows; b < kBarRing; ++b)  // (the sketch barrier is armed off the dense path)
+    if (b != kBarSketch || !dense) mbar_wait(&M.bar[b], 0, err, limit);
+}
+
+// Issue the bulk copy of channel `ch`'s record into ring slot `slot`.
+__device__ __forceinline__ void issue_record(const FusedParams& P, Misc& M, uint16_t* ring, int e,
+                                             int ch, int slot) {
+  const uint32_t rb = 6u * (uint32_t)P.D.d;
+  mbar_arrive_expect_tx(&M.bar[kBarRing + slot], rb);
+  bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * P.D.inter + ch) * 3 * P.D.d, rb,
+           &M.bar[kBarRing + slot]);
+}
+
+
+// On a failed wait: wait (bounded) for this CTA's record copies still in flight,
+// so that none lands after the CTA has exited.
+__device__ __noinline__ void drain_ring(Misc& M, int issued, int landed, int ring, uint32_t* err,
+                                        uint64_t limit) {
+  if (threadIdx.x != 0) return;
+#pragma unroll 1
+  for (int i = landed; i < issued; ++i)
+    mbar_wait(&M.bar[kBarRing + i % ring], (uint32_t)(i / ring) & 1u, err, limit);
+}
+
+// ---------------------------------------------------------------- the kernel's phases
+// Each phase is its own function so that the code a launch runs stays small and in one
+// piece (the per-launch instruction fetch is the cost that matters at this size); the
+// shared-memory views are recomputed from the parameters in each.
+
+__device__ __forceinline__ Misc& misc(const FusedParams& P) { return *reinterpret_cast<Misc*>(g_sm + P.o_misc); }
+__device__ __forceinline__ uint8_t* big_of(const FusedParams& P) { return g_sm + P.o_big; }
+template <typename T>
+__device__ __forceinline__ T* in_big(const FusedParams& P, int off) { return reinterpret_cast<T*>(g_sm + P.o_big + off); }
+
+// Barrier set-up, the router rows' copy, zero-fills; before the grid dependency wait.
+__device__ __forceinline__ void phase_prologue(const FusedParams& P, int q) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, d = P.D.d, E = P.D.experts;
+  if (tid == 0) {
+#pragma unroll 1
+    for (int i = 0; i < kBarRing + P.ring; ++i) mbar_init(&M.bar[i], 1);
+    M.cmax = 0u;
+    M.tie = 0u;
+    M.ccount = 0u;
+    fence_mbar_init();
+    const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
+    mbar_arrive_expect_tx(&M.bar[kBarRows], (uint32_t)(e_hi - e_lo) * 2u * d);
+    uint16_t* rows = reinterpret_cast<uint16_t*>(big_of(P));
+#pragma unroll 1
+    for (int j = 0; j < e_hi - e_lo; ++j)
+      bulk_g2s(rows + (size_t)j * P.rrs, P.router_t + (size_t)(e_lo + j) * d, 2u * d, &M.bar[kBarRows]);
+    // bytes the other CTAs will push into this one
+    mbar_arrive_expect_tx(&M.bar[kBarLogits], P.x1_bytes);
+    mbar_arrive_expect_tx(&M.bar[kBarScores], P.sc_bytes);
+    mbar_arrive_expect_tx(&M.bar[kBarZ], P.z_bytes);
+    mbar_arrive_expect_tx(&M.bar[kBarY], P.y_bytes);
+  }
+  if (tid < MSB_MAX_TOP_E) M.ids[tid] = -1;
+  if (tid < kWordsMax) M.csel[tid] = 0u;
+
+  float* logits = in_big<float>(P, P.o_logits);
+  if (E + tid < P.epad) logits[E + tid] = -INFINITY;
+  if (!P.dense) {
+    uint4* hist = in_big<uint4>(P, P.o_hist);
+#pragma unroll 1
+    for (int i = tid; i < kSelBins / 4; i += kFT) hist[i] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The warp sums of 8 values at once by a transposed butterfly (9 shuffles instead of 40):
+// afterwards lane l holds the sum over the warp of v[(l >> 2) & 7].
+__device__ __forceinline__ float warp_sum8(const float (&v)[8]) {
+  const int lane = threadIdx.x & 31;
+  const bool u16 = lane & 16, u8 = lane & 8, u4 = lane & 4;
+  float a[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    a[j] = (u16 ? v[j + 4] : v[j]) + __shfl_xor_sync(0xffffffffu, u16 ? v[j] : v[j + 4], 16);
+  float b[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j)
+    b[j] = (u8 ? a[j + 2] : a[j]) + __shfl_xor_sync(0xffffffffu, u8 ? a[j] : a[j + 2], 8);
+  float c = (u4 ? b[1] : b[0]) + __shfl_xor_sync(0xffffffffu, u4 ? b[0] : b[1], 4);
+  c += __shfl_xor_sync(0xffffffffu, c, 2);
+  c += __shfl_xor_sync(0xffffffffu, c, 1);
+  return c;
+}
+
+// acc + (8 bf16 of a) . xf[0..8)
+__device__ __forceinline__ float dot8xf(uint4 a, const float (&xf)[8], float acc) {
+  acc = fmaf(bf16_lo(a.x), xf[0], acc);
+  acc = fmaf(bf16_hi(a.x), xf[1], acc);
+  acc = fmaf(bf16_lo(a.y), xf[2], acc);
+  acc = fmaf(bf16_hi(a.y), xf[3], acc);
+  acc = fmaf(bf16_lo(a.z), xf[4], acc);
+  acc = fmaf(bf16_hi(a.z), xf[5], acc);
+  acc = fmaf(bf16_lo(a.w), xf[6], acc);
+  acc = fmaf(bf16_hi(a.w), xf[7], acc);
+  return acc;
+}
+
+// A: logits of this CTA's router rows, 8 rows at a time (each thread its 8-element
+// groups of every row, one transposed warp reduction, the warps' sums in shared memory),
+// pushed to every CTA of the cluster; the x permutation for scoring.  Returns ok.
+template <int IT>
+__device__ __forceinline__ bool phase_router(const FusedParams& P, int q, bool ok, const float (&xf)[IT][8]) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, d = P.D.d, E = P.D.experts;
+  const uint16_t* xs = in_big<uint16_t>(P, P.o_x);
+  const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
+  const uint32_t rbar = smem_addr(&M.bar[kBarLogits]);
+  const uint32_t la = smem_addr(in_big<float>(P, P.o_logits) + e_lo);
+  const uint16_t* rows = reinterpret_cast<const uint16_t*>(big_of(P));
+#pragma unroll 1
+  for (int r0 = 0; r0 < e_hi - e_lo; r0 += 8) {
+    const int nb = min(8, e_hi - e_lo - r0);
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int el = (it * kFT + tid) * 8;
+      if (el < d) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (j < nb) v[j] = dot8xf(*reinterpret_cast<const uint4*>(rows + (size_t)(r0 + j) * P.rrs + el), xf[it], v[j]);
       }
     }
-  }
-
-  // Per group: gate . x and up . x of the group's channels on the tensor cores (A =
-  // the records' gate/up rows, bf16 straight from the ring via ldmatrix; B = x; warp w
-  // takes k-steps [ks0, ks1) and the warps' partials meet in
-  // M.red), then h, then y += h_i * down_i with every thread owning 8-element groups.
-  const int KS = d / 16;
-  const int ks0 = warp * KS / kFW, ks1 = (warp + 1) * KS / kFW;
-  const uint32_t* x32 = reinterpret_cast<const uint32_t*>(P.x);
-  const int c4 = lane & 3, g8 = lane >> 2;
-  // d <= 2048: the x B-fragments of this warp's k-steps sit in registers (loaded while
-  // the records are in flight); larger d reads them through L1 at each k-step
-  constexpr int KSW = IT == 1 ? 16 : 0;
-  uint32_t xb[KSW > 0 ? KSW : 1][2];
+    const float sw = warp_sum8(v);
+    if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
+    __syncthreads();
+    if (tid < nb) {
+      float acc = 0.f;
 #pragma unroll
-  for (int i = 0; i < KSW; ++i)
-    if (ks0 + i < ks1) {
-      xb[i][0] = __ldg(x32 + (ks0 + i) * 8 + c4);
-      xb[i][1] = __ldg(x32 + (ks0 + i) * 8 + 4 + c4);
+      for (int w = 0; w < kFW; ++w) acc += M.red8[w][tid];
+#pragma unroll 1
+      for (int dst = 0; dst < P.cs; ++dst)
+        st_async(mapa(la + 4u * (r0 + tid), dst), __float_as_uint(acc), mapa(rbar, dst));
     }
+    __syncthreads();
+  }
+  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
+  if (!P.dense) {
+    uint32_t* xperm = in_big<uint32_t>(P, P.o_xperm);
+#pragma unroll 1
+    for (int i = tid; i < d / 2; i += kFT) {
+      const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
+      xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
+    }
+  }
+  return wait_phase(&M.bar[kBarLogits], 0, P.err) && ok;
+}
+
+// The copies of routed expert e: sketch tiles and alpha of this CTA's rows, B_e rows of
+// its z entries; the A_e rows of its output slice into L2 (thread 0).
+__device__ __forceinline__ void issue_expert(const FusedParams& P, int e, int q, int nt, int lt0, int nz) {
+  Misc& M = misc(P);
+  const int d = P.D.d, r = P.D.rank, KC = d / kColChunk, CS = P.cs;
+  const int ntile_all = P.D.ipad / kRowTile;
+  fence_proxy_async();  // the router rows were read through the generic proxy
+  if (!P.dense) {
+    const uint32_t code_bytes = (uint32_t)nt * KC * kChunkWords * 4u;
+    mbar_arrive_expect_tx(&M.bar[kBarSketch], code_bytes + (uint32_t)nt * kRowTile * 4u);
+    if (nt) {
+      bulk_g2s(big_of(P), P.sketch + ((size_t)e * ntile_all + lt0) * KC * kChunkWords, code_bytes,
+               &M.bar[kBarSketch]);
+      bulk_g2s(in_big<float>(P, P.o_alpha), P.alpha + (size_t)e * P.D.ipad + (size_t)lt0 * kRowTile,
+               nt * kRowTile * 4u, &M.bar[kBarSketch]);
+    }
+  }
+  mbar_arrive_expect_tx(&M.bar[kBarLow], (uint32_t)nz * 2u * d);
+  uint16_t* brows = in_big<uint16_t>(P, P.o_brows);
+#pragma unroll 1
+  for (int i = 0; i < nz; ++i)
+    bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[kBarLow]);
+  if (r > 0) prefetch_l2(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, 2u * P.slice * r);
+}
+
+// B: sketch scores of this CTA's rows on the tensor cores, pushed with the warps'
+// largest keys; z = B_e x rows, pushed.  Returns ok.
+__device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc, int nt, int lt0, int nz,
+                                          bool ok) {
+  Misc& M = misc(P);
+  const int warp = threadIdx.x >> 5, KC = P.D.d / kColChunk;
+  float* part = in_big<float>(P, P.o_part);
+  if (!P.dense) {
+    ok = wait_phase(&M.bar[kBarSketch], 0, P.err) && ok;
+    MARK(4);
+    if (nt > 0)
+      score_tiles(reinterpret_cast<const uint2*>(big_of(P)), in_big<const uint4>(P, P.o_xperm), nt, KC,
+                  part + warp * P.tpc * kRowTile);
+    __syncthreads();
+    MARK(5);
+    push_scores(P, M, part, in_big<float>(P, P.o_alpha), in_big<uint32_t>(P, P.o_keys), nt * kRowTile, lt0,
+                rc, q);
+  }
+  if (nz > 0) {
+    ok = wait_phase(&M.bar[kBarLow], 0, P.err) && ok;
+    push_z(P, M, in_big<uint16_t>(P, P.o_brows), in_big<uint16_t>(P, P.o_x), q, nz);
+  }
+  return ok;
+}
+
+// C: exact top-k over the cluster's scores (or, dense, every channel) and this CTA's
+// share of it into M.mysel; then the first record copies.  Returns ok.
+__device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q, int rc, int nmine, int c0,
+                                          bool ok) {
+  Misc& M = misc(P);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, I = P.D.inter;
+  const int nw = (I + 31) / 32;
+  if (!P.dense) {
+    ok = wait_phase(&M.bar[kBarScores], 0, P.err) && ok;
+    MARK(7);
+    select_topk(in_big<uint32_t>(P, P.o_keys), I, P.k, M.cmax, in_big<uint32_t>(P, P.o_hist), M);
+    MARK(8);
+    if (warp == 0) positions(nw, I, c0, nmine, M, MYSEL(P), P.err);
+  } else {
+    if (warp == 0)
+#pragma unroll 1
+      for (int t = lane; t < nmine; t += 32) MYSEL(P)[t] = (uint16_t)(c0 + t);
+    __syncthreads();  // (the dense path had no barrier since phase A: big is free now)
+  }
+  MARK(9);
+  if (q == 0 && (P.tr.sel || P.tr.sel_count) && warp == 0) trace_selection(P, M, nw, rc);
+  if (blockIdx.x == 0 && (P.tr.expert_ids || P.tr.expert_w || P.tr.union_count))
+    trace_routing(P.tr, M, P.D.experts, P.D.top_e, P.k);
+  // the ring now takes over `big`: every thread is past its last use of phases A-C
+  if (warp == 0 && ok) {
+    fence_proxy_async();
+    uint16_t* ring = reinterpret_cast<uint16_t*>(big_of(P));
+    const int nfirst = min(P.ring, nmine);
+#ifdef MSB_INSTRUMENTED
+    if (lane < nfirst && !(P.skip == 1u && blockIdx.x == 0 && lane == 0))
+#else
+    if (lane < nfirst)
+#endif
+      issue_record(P, M, ring, e, MYSEL(P)[lane], lane);
+  }
+  return ok;
+}
+
+// D: the records in batches as they land (the first batch of one record, so that a
+// slot frees early, then up to bmax = min(4, ring / 2)).  gate.x and up.x of a batch: each
+// thread its 8-element groups of every gate and up row, one transposed warp reduction of
+// the (up to) 8 values, the warps' sums in shared memory; h = silu(gate.x) * up.x; then
+// every thread adds h * down over its groups.  After the first barrier of a batch the
+// previous batch's slots are refilled.  Then y is pushed, slice by slice, to each slice's
+// owner.  Returns ok.
+template <int IT>
+__device__ __forceinline__ bool phase_records(const FusedParams& P, int e, int q, int nmine, bool ok,
+                                              const float (&xf)[IT][8]) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, d = P.D.d;
+  const uint16_t* ring = reinterpret_cast<const uint16_t*>(big_of(P));
+  const int bmax = max(1, min(4, P.ring / 2));
   float y[IT][8];
 #pragma unroll
   for (int it = 0; it < IT; ++it)
 #pragma unroll
     for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
-  // channel g0 + i of a group sits in slot s0 + i (wrapping at the ring size, where the
-  // slot's phase parity flips); s0 and its parity par0 advance group by group
-  int s0 = 0;
-  uint32_t par0 = 0;
+  int s0 = 0, pb0 = 0, pnb = 0;  // first slot of this batch; first slot and size of the previous
+  uint32_t par0 = 0;             // phase parity of slot s0
+  int issued = ok ? min(P.ring, nmine) : 0, landed = 0;
 #pragma unroll 1
-  for (int g0 = 0; g0 < nmine; g0 += P.group) {
-    const int ng = min(P.group, nmine - g0);
+  for (int i = 0; i < nmine;) {
+    const int nb = i == 0 ? 1 : min(bmax, nmine - i);
+    if (ok) {
 #pragma unroll 1
-    for (int i = 0; i < ng; ++i) {
-      const int sl = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
-      ok = ok && wait_phase(&M.bar[2 + sl], s0 + i < P.ring ? par0 : par0 ^ 1u, P.err);
+      for (int j = 0; j < nb && ok; ++j) {
+        const int sl = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
+        ok = wait_phase(&M.bar[kBarRing + sl], s0 + j < P.ring ? par0 : par0 ^ 1u, P.err);
+      }
+      if (ok) landed = i + nb;
     }
-#pragma unroll 1
-    for (int tb = 0; tb < ng; tb += 8) {
-      // this lane's ldmatrix row: channel tb + lane % 8 (rows past ng repeat channel tb;
-      // their results are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 * (lane / 16)
-      const int ch = (tb + (lane & 7) < ng) ? tb + (lane & 7) : tb;
-      const int csl = s0 + ch < P.ring ? s0 + ch : s0 + ch - P.ring;
-      uint32_t a_addr = smem_addr(ring + (size_t)csl * P.rs + ((lane >> 3) & 1) * d +
-                                  8 * (lane >> 4)) + 32u * ks0;
-      float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
-      int ks = ks0;
-      if (ok && KSW > 0) {
+    {
+      // value 2j: gate_j . x, value 2j + 1: up_j . x (record j of the batch)
+      float v[8];
 #pragma unroll
-        for (int i = 0; i < KSW; i += 2) {
-          if (ks0 + i + 1 < ks1) {
-            uint32_t a[2][4];
-            ldsm_x4(a_addr + 32u * i, a[0][0], a[0][1], a[0][2], a[0][3]);
-            ldsm_x4(a_addr + 32u * (i + 1), a[1][0], a[1][1], a[1][2], a[1][3]);
-            mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], xb[i][0], xb[i][1]);
-            mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], xb[i + 1][0], xb[i + 1][1]);
-          } else if (ks0 + i < ks1) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(a_addr + 32u * i, a0, a1, a2, a3);
-            mma_bf16(acc0, a0, a1, a2, a3, xb[i][0], xb[i][1]);
+      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j < nb) {
+          const int sl = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
+          const uint16_t* rec = ring + (size_t)sl * P.rs;
+#pragma unroll
+          for (int it = 0; it < IT; ++it) {
+            const int el = (it * kFT + tid) * 8;
+            if (el < d) {
+              v[2 * j] = dot8xf(*reinterpret_cast<const uint4*>(rec + el), xf[it], v[2 * j]);
+              v[2 * j + 1] = dot8xf(*reinterpret_cast<const uint4*>(rec + d + el), xf[it], v[2 * j + 1]);
+            }
           }
         }
-      } else if (ok) {
-#pragma unroll 1
-        for (; ks + 4 <= ks1; ks += 4, a_addr += 128u) {
-          uint32_t a[4][4], b[4][2];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            ldsm_x4(a_addr + 32u * u, a[u][0], a[u][1], a[u][2], a[u][3]);
-            b[u][0] = __ldg(x32 + (ks + u) * 8 + c4);
-            b[u][1] = __ldg(x32 + (ks + u) * 8 + 4 + c4);
-          }
-          mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b[0][0], b[0][1]);
-          mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b[1][0], b[1][1]);
-          mma_bf16(acc0, a[2][0], a[2][1], a[2][2], a[2][3], b[2][0], b[2][1]);
-          mma_bf16(acc1, a[3][0], a[3][1], a[3][2], a[3][3], b[3][0], b[3][1]);
-        }
-#pragma unroll 1
-        for (; ks < ks1; ++ks, a_addr += 32u) {
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(a_addr, a0, a1, a2, a3);
-          mma_bf16(acc0, a0, a1, a2, a3, __ldg(x32 + ks * 8 + c4), __ldg(x32 + ks * 8 + 4 + c4));
-        }
       }
-      // column 0 of D: lanes with lane % 4 == 0 hold gate (row g8) and up (row g8 + 8)
-      if (c4 == 0 && tb + g8 < ng) {
-        M.red[warp][2 * (tb + g8)] = acc0[0] + acc1[0];
-        M.red[warp][2 * (tb + g8) + 1] = acc0[2] + acc1[2];
-      }
+      const float sw = warp_sum8(v);
+      if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
     }
     ok = __syncthreads_and(ok);
-    if (tid < ng) {
+    // every thread has finished the previous batch: refill its slots (warp 1, while warp 0
+    // forms h)
+    if (tid == 32 && ok && pnb > 0 && issued < nmine) {
+      uint16_t* wring = reinterpret_cast<uint16_t*>(big_of(P));
+      fence_proxy_async();
+#pragma unroll 1
+      for (int j = 0; j < pnb && issued < nmine; ++j, ++issued)
+        issue_record(P, M, wring, e, MYSEL(P)[issued], pb0 + j < P.ring ? pb0 + j : pb0 + j - P.ring);
+    }
+    if (i == 0) MARK(11);
+    if (tid < nb) {
       float g = 0.f, u = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFW; ++w) { g += M.red[w][2 * tid]; u += M.red[w][2 * tid + 1]; }
+      for (int w = 0; w < kFW; ++w) {
+        g += M.red8[w][2 * tid];
+        u += M.red8[w][2 * tid + 1];
+      }
       M.h[tid] = __fdividef(g, 1.0f + __expf(-g)) * u;
     }
     __syncthreads();
-    if (ok) {
-      // y += h_i * down_i over this thread's elements
-#pragma unroll 4
-      for (int i = 0; i < ng; ++i) {
-        const int sl = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
-        const uint16_t* rec = ring + (size_t)sl * P.rs + 2 * d;
-        const float h = M.h[i];
+    // y += h_j * down_j over this thread's groups, two records at a time
+#pragma unroll 1
+    for (int j = 0; j < nb; j += 2) {
+      const int sa = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
+      const int sb = s0 + j + 1 < P.ring ? s0 + j + 1 : s0 + j + 1 - P.ring;
+      const uint16_t* reca = ring + (size_t)sa * P.rs + 2 * d;
+      const uint16_t* recb = ring + (size_t)sb * P.rs + 2 * d;
+      const float ha = M.h[j], hb = j + 1 < nb ? M.h[j + 1] : 0.f;
 #pragma unroll
-        for (int it = 0; it < IT; ++it) {
-          const int el = (it * kFT + tid) * 8;
-          if (el < d) {
-            const uint4 dv = *reinterpret_cast<const uint4*>(rec + el);
-            y[it][0] = fmaf(h, bf16_lo(dv.x), y[it][0]);
-            y[it][1] = fmaf(h, bf16_hi(dv.x), y[it][1]);
-            y[it][2] = fmaf(h, bf16_lo(dv.y), y[it][2]);
-            y[it][3] = fmaf(h, bf16_hi(dv.y), y[it][3]);
-            y[it][4] = fmaf(h, bf16_lo(dv.z), y[it][4]);
-            y[it][5] = fmaf(h, bf16_hi(dv.z), y[it][5]);
-            y[it][6] = fmaf(h, bf16_lo(dv.w), y[it][6]);
-            y[it][7] = fmaf(h, bf16_hi(dv.w), y[it][7]);
-          }
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kFT + tid) * 8;
+        if (el < d) {
+          const uint4 va = *reinterpret_cast<const uint4*>(reca + el);
+          const uint4 vb = j + 1 < nb ? *reinterpret_cast<const uint4*>(recb + el) : make_uint4(0u, 0u, 0u, 0u);
+          axpy8(y[it], ha, va);
+          axpy8(y[it], hb, vb);
         }
       }
     }
-    __syncthreads();
-    // refill the slots just consumed
-    if (warp == 0 && ok) {  // channel g0 + i + ring goes where g0 + i was; lane i issues it
-      fence_proxy_async();
-      const int i = lane, nx = g0 + lane + P.ring;
-      if (i < ng && nx < nmine) {
-        const int ch = M.mysel[nx];
-        const int slot = s0 + i < P.ring ? s0 + i : s0 + i - P.ring;
-        mbar_arrive_expect_tx(&M.bar[2 + slot], rec_bytes);
-        bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * I + ch) * 3 * d, rec_bytes,
-                 &M.bar[2 + slot]);
-      }
-    }
-    s0 += ng;
-    if (s0 >= P.ring) {
-      s0 -= P.ring;
-      par0 ^= 1u;
-    }
+    pb0 = s0;
+    pnb = nb;
+    s0 += nb;
+    if (s0 >= P.ring) { s0 -= P.ring; par0 ^= 1u; }
+    i += nb;
   }
-
-  // ------------------------------------------------------------------ phase D: reduce, combine
-  // partial output to this CTA's shared buffer; each owner then sums its slice over
-  // the cluster with 16-byte DSMEM loads
+  if (!ok) drain_ring(M, issued, landed, P.ring, P.err, WAIT_LIMIT);
+  // every thread waits for the drain: no thread pushes or arrives at the cluster barrier
+  // ahead of it (the arrive is warp-aligned, and every push of this CTA must be issued
+  // before any CTA of the cluster can pass the barrier)
+  __syncthreads();
+  MARK(12);
+  // push each 8-element group to the owner of its slice: rbuf[q][offset in slice]
+  const uint32_t rbuf = smem_addr(g_sm + P.o_rbuf), rbar_y = smem_addr(&M.bar[kBarY]);
 #pragma unroll
   for (int it = 0; it < IT; ++it) {
     const int el = (it * kFT + tid) * 8;
     if (el < d) {
-      *reinterpret_cast<float4*>(ybuf + el) = make_float4(y[it][0], y[it][1], y[it][2], y[it][3]);
-      *reinterpret_cast<float4*>(ybuf + el + 4) = make_float4(y[it][4], y[it][5], y[it][6], y[it][7]);
+      const int owner = el / P.slice, off = el - owner * P.slice;
+      const uint32_t ra = mapa(rbuf + 4u * (q * P.slice + off), owner), rb = mapa(rbar_y, owner);
+      st_async4(ra, y[it][0], y[it][1], y[it][2], y[it][3], rb);
+      st_async4(ra + 16u, y[it][4], y[it][5], y[it][6], y[it][7], rb);
     }
   }
-  cluster.sync();
+  return ok;
+}
+
+// E: the owner of slice q sums the cluster's partials of it, adds A_e z, weights by
+// the router and reduction-adds into the FP32 accumulator; the last of the K
+// contributions converts the slice to BF16 and re-zeroes it.  Returns ok.
+__device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int rc, bool ok) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, K = P.D.top_e;
+  const float* lr = reinterpret_cast<const float*>(g_sm + P.o_lr);
+  const float* rbuf = reinterpret_cast<const float*>(g_sm + P.o_rbuf);
+  ok = wait_phase(&M.bar[kBarY], 0, P.err) && ok;
+  MARK(13);
+  const float we = M.wk[rc];
   if (ok) {
 #pragma unroll 1
     for (int j = tid; j < P.slice / 4; j += kFT) {
-      const int el = q * P.slice + 4 * j;
-      // all CS remote loads in flight at once
-      float4 v[16];
-#pragma unroll
-      for (int src = 0; src < 16; ++src)
-        if (src < CS) v[src] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(ybuf, src) + el);
-      float4 acc = v[0];
-#pragma unroll
-      for (int src = 1; src < 16; ++src)
-        if (src < CS) { acc.x += v[src].x; acc.y += v[src].y; acc.z += v[src].z; acc.w += v[src].w; }
-      if (lr_out) {
-        acc.x += ylr[4 * j]; acc.y += ylr[4 * j + 1]; acc.z += ylr[4 * j + 2]; acc.w += ylr[4 * j + 3];
+      float4 acc = P.D.rank > 0 ? *reinterpret_cast<const float4*>(lr + 4 * j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int src = 0; src < P.cs; ++src) {
+        const float4 v = *reinterpret_cast<const float4*>(rbuf + src * P.slice + 4 * j);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      red_add_v4(P.y_acc + el, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
+      red_add_v4(P.y_acc + q * P.slice + 4 * j, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
     }
   }
-  cluster.sync();  // no CTA leaves while its buffer may still be read
-  // the barrier orders warp 0's reduction-adds before thread 0's fence, which makes them
-  // visible GPU-wide before the slice counter moves
+  __threadfence();
+  __syncthreads();
   if (tid == 0) {
-    __threadfence();
-    M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K * P.cpe - 1));
+    M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K - 1));
     if (M.last) __threadfence();
   }
   __syncthreads();
   if (M.last) {
     // every contribution to this slice has arrived: convert, re-zero, reset
 #pragma unroll 1
-    for (int i = tid; i < P.slice; i += kFT) {
-      const float v = atomicExch(P.y_acc + q * P.slice + i, 0.f);
-      P.out[q * P.slice + i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    for (int j = tid; j < P.slice / 4; j += kFT) {
+      float4* p = reinterpret_cast<float4*>(P.y_acc + q * P.slice) + j;
+      const float4 v = __ldcg(p);
+      __stcg(p, make_float4(0.f, 0.f, 0.f, 0.f));
+      const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.y)) << 16);
+      const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
+                          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.w)) << 16);
+      reinterpret_cast<uint2*>(P.out + q * P.slice)[j] = make_uint2(lo, hi);
     }
     if (tid == 0) P.slice_cnt[q] = 0u;
   }
+  return ok;
+}
+
+template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
+__global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_constant__ FusedParams P) {
+  const int CS = P.cs;
+  const int q = (int)cluster_rank();
+  const int rc = blockIdx.x / CS;  // which routed expert (rank order)
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int d = P.D.d, r = P.D.rank;
+  Misc& M = misc(P);
+
+  phase_prologue(P, q);
+  MARK(0);
+  __syncthreads();
+  // barrier inits, cmax = 0 and the zero-fills above precede any remote access
+  cluster_arrive();
+  // x and the accumulator may be written by the previous launch: wait for it here
+  pdl_wait();
+  pdl_trigger();  // the next launch may start its weight-only prologue
+  uint16_t* xs = in_big<uint16_t>(P, P.o_x);
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&M.bar[kBarX], 2u * d);
+    bulk_g2s(xs, P.x, 2u * d, &M.bar[kBarX]);
+  }
+  cluster_wait();  // every CTA of the cluster has initialised its barriers
+  bool ok = wait_phase(&M.bar[kBarX], 0, P.err);
+  ok = wait_phase(&M.bar[kBarRows], 0, P.err) && ok;
+  MARK(1);
+  // this thread's 8-element groups of x as floats (for the router rows and the records;
+  // x itself is overwritten by the ring later)
+  float xf[IT][8];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int el = (it * kFT + tid) * 8;
+    const uint4 xv = el < d ? reinterpret_cast<const uint4*>(xs)[el / 8] : make_uint4(0u, 0u, 0u, 0u);
+    xf[it][0] = bf16_lo(xv.x); xf[it][1] = bf16_hi(xv.x); xf[it][2] = bf16_lo(xv.y); xf[it][3] = bf16_hi(xv.y);
+    xf[it][4] = bf16_lo(xv.z); xf[it][5] = bf16_hi(xv.z); xf[it][6] = bf16_lo(xv.w); xf[it][7] = bf16_hi(xv.w);
+  }
+
+  ok = phase_router<IT>(P, q, ok, xf);
+  MARK(2);
+  router_rank(in_big<float>(P, P.o_logits), P.D.experts, P.epad, P.D.top_e, M, P.err);
+  int e = M.ids[rc];
+  if (e < 0) {  // a rank left empty (non-finite logits): keep a valid index, the call is flagged
+    e = rc;
+    if (tid == 0) atomicOr(P.err, kErrNonFinite);
+  }
+  MARK(3);
+  const int ntile_all = P.D.ipad / kRowTile;
+  const int lt0 = min(ntile_all, q * P.tpc), lt1 = min(ntile_all, lt0 + P.tpc);
+  const int nt = lt1 - lt0;
+  const int nz = r > q ? (r - q + CS - 1) / CS : 0;  // z rows q, q+CS, ... below r
+  if (tid == 0) issue_expert(P, e, q, nt, lt0, nz);
+  // combine weights (warp 0; read in phase E, many barriers later)
+  if (warp == 0) router_weights(in_big<float>(P, P.o_logits), P.D.experts, P.D.top_e, P.D.renorm, M);
+
+  ok = phase_scores(P, q, rc, nt, lt0, nz, ok);
+  MARK(6);
+  const int c0 = q * P.k / CS, c1 = (q + 1) * P.k / CS;
+  const int nmine = c1 - c0;
+  ok = phase_select(P, e, q, rc, nmine, c0, ok);
+  // A_e z on this CTA's output slice while the first records fly (A_e from L2)
+  if (r > 0) {
+    ok = wait_phase(&M.bar[kBarZ], 0, P.err) && ok;
+    lowrank_slice(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, P.slice, r, M.z,
+                  reinterpret_cast<float*>(g_sm + P.o_lr));
+  }
+  MARK(10);
+  ok = phase_records<IT>(P, e, q, nmine, ok, xf);
+  cluster_arrive();  // paired with the wait before exit: no CTA leaves while pushes may target it
+  __syncthreads();   // lr complete (a CTA may have had no records, hence no barrier since)
+  ok = phase_combine(P, q, rc, ok);
+  MARK(14);
+  cluster_wait();
+  // every push aimed at this CTA has now been issued: if any wait of this CTA ran out,
+  // wait (bounded) for whatever may still be landing before the CTA exits
+  if (__syncthreads_or(!ok)) quiesce(M, P.dense, P.err, WAIT_LIMIT);
+#ifdef MSB_INSTRUMENTED
+  if (P.marks && tid == 0) {
+    uint32_t smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    P.marks[blockIdx.x * kMarks + 15] = smid;
+  }
+#endif
 }
 
 // =====================================================================================
@@ -836,74 +1135,82 @@ KernelFn kernel_for(int d) {
 }
 
 // Fill the carve-up for cluster size cs within `limit` bytes of shared memory.
-bool plan(FusedParams& P, const Dims& D, int k, int cs, int cpe, int limit) {
-  const int d = D.d, E = D.experts, ipad = D.ipad, r = D.rank;
-  if (d % (8 * cs) != 0) return false;
+bool plan(FusedParams& P, const Dims& D, int k, int cs, int limit) {
+  const int d = D.d, E = D.experts, ipad = D.ipad, r = D.rank, I = D.inter;
+  if (d % (8 * cs) != 0 || D.top_e < 1) return false;
   P.cs = cs;
-  P.cpe = cpe;
   P.rpc = (E + cs - 1) / cs;
   P.tpc = (ipad / kRowTile + cs - 1) / cs;
-  P.zpc = (r + cs - 1) / cs;
   P.slice = d / cs;
-  int o = 0;
-  P.o_z = o;      o = align_up(o + 4 * (r > 0 ? r : 1), 128);
-  P.o_ylr = o;    o = align_up(o + 4 * P.slice, 128);
-  P.o_misc = o;   o = align_up(o + (int)sizeof(Misc), 128);
-  P.o_big = o;
-  // offsets inside big (see the kernel): phase A and phase B scratch
-  const int need_rows = align_up(P.rpc * 2 * d, 128);
-  P.o_logits = need_rows;
   P.epad = (E + 63) / 64 * 64;
-  const int need_a = need_rows + align_up(4 * P.epad, 128);
-  int b = (P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4) + P.zpc * 2 * d;
+  const int per_cta = (k + cs - 1) / cs;  // channels a CTA reads
+  if (per_cta > kMyselMax) return false;
+  int o = 0;
+  P.o_misc = o;  o = align_up(o + (int)sizeof(Misc), 128);
+  P.o_lr = o;    o = align_up(o + 4 * P.slice, 128);
+  P.o_rbuf = o;  o = align_up(o + 4 * d, 128);
+  P.o_mysel = o; o = align_up(o + 2 * per_cta, 128);
+  P.o_big = o;
+  // phase A/B region at the start of big: router rows, then (reused) sketch tiles,
+  // alpha and B_e rows
+  P.rrs = d + 8;
+  P.rs = 3 * d + 8;
+  const int rows_b = align_up(P.rpc * 2 * P.rrs, 128);
+  int b = P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4;
   b = align_up(b, 128);
   P.o_alpha = b;  b = align_up(b + 4 * P.tpc * kRowTile, 128);
-  P.o_part = b;   b = align_up(b + 4 * kFW * P.tpc * kRowTile, 128);
-  P.o_xperm = b;  b = align_up(b + 2 * d, 128);
-  P.o_keys = b;   b = align_up(b + 4 * ipad, 128);
-  P.o_hist = b;   b = align_up(b + (P.dense ? 0 : 4 * kSelBins), 128);
-  // x lives past both phases' scratch until the ring takes over
-  P.o_xbig = align_up(need_a > b ? need_a : b, 128);
-  const int need_b = align_up(P.o_xbig + 2 * d, 128);
-  const int need_d = 4 * d;
-  if ((k + cs * cpe - 1) / (cs * cpe) > kMyselMax) return false;
-  P.aslice_regs = (r > 0 && r % 8 == 0 && P.slice * r / 8 <= kAregs * kFT) ? 1 : 0;
-  const int aslice_bytes = P.aslice_regs ? 0 : align_up(P.slice * r * 2, 128);
-  const int avail = limit - o - aslice_bytes;
-  P.rs = 3 * d + 8;
+  P.o_brows = b;  b = align_up(b + ((r + cs - 1) / cs) * 2 * d, 128);
+  int s = rows_b > b ? rows_b : b;
+  P.o_x = s;      s = align_up(s + 2 * d, 128);
+  P.o_xperm = s;  s = align_up(s + 2 * d, 128);
+  P.o_logits = s; s = align_up(s + 4 * P.epad, 128);
+  P.o_keys = s;   s = align_up(s + 4 * ipad, 128);
+  P.o_hist = s;   s = align_up(s + (P.dense ? 0 : 4 * kSelBins), 128);
+  P.o_part = s;   s = align_up(s + 4 * kFW * P.tpc * kRowTile, 128);
+  const int need_abc = s;
   const int rec = 2 * P.rs;
+  const int avail = limit - o;
   int ring = avail / rec;
   if (ring > kRingMax) ring = kRingMax;
-  if (ring < 2 || need_a > avail || need_b > avail || need_d > avail) return false;
-  const int per_cta = (k + cs * cpe - 1) / (cs * cpe);  // channels a CTA reads
-  if (ring > per_cta) ring = per_cta < 2 ? 2 : per_cta;
+  if (ring > per_cta) ring = per_cta < 1 ? 1 : per_cta;
+  if (ring < 1 || need_abc > avail) return false;
+  // a record's slot is refilled one record later: with refills the ring needs two slots
+  if (per_cta > ring && ring < 2) return false;
   P.ring = ring;
-  // one group when every record fits the ring, else two groups in flight
-  P.group = per_cta <= ring ? ring : (ring + 1) / 2;
-  int bigb = ring * rec;
-  if (need_a > bigb) bigb = need_a;
-  if (need_b > bigb) bigb = need_b;
-  if (need_d > bigb) bigb = need_d;
-  P.o_aslice_off = bigb;
-  P.smem = o + bigb + aslice_bytes;
+  const int bigb = ring * rec > need_abc ? ring * rec : need_abc;
+  P.smem = o + bigb;
+  // bytes pushed into each CTA: every logit; every sketch row's key and one max per
+  // (CTA, warp of rows); every z entry; every partial output element
+  uint32_t maxmsgs = 0;
+  const int ntile_all = ipad / kRowTile;
+  for (int qq = 0; qq < cs; ++qq) {
+    const int t0 = qq * P.tpc < ntile_all ? qq * P.tpc : ntile_all;
+    const int t1 = t0 + P.tpc < ntile_all ? t0 + P.tpc : ntile_all;
+    const int nrows = (t1 - t0) * kRowTile;
+    maxmsgs += (uint32_t)((nrows + 31) / 32);
+  }
+  P.x1_bytes = 4u * (uint32_t)E;
+  P.sc_bytes = P.dense ? 0u : 4u * ((uint32_t)ipad + maxmsgs);
+  P.z_bytes = 4u * (uint32_t)r;
+  P.y_bytes = 4u * (uint32_t)d;
+  (void)I;
   return P.smem <= limit;
 }
 
-// Prefer plans whose CTAs can pair on an SM (all clusters then fit the GPCs), then
-// one 16-CTA cluster per routed expert when all K are resident, then two 8-CTA
-// clusters per expert; otherwise any plan (non-resident clusters run later).
+// Prefer 16-CTA clusters small enough to pair on an SM (all K clusters then fit the
+// GPCs), then 16-CTA clusters at any size when all K are resident, then 8-CTA
+// clusters; otherwise decline (the multi-kernel path runs).
 bool choose(FusedParams& P, const Dims& D, int k) {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64 || !g_ready[dev]) return false;
   const int K = D.top_e;
   const int pair = g_pair_smem[dev];
   const bool have16 = g_max_clusters16[dev] >= 1, have8 = g_max_clusters8[dev] >= 1;
-  if (have16 && plan(P, D, k, 16, 1, pair)) return true;
-  if (have8 && plan(P, D, k, 8, 2, pair)) return true;
-  if (have16 && g_max_clusters16[dev] >= K && plan(P, D, k, 16, 1, kSmemMax)) return true;
-  if (have8 && g_max_clusters8[dev] >= 2 * K && plan(P, D, k, 8, 2, kSmemMax)) return true;
-  if (have16 && plan(P, D, k, 16, 1, kSmemMax)) return true;
-  if (have8 && plan(P, D, k, 8, 2, kSmemMax)) return true;
+  if (have16 && plan(P, D, k, 16, pair)) return true;
+  if (have16 && g_max_clusters16[dev] >= K && plan(P, D, k, 16, kSmemMax)) return true;
+  if (have8 && plan(P, D, k, 8, pair)) return true;
+  if (have8 && g_max_clusters8[dev] >= K && plan(P, D, k, 8, kSmemMax)) return true;
+  if (have16 && plan(P, D, k, 16, kSmemMax)) return true;
   return false;
 }
 
@@ -937,6 +1244,10 @@ int fused_setup() {
       return MSB_ECUDA;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
       cudaGetLastError();
+    // one CTA of a cluster per SM where the GPC has room, rather than two on one SM
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeClusterSchedulingPolicyPreference,
+                             cudaClusterSchedulingPolicySpread) != cudaSuccess)
+      cudaGetLastError();
   }
   int per_sm = 0, reserved = 0;
   if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
@@ -957,11 +1268,11 @@ void fused_plan_info(const Dims& D, int k, int* info) {
   FusedParams P{};
   P.dense = (k == D.inter);
   const int dev = cur_dev();
-  #pragma unroll 1
+#pragma unroll 1
   for (int i = 0; i < 6; ++i) info[i] = 0;
   if (choose(P, D, k)) {
     info[0] = P.cs;
-    info[1] = P.cpe;
+    info[1] = 1;
     info[2] = P.ring;
     info[3] = P.smem;
   }
@@ -976,6 +1287,7 @@ bool fused_supported(const Dims& D, int k) {
   P.dense = (k == D.inter);
   return choose(P, D, k);
 }
+
 
 int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* records,
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
@@ -993,25 +1305,32 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
   P.err = err;
   P.slice_cnt = counters + kCntFusedSlices;
   P.y_acc = y_acc;
+#ifdef MSB_INSTRUMENTED
+  P.marks = debug_ctl().marks;
+  P.skip = debug_ctl().skip;
+  P.wait_ns = debug_ctl().wait_ns ? debug_ctl().wait_ns : kWaitLimitNs;
+#endif
   P.tr = tr;
   P.D = D;
   P.k = k;
   P.dense = (k == D.inter);
   if (!choose(P, D, k)) return MSB_ENOTFUSED;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P.cs * P.cpe * D.top_e, 1, 1);
+  cfg.gridDim = dim3(P.cs * D.top_e, 1, 1);
   cfg.blockDim = dim3(kFT, 1, 1);
   cfg.dynamicSmemBytes = P.smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = P.cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
+  attr[2].id = cudaLaunchAttributeClusterSchedulingPolicyPreference;
+  attr[2].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 3;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(D.d), P);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }

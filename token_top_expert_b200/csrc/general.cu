@@ -473,6 +473,10 @@ struct GatherCfg {
   int ch;       // channels per work item (<= kGCh)
   int nlr;      // low-rank work items per slot
   int dense;    // 1: every channel is selected (no sketch)
+  uint64_t wait_ns;  // bounded-wait limit
+#ifdef MSB_INSTRUMENTED
+  uint32_t skip;     // 2: the CTA of work item 0 never issues its first stage (test only)
+#endif
 };
 
 __device__ __forceinline__ void red_add_v2(float* dst, float a, float b) {
@@ -632,6 +636,9 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
       }
       if (tid == 0)  // fill: stages 0 .. kGBufs - 2
         for (int st = 0; st < min(kGBufs - 1, nst); ++st)
+#ifdef MSB_INSTRUMENTED
+          if (!(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0))
+#endif
           gather_issue(buf0 + st * bstride, records, s_run, e, st * CH, min(CH, nrun - st * CH), d, I,
                        s_list[st], &bar[st]);
       __syncthreads();  // s_tok, the fill's lists
@@ -665,10 +672,10 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
           gather_issue(buf0 + bn * bstride, records, s_run, e, sn * CH, min(CH, nrun - sn * CH), d, I,
                        s_list[bn], &bar[bn]);
         }
-        const bool okw = mbar_wait(&bar[b], (phases >> b) & 1u, ws.err);
+        const bool okw = mbar_wait(&bar[b], (phases >> b) & 1u, ws.err, cfg.wait_ns);
         if (!__syncthreads_and(okw)) {  // sticky error set; let copies in flight land
           for (int q = stg; q < min(nst, stg + kGBufs); ++q)
-            mbar_wait(&bar[q % kGBufs], (phases >> (q % kGBufs)) & 1u, ws.err);
+            mbar_wait(&bar[q % kGBufs], (phases >> (q % kGBufs)) & 1u, ws.err, cfg.wait_ns);
           ok = false;
           break;
         }
@@ -879,6 +886,11 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   cfg.ch = max(1, min(kGCh, (196 * 1024 / kGBufs) / (6 * d + 16)));
   cfg.nlr = D.rank > 0 ? (d + kLrRows - 1) / kLrRows : 0;
   cfg.dense = dense;
+  cfg.wait_ns = kWaitLimitNs;
+#ifdef MSB_INSTRUMENTED
+  cfg.skip = debug_ctl().skip;
+  if (debug_ctl().wait_ns) cfg.wait_ns = debug_ctl().wait_ns;
+#endif
   // persistent CTAs, one per SM, taking work items (runs of union channels, then
   // low-rank row blocks) off a counter
   const int ngrid = sm_count();

@@ -15,6 +15,19 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
                    const Workspace& ws, const TraceDev& tr, cudaStream_t st);
 int general_set_smem_limits();
 
+#ifdef MSB_INSTRUMENTED
+// Test and profiling controls of the instrumented build (libmsb_instr.so); the product
+// library is compiled without them.
+struct DebugCtl {
+  unsigned long long* marks;  // phase marks of the single-launch kernel ([grid][16]), or null
+  uint32_t skip;              // 1: the single-launch kernel's first CTA never issues its first
+                              //    record copy; 2: the gather CTA of work item 0 never issues
+                              //    its first stage -- so that a bounded wait runs out
+  uint64_t wait_ns;           // bounded-wait limit (0: the product's)
+};
+DebugCtl& debug_ctl();
+#endif
+
 // Residual add + RMSNorm glue between stacked layers.
 int launch_residual_rmsnorm(float* h, const uint16_t* y, uint16_t* x_next, int B, int d, float eps,
                             cudaStream_t st);

@@ -124,3 +124,21 @@ extern "C" int32_t moe_sparse_block_noalloc(const void* x, const void* router_t,
                               static_cast<uint16_t*>(out), D, err, counters, y_acc, tr, st);
   return rc == MSB_ENOTFUSED ? MSB_EUNSUPPORTED : rc;
 }
+
+// The kernel records a non-finite router logit, an expired bounded wait or a failed
+// consistency check in the array's first word; this reads it (and clears it) for the
+// caller, who has no workspace for msb_check to read.
+extern "C" int32_t msb_noalloc_check(void* stream) {
+  int status = MSB_OK;
+  unsigned char* base = static_cast<unsigned char*>(scratch_address(&status));
+  if (!base) return status;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t err = 0;
+  if (cudaMemcpyAsync(&err, base, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MSB_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MSB_ECUDA;
+  if (err == 0) return MSB_OK;
+  if (cudaMemsetAsync(base, 0, 4, st) != cudaSuccess) return MSB_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MSB_ECUDA;
+  if (err & kErrInternal) return MSB_EINTERNAL;
+  return (err & kErrTimeout) ? MSB_ETIMEOUT : MSB_ENONFINITE;
+}
