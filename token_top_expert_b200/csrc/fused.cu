@@ -52,10 +52,12 @@ constexpr int kSelShift = 15;
 constexpr int kCandMax = 64;           // keys of the k-th key's bin ranked directly
 constexpr int kWordsMax = (MSB_MAX_INTER + 31) / 32;
 constexpr int kMyselMax = 512;         // channels one CTA reads at most
-constexpr int kMarks = 16;             // phase marks per CTA (instrumented builds)
+#ifdef MSB_INSTRUMENTED
+constexpr int kMarks = 16;             // phase marks per CTA
+#endif
 
 // mbarriers: fixed ones, then one per record slot
-enum { kBarRows = 0, kBarX, kBarLogits, kBarSketch, kBarLow, kBarScores, kBarZ, kBarY, kBarRing };
+enum { kBarRows = 0, kBarX, kBarLogits, kBarIds, kBarSketch, kBarLow, kBarScores, kBarZ, kBarY, kBarRing };
 
 struct FusedParams {
   const uint16_t* x;
@@ -95,10 +97,10 @@ struct FusedParams {
 
 struct Misc {
   uint64_t bar[kBarRing + kRingMax];
-  int ids[MSB_MAX_TOP_E];
-  float lv[MSB_MAX_TOP_E];  // routed logits in rank order
+  uint2 rk[MSB_MAX_TOP_E];  // routed experts in rank order: (expert id, logit bits), pushed
+                            // by the CTA that owns the expert's router row
   float wk[MSB_MAX_TOP_E];  // combine weights of the routed experts, rank order
-  uint32_t tie, cmax, kb, rem, cnt, ccount, kth, need;
+  uint32_t cmax, kb, rem, cnt, ccount, kth, need;
   uint32_t info[2];
   uint32_t wt[kFW];
   float red8[kFW][8];    // per-warp sums of up to 8 dot products (logits; gate/up of a batch)
@@ -113,7 +115,8 @@ struct Misc {
 
 // the kernel's dynamic shared memory (carved up by the offsets in FusedParams)
 extern __shared__ __align__(128) uint8_t g_sm[];
-// this CTA's share of the selected channels (positions [c0, c1) of the ascending list)
+// this CTA's share of the selected channels (positions q, q + cs, q + 2 cs, ... of the
+// ascending list)
 #define MYSEL(P) reinterpret_cast<uint16_t*>(g_sm + (P).o_mysel)
 
 // ---------------------------------------------------------------- cluster PTX
@@ -134,6 +137,11 @@ __device__ __forceinline__ void st_async(uint32_t ra, uint32_t v, uint32_t rbar)
                "r"(v), "r"(rbar)
                : "memory");
 }
+__device__ __forceinline__ void st_async2(uint32_t ra, uint32_t a, uint32_t b, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1,%2}, [%3];" ::"r"(ra),
+               "r"(a), "r"(b), "r"(rbar)
+               : "memory");
+}
 __device__ __forceinline__ void st_async4(uint32_t ra, float a, float b, float c, float d, uint32_t rbar) {
   asm volatile(
       "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(ra),
@@ -151,8 +159,19 @@ __device__ __forceinline__ void red_async_max(uint32_t ra, uint32_t v, uint32_t 
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
+// arrive without release semantics: orders nothing, only counts (the exchanges it follows
+// are each tracked by the receiver's own mbarrier)
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// atomic add with acquire-release semantics at GPU scope; returns the old value
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -179,76 +198,50 @@ __device__ __noinline__ bool wait_slow(uint64_t* bar, uint32_t parity, uint32_t*
 #define wait_phase(bar, parity, err) \
   (mbar_try_wait((bar), (parity)) || wait_slow((bar), (parity), (err), WAIT_LIMIT))
 
-// Router top-K, exact pass: rank = #{e' : l_e' > l_e} + #{e' < e : l_e' == l_e} (ties
-// to the lower index), one thread per logit.  Rare (taken after a tie among the top K).
-// Ends with a barrier.
-__device__ __noinline__ void router_rank_exact(const float* logits, int E, int K, Misc& M) {
-  if (threadIdx.x < K) M.ids[threadIdx.x] = -1;
-  __syncthreads();
+// Order-preserving key of a logit: integer order is value order, -0 equals +0, and a
+// NaN ranks below everything.
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t b = __float_as_uint(v);
+  if (v != v) return 0u;
+  if (b == 0x80000000u) b = 0u;
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Router top-K, distributed over the cluster: the CTA that owns router rows [e_lo, e_hi)
+// ranks each of its logits exactly against all E (rank = #{e' : l_e' > l_e} + #{e' < e :
+// l_e' == l_e}, one warp per logit, one ballot per 32 logits) and, for a rank r < K,
+// pushes (e, l_e) into slot r of every CTA's M.rk.  The ranks form a permutation of 0..E-1,
+// so every CTA receives exactly K pushes.  A non-finite logit flags the call.
+__device__ __forceinline__ void router_rank(const FusedParams& P, const float* logits, int q) {
+  Misc& M = *reinterpret_cast<Misc*>(g_sm + P.o_misc);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = P.D.experts, K = P.D.top_e;
+  const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
+  const uint32_t rbar = smem_addr(&M.bar[kBarIds]);
 #pragma unroll 1
-  for (int ee = threadIdx.x; ee < E; ee += kFT) {
+  for (int ee = e_lo + warp; ee < e_hi; ee += kFW) {
     const float v = logits[ee];
-    int r = 0;
-#pragma unroll 1
-    for (int j = 0; j < E; ++j) {
-      const float u = logits[j];
-      r += (u > v) || (u == v && j < ee);
-    }
-    if (r < K) {
-      M.ids[r] = ee;
-      M.lv[r] = v;
-    }
-  }
-  __syncthreads();
-}
-
-// Router top-K over the E logits in shared memory (padded with -inf to Epad, a
-// multiple of 64), by rank counting, P = 256/E threads per logit (at most 4) on
-// 16-value vector steps: rank = #{e' : l_e' > l_e}; the owner of rank j < K claims
-// slot j.  Without ties among the top K every claim lands in its own slot and these
-// ranks are exact; two logits with the same value have the same count, so a tie shows
-// as a second claim on one slot, and then the exact pass runs.  M.ids must be -1 and
-// M.tie 0 on entry.  Ends with a barrier.
-__device__ __noinline__ void router_rank(const float* logits, int E, int Epad, int K, Misc& M,
-                                         uint32_t* err) {
-  const int tid = threadIdx.x;
-  const int lgP = E <= 64 ? 2 : (E <= 128 ? 1 : 0);
-  const int span = Epad >> lgP;
-#pragma unroll 1
-  for (int base = 0; base < (E << lgP); base += kFT) {
-    const int item = base + tid, ee = item >> lgP, h = item & ((1 << lgP) - 1);
-    float gt = 0.f;
-    float v = 0.f;
-    if (ee < E) {
-      v = logits[ee];
-      if (!isfinite(v)) atomicOr(err, kErrNonFinite);
-      const float4* lp = reinterpret_cast<const float4*>(logits + h * span);
+    const uint32_t kv = logit_key(v);
+    uint32_t rank = 0;
 #pragma unroll 4
-      for (int c = 0; c < span / 4; ++c) {
-        const float4 u = lp[c];
-        gt += (u.x > v ? 1.f : 0.f) + (u.y > v ? 1.f : 0.f);
-        gt += (u.z > v ? 1.f : 0.f) + (u.w > v ? 1.f : 0.f);
-      }
+    for (int j0 = 0; j0 < E; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t ku = j < E ? logit_key(logits[j]) : 0u;
+      rank += (uint32_t)__popc(__ballot_sync(0xffffffffu, j < E && (ku > kv || (ku == kv && j < ee))));
     }
-    if (lgP >= 1) gt += __shfl_xor_sync(0xffffffffu, gt, 1);
-    if (lgP >= 2) gt += __shfl_xor_sync(0xffffffffu, gt, 2);
-    const int rank = (int)gt;
-    if (ee < E && h == 0 && rank < K) {
-      if (atomicCAS(&M.ids[rank], -1, ee) != -1) M.tie = 1u;
-      M.lv[rank] = v;
-    }
+    if (lane == 0 && !isfinite(v)) atomicOr(P.err, kErrNonFinite);
+    if (rank < (uint32_t)K && lane < P.cs)
+      st_async2(mapa(smem_addr(&M.rk[rank]), lane), (uint32_t)ee, __float_as_uint(v), mapa(rbar, lane));
   }
-  __syncthreads();
-  if (M.tie) router_rank_exact(logits, E, K, M);
 }
 
-// Warp 0, after router_rank: the combine weights of the K routed experts into M.wk
+// Warp 0, after the routing: the combine weights of the K routed experts into M.wk
 // (rank order): softmax over the K routed logits (renorm) or over all E logits.
-// lv[0] is the largest logit.
+// rk[0] holds the largest logit.
 __device__ __noinline__ void router_weights(const float* logits, int E, int K, int renorm, Misc& M) {
   const int lane = threadIdx.x & 31;
-  const float mx = M.lv[0];
-  const float pl = lane < K ? __expf(M.lv[lane] - mx) : 0.f;
+  const float mx = __uint_as_float(M.rk[0].y);
+  const float pl = lane < K ? __expf(__uint_as_float(M.rk[lane].y) - mx) : 0.f;
   float denom = 0.f;
   if (renorm) {
     denom = pl;
@@ -263,14 +256,14 @@ __device__ __noinline__ void router_weights(const float* logits, int E, int K, i
 // Trace of the routing (one CTA): expert ids, weights, and the channels read per expert.
 __device__ __noinline__ void trace_routing(const TraceDev& tr, const Misc& M, int E, int K, int k) {
   const int tid = threadIdx.x;
-  if (tid < K && tr.expert_ids) tr.expert_ids[tid] = M.ids[tid] < 0 ? tid : M.ids[tid];
+  if (tid < K && tr.expert_ids) tr.expert_ids[tid] = (int)M.rk[tid].x;
   if (tid < K && tr.expert_w) tr.expert_w[tid] = M.wk[tid];
   if (tr.union_count)
 #pragma unroll 1
     for (int i = tid; i < E; i += kFT) {
       int c = 0;
 #pragma unroll 1
-      for (int j = 0; j < K; ++j) c = (M.ids[j] == i) ? k : c;  // (-1 never matches)
+      for (int j = 0; j < K; ++j) c = ((int)M.rk[j].x == i) ? k : c;
       tr.union_count[i] = c;
     }
 }
@@ -350,138 +343,141 @@ __device__ __noinline__ void select_fallback(const uint32_t* keys, int n, int k,
   __syncthreads();
 }
 
+// Exclusive prefix over the warp of v (v < 2^NB) by bit-sliced ballots: no shuffle chain.
+template <int NB>
+__device__ __forceinline__ uint32_t warp_excl_prefix(uint32_t v) {
+  const uint32_t lt = (1u << (threadIdx.x & 31)) - 1u;
+  uint32_t pre = 0;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) pre += (uint32_t)__popc(__ballot_sync(0xffffffffu, (v >> b) & 1u) & lt) << b;
+  return pre;
+}
+
 // Exact top-k of the n channel keys (float bits of non-negative scores, so integer
 // order is value order), ties to the lower index, as a bitmap M.selw over the
 // channels.  Keys are binned by (maxkey - key) >> 15 (256 bins per octave below the
-// largest key, bin 0 the largest, the last bin catching the rest): one counting
-// pass and one scan find the bin of the k-th key, whose keys are then ranked
-// directly.  hist (kSelBins words), M.csel and M.ccount must be zero on entry.
+// largest key, bin 0 the largest, the last bin catching the rest); one counting pass,
+// per-warp bin totals and a ballot prefix find the bin of the k-th key.  If that bin
+// is taken whole the bitmap is one ballot per word; otherwise its keys are ranked
+// directly (ties to the lower index).  Key j is read by thread j % 256, so a warp's
+// ballot over one stride of 256 keys is one bitmap word.  hist (kSelBins words), M.csel
+// and M.ccount must be zero on entry.  Ends with a barrier.
 __device__ __noinline__ void select_topk(const uint32_t* keys, int n, int k, uint32_t maxkey,
                                          uint32_t* hist, Misc& M) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 #pragma unroll 1
   for (int j = tid; j < n; j += kFT) atomicAdd(&hist[sel_bin(maxkey, keys[j])], 1u);
   __syncthreads();
-  // thread t owns bins [8t, 8t + 8): find the bin holding the k-th largest key
+  // thread t owns bins [8t, 8t + 8): warp totals, then the warp and lane of the k-th key
   const uint4 h0 = reinterpret_cast<const uint4*>(hist)[2 * tid];
   const uint4 h1 = reinterpret_cast<const uint4*>(hist)[2 * tid + 1];
-  const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  uint32_t local = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) local += c[i];
-  uint32_t incl = local;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += t;
-  }
-  if (lane == 31) M.wt[warp] = incl;
+  const uint32_t local = ((h0.x + h0.y) + (h0.z + h0.w)) + ((h1.x + h1.y) + (h1.z + h1.w));
+  const uint32_t wtot = __reduce_add_sync(0xffffffffu, local);
+  if (lane == 0) M.wt[warp] = wtot;
   __syncthreads();
-  uint32_t above = incl - local;
+  uint32_t above = 0;
 #pragma unroll
   for (int w = 0; w < kFW; ++w) above += w < warp ? M.wt[w] : 0u;
   const uint32_t kk = (uint32_t)k;
-  if (above < kk && kk <= above + local) {
+  if (above < kk && kk <= above + wtot) {  // (warp-uniform)
+    above += warp_excl_prefix<13>(local);  // local <= n <= 4096
+    if (above < kk && kk <= above + local) {
+      const uint32_t c[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (above < kk && kk <= above + c[i]) { M.kb = 8 * tid + i; M.rem = kk - above; M.cnt = c[i]; }
-      above += c[i];
-    }
-  }
-  __syncthreads();
-  const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
-  if (cnt > (uint32_t)kCandMax) {
-    select_fallback(keys, n, k, hist, M);
-    return;
-  }
-  // gather the keys of bin kb with their indices (warp-aggregated slots)
-  const uint32_t lt = (1u << lane) - 1u;
-#pragma unroll 1
-  for (int j0 = warp * 32; j0 < n; j0 += kFT) {
-    const int j = j0 + lane;
-    const uint32_t key = j < n ? keys[j] : 0u;
-    const bool m = j < n && sel_bin(maxkey, key) == kb;
-    const uint32_t mb = __ballot_sync(0xffffffffu, m);
-    if (mb) {
-      const int leader = __ffs(mb) - 1;
-      uint32_t slot0 = 0;
-      if (lane == leader) slot0 = atomicAdd(&M.ccount, (uint32_t)__popc(mb));
-      slot0 = __shfl_sync(0xffffffffu, slot0, leader) + __popc(mb & lt);
-      if (m) {
-        M.ck[slot0] = key;
-        M.ci[slot0] = (uint32_t)j;
+      for (int i = 0; i < 8; ++i) {
+        if (above < kk && kk <= above + c[i]) { M.kb = 8 * tid + i; M.rem = kk - above; M.cnt = c[i]; }
+        above += c[i];
       }
     }
   }
   __syncthreads();
-  // rank inside the bin by (key desc, index asc); the first `rem` are selected
-  if (tid < (int)cnt) {
-    const uint32_t mk = M.ck[tid], mi = M.ci[tid];
-    uint32_t rank = 0;
-#pragma unroll 4
-    for (int i = 0; i < (int)cnt; ++i) {
-      const uint32_t ok_ = M.ck[i];
-      rank += (ok_ > mk) || (ok_ == mk && M.ci[i] < mi);
+  const uint32_t kb = M.kb, rem = M.rem, cnt = M.cnt;
+  const bool whole = (cnt == rem);
+  if (!whole) {
+    if (cnt > (uint32_t)kCandMax) {
+      select_fallback(keys, n, k, hist, M);
+      return;
     }
-    if (rank < rem) atomicOr(&M.csel[mi >> 5], 1u << (mi & 31));
-  }
-  __syncthreads();
-  // selection bitmap: keys of higher bins, plus the selected keys of bin kb
+    // the keys of bin kb with their indices (warp-aggregated slots), each ranked among
+    // them by (key desc, index asc); the first `rem` are taken
+    const uint32_t lt = (1u << lane) - 1u;
 #pragma unroll 1
-  for (int cw = warp; cw < (n + 31) / 32; cw += kFW) {
-    const int j = 32 * cw + lane;
-    const uint32_t key = j < n ? keys[j] : 0u;
-    const uint32_t w = __ballot_sync(0xffffffffu, j < n && sel_bin(maxkey, key) < kb);
-    if (lane == 0) M.selw[cw] = w | M.csel[cw];
+    for (int j0 = warp * 32; j0 < n; j0 += kFT) {
+      const int j = j0 + lane;
+      const uint32_t key = j < n ? keys[j] : 0u;
+      const bool m = j < n && sel_bin(maxkey, key) == kb;
+      const uint32_t mb = __ballot_sync(0xffffffffu, m);
+      if (mb) {
+        const int leader = __ffs(mb) - 1;
+        uint32_t slot0 = 0;
+        if (lane == leader) slot0 = atomicAdd(&M.ccount, (uint32_t)__popc(mb));
+        slot0 = __shfl_sync(0xffffffffu, slot0, leader) + __popc(mb & lt);
+        if (m) {
+          M.ck[slot0] = key;
+          M.ci[slot0] = (uint32_t)j;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < (int)cnt) {
+      const uint32_t mk = M.ck[tid], mi = M.ci[tid];
+      uint32_t rank = 0;
+#pragma unroll 1
+      for (int i = 0; i < (int)cnt; ++i) {
+        const uint32_t ok_ = M.ck[i];
+        rank += (ok_ > mk) || (ok_ == mk && M.ci[i] < mi);
+      }
+      if (rank < rem) atomicOr(&M.csel[mi >> 5], 1u << (mi & 31));
+    }
+    __syncthreads();
+  }
+  // the bitmap: word 8 s + w is warp w's ballot over stride s
+#pragma unroll 1
+  for (int j0 = warp * 32; j0 < n; j0 += kFT) {
+    const int j = j0 + lane;
+    const uint32_t b = j < n ? sel_bin(maxkey, keys[j]) : 0xffffffffu;
+    const uint32_t w = __ballot_sync(0xffffffffu, b < kb || (whole && b == kb));
+    if (lane == 0) M.selw[j0 >> 5] = whole ? w : (w | M.csel[j0 >> 5]);
   }
   __syncthreads();
 }
 
-// Warp 0: exclusive prefix of the selection words' popcounts into M.pref, then the
-// channels at positions [c0, c0 + nmine) of the ascending selected list into
-// M.mysel.  nw <= 128 words.  A position the bitmap does not hold (a selection of
-// the wrong size) reads channel 0 and flags the call.
-__device__ __noinline__ void positions(int nw, int n, int c0, int nmine, Misc& M, uint16_t* mysel,
-                                      uint32_t* err) {
+// Warp 0: each selection word's exclusive prefix of popcounts into M.pref (ballot
+// prefix, 32 words at a time).  A selection of the wrong size (not k channels) flags the
+// call and fills this CTA's share with channel 0 (positions_place then overwrites what
+// it can).
+__device__ __noinline__ void positions_prefix(int nw, int k, int nmine, Misc& M, uint16_t* mysel, uint32_t* err) {
   const int lane = threadIdx.x & 31;
-  // exclusive prefix over the words, 32 at a time (nw <= 128)
   uint32_t carry = 0;
 #pragma unroll 1
-  for (int c0w = 0; c0w < nw; c0w += 32) {
-    const int c = c0w + lane;
+  for (int cb = 0; cb < nw; cb += 32) {
+    const int c = cb + lane;
     const uint32_t cnt = c < nw ? (uint32_t)__popc(M.selw[c]) : 0u;
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    if (c < nw) M.pref[c] = carry + incl - cnt;
-    carry += __shfl_sync(0xffffffffu, incl, 31);
+    const uint32_t p = carry + warp_excl_prefix<6>(cnt);
+    if (c < nw) M.pref[c] = p;
+    carry = __shfl_sync(0xffffffffu, p + cnt, 31);
   }
-  __syncwarp();
+  if (carry != (uint32_t)k) {
 #pragma unroll 1
-  for (int t = lane; t < nmine; t += 32) {
-    const uint32_t p = (uint32_t)(c0 + t);
-    int lo = 0, hi = nw - 1;  // largest c with pref[c] <= p
-#pragma unroll 1
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if (M.pref[mid] <= p) lo = mid; else hi = mid - 1;
-    }
-    // the (p - pref + 1)-th set bit of the word
-    uint32_t w = M.selw[lo];
-#pragma unroll 1
-    for (uint32_t i = M.pref[lo]; i < p; ++i) w &= w - 1u;
-    const uint32_t bit = w ? (uint32_t)(__ffs(w) - 1) : 32u;
-    int ch = 32 * lo + (int)bit;
-    if (bit > 31u || ch >= n) {
-      ch = 0;
-      atomicOr(err, kErrInternal);
-    }
-    mysel[t] = (uint16_t)ch;
+    for (int t = lane; t < nmine; t += 32) mysel[t] = 0;
+    if (lane == 0) atomicOr(err, kErrInternal);
   }
-  __syncwarp();
+}
+
+// All threads, after positions_prefix and a barrier: this CTA's share of the ascending
+// selected list into mysel -- the channels at positions p = q + t * 2^lgcs (t < nmine),
+// so that the CTAs of the cluster interleave over the list.  Thread j % 256 places
+// channel j: its position is its word's prefix plus the set bits below it.
+__device__ __forceinline__ void positions_place(int n, int q, int lgcs, int nmine, const Misc& M, uint16_t* mysel) {
+  const uint32_t cm = (1u << lgcs) - 1u;
+#pragma unroll 1
+  for (int j = threadIdx.x; j < n; j += kFT) {
+    const uint32_t w = M.selw[j >> 5], bit = 1u << (j & 31);
+    if (w & bit) {
+      const uint32_t p = M.pref[j >> 5] + (uint32_t)__popc(w & (bit - 1u));
+      if ((p & cm) == (uint32_t)q && (p >> lgcs) < (uint32_t)nmine) mysel[p >> lgcs] = (uint16_t)j;
+    }
+  }
 }
 
 // Warp 0 of one CTA per cluster: the expert's whole ascending selected list (k entries)
@@ -587,25 +583,6 @@ __device__ __forceinline__ void push_scores(const FusedParams& P, Misc& M, const
   }
 }
 
-// z rows of this CTA: z[q + i*CS] = B_e[q + i*CS] . x (rows staged in shared memory,
-// one warp per row), pushed to every CTA of the cluster.
-__device__ __forceinline__ void push_z(const FusedParams& P, Misc& M, const uint16_t* brows,
-                                    const uint16_t* xs, int q, int nz) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, CS = P.cs;
-  const int d = P.D.d;
-  const uint32_t rbar_z = smem_addr(&M.bar[kBarZ]);
-#pragma unroll 1
-  for (int i = warp; i < nz; i += kFW) {
-    const uint4* br = reinterpret_cast<const uint4*>(brows + (size_t)i * d);
-    const uint4* xv = reinterpret_cast<const uint4*>(xs);
-    float acc = 0.f;
-#pragma unroll 2
-    for (int j = lane; j < d / 8; j += 32) acc = dot8(br[j], xv[j], acc);
-    acc = warp_sum(acc);
-    if (lane < CS) st_async(mapa(smem_addr(&M.z[q + i * CS]), lane), __float_as_uint(acc), mapa(rbar_z, lane));
-  }
-}
-
 // After a wait of this CTA ran out: wait (bounded) for every barrier whose bytes may
 // still be landing -- the copies into this CTA and the other CTAs' pushes -- so that
 // nothing lands in its shared memory after it has exited.
@@ -653,8 +630,8 @@ __device__ __forceinline__ void phase_prologue(const FusedParams& P, int q) {
   if (tid == 0) {
 #pragma unroll 1
     for (int i = 0; i < kBarRing + P.ring; ++i) mbar_init(&M.bar[i], 1);
+
     M.cmax = 0u;
-    M.tie = 0u;
     M.ccount = 0u;
     fence_mbar_init();
     const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
@@ -665,11 +642,11 @@ __device__ __forceinline__ void phase_prologue(const FusedParams& P, int q) {
       bulk_g2s(rows + (size_t)j * P.rrs, P.router_t + (size_t)(e_lo + j) * d, 2u * d, &M.bar[kBarRows]);
     // bytes the other CTAs will push into this one
     mbar_arrive_expect_tx(&M.bar[kBarLogits], P.x1_bytes);
+    mbar_arrive_expect_tx(&M.bar[kBarIds], 8u * (uint32_t)P.D.top_e);
     mbar_arrive_expect_tx(&M.bar[kBarScores], P.sc_bytes);
     mbar_arrive_expect_tx(&M.bar[kBarZ], P.z_bytes);
     mbar_arrive_expect_tx(&M.bar[kBarY], P.y_bytes);
   }
-  if (tid < MSB_MAX_TOP_E) M.ids[tid] = -1;
   if (tid < kWordsMax) M.csel[tid] = 0u;
 
   float* logits = in_big<float>(P, P.o_logits);
@@ -715,12 +692,11 @@ __device__ __forceinline__ float dot8xf(uint4 a, const float (&xf)[8], float acc
 
 // A: logits of this CTA's router rows, 8 rows at a time (each thread its 8-element
 // groups of every row, one transposed warp reduction, the warps' sums in shared memory),
-// pushed to every CTA of the cluster; the x permutation for scoring.  Returns ok.
+// pushed to every CTA of the cluster.  Returns ok.
 template <int IT>
 __device__ __forceinline__ bool phase_router(const FusedParams& P, int q, bool ok, const float (&xf)[IT][8]) {
   Misc& M = misc(P);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, d = P.D.d, E = P.D.experts;
-  const uint16_t* xs = in_big<uint16_t>(P, P.o_x);
   const int e_lo = min(E, q * P.rpc), e_hi = min(E, e_lo + P.rpc);
   const uint32_t rbar = smem_addr(&M.bar[kBarLogits]);
   const uint32_t la = smem_addr(in_big<float>(P, P.o_logits) + e_lo);
@@ -731,13 +707,18 @@ __device__ __forceinline__ bool phase_router(const FusedParams& P, int q, bool o
     float v[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) v[j] = 0.f;
+    // rows past nb repeat row nb - 1 (their sums are dropped), so that all eight loads
+    // issue together
 #pragma unroll
     for (int it = 0; it < IT; ++it) {
       const int el = (it * kFT + tid) * 8;
       if (el < d) {
+        uint4 a[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          if (j < nb) v[j] = dot8xf(*reinterpret_cast<const uint4*>(rows + (size_t)(r0 + j) * P.rrs + el), xf[it], v[j]);
+          a[j] = *reinterpret_cast<const uint4*>(rows + (size_t)(r0 + min(j, nb - 1)) * P.rrs + el);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = dot8xf(a[j], xf[it], v[j]);
       }
     }
     const float sw = warp_sum8(v);
@@ -752,15 +733,6 @@ __device__ __forceinline__ bool phase_router(const FusedParams& P, int q, bool o
         st_async(mapa(la + 4u * (r0 + tid), dst), __float_as_uint(acc), mapa(rbar, dst));
     }
     __syncthreads();
-  }
-  // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p
-  if (!P.dense) {
-    uint32_t* xperm = in_big<uint32_t>(P, P.o_xperm);
-#pragma unroll 1
-    for (int i = tid; i < d / 2; i += kFT) {
-      const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
-      xperm[i] = reinterpret_cast<const uint32_t*>(xs)[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
-    }
   }
   return wait_phase(&M.bar[kBarLogits], 0, P.err) && ok;
 }
@@ -790,15 +762,68 @@ __device__ __forceinline__ void issue_expert(const FusedParams& P, int e, int q,
   if (r > 0) prefetch_l2(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, 2u * P.slice * r);
 }
 
-// B: sketch scores of this CTA's rows on the tensor cores, pushed with the warps'
-// largest keys; z = B_e x rows, pushed.  Returns ok.
+// z entries of this CTA: z[q + i CS] = B_e[q + i CS] . x for i < nz, 8 rows at a time with
+// every thread on its 8-element groups (rows past the chunk repeat its last row, their
+// sums dropped), one transposed warp reduction, the warps' sums in shared memory; each
+// entry pushed to every CTA of the cluster.  Rows staged in shared memory at stride d.
+template <int IT>
+__device__ __forceinline__ void push_z(const FusedParams& P, int q, int nz, const float (&xf)[IT][8]) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, d = P.D.d, CS = P.cs;
+  const uint16_t* brows = in_big<const uint16_t>(P, P.o_brows);
+  const uint32_t rbar = smem_addr(&M.bar[kBarZ]);
+#pragma unroll 1
+  for (int r0 = 0; r0 < nz; r0 += 8) {
+    const int nb = min(8, nz - r0);
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = 0.f;
+#pragma unroll
+    for (int it = 0; it < IT; ++it) {
+      const int el = (it * kFT + tid) * 8;
+      if (el < d) {
+        uint4 a[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a[j] = *reinterpret_cast<const uint4*>(brows + (size_t)(r0 + min(j, nb - 1)) * d + el);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = dot8xf(a[j], xf[it], v[j]);
+      }
+    }
+    const float sw = warp_sum8(v);
+    if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
+    __syncthreads();
+    if (tid < nb) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFW; ++w) acc += M.red8[w][tid];
+      const uint32_t za = smem_addr(&M.z[q + (r0 + tid) * CS]);
+#pragma unroll 1
+      for (int dst = 0; dst < CS; ++dst) st_async(mapa(za, dst), __float_as_uint(acc), mapa(rbar, dst));
+    }
+    __syncthreads();
+  }
+}
+
+// B: the x permutation for scoring; sketch scores of this CTA's rows on the tensor
+// cores, pushed with the warps' largest keys; then z = B_e x rows, pushed.  Returns ok.
+template <int IT>
 __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc, int nt, int lt0, int nz,
-                                          bool ok) {
+                                          bool ok, const float (&xf)[IT][8]) {
   Misc& M = misc(P);
   const int warp = threadIdx.x >> 5, KC = P.D.d / kColChunk;
   float* part = in_big<float>(P, P.o_part);
   if (!P.dense) {
+    // xperm[kc][c][s][p] = the bf16 pair of x at column 64*kc + 16*s + 2*c + 8*p (built
+    // while the sketch tiles are in flight)
+    uint32_t* xperm = in_big<uint32_t>(P, P.o_xperm);
+    const uint32_t* x32 = in_big<const uint32_t>(P, P.o_x);
+#pragma unroll 1
+    for (int i = threadIdx.x; i < P.D.d / 2; i += kFT) {
+      const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
+      xperm[i] = x32[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
+    }
     ok = wait_phase(&M.bar[kBarSketch], 0, P.err) && ok;
+    __syncthreads();  // xperm complete
     MARK(4);
     if (nt > 0)
       score_tiles(reinterpret_cast<const uint2*>(big_of(P)), in_big<const uint4>(P, P.o_xperm), nt, KC,
@@ -808,16 +833,17 @@ __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc
     push_scores(P, M, part, in_big<float>(P, P.o_alpha), in_big<uint32_t>(P, P.o_keys), nt * kRowTile, lt0,
                 rc, q);
   }
+  // z = B_e x while the scores cross the cluster (B_e rows landed long ago)
   if (nz > 0) {
     ok = wait_phase(&M.bar[kBarLow], 0, P.err) && ok;
-    push_z(P, M, in_big<uint16_t>(P, P.o_brows), in_big<uint16_t>(P, P.o_x), q, nz);
+    push_z<IT>(P, q, nz, xf);
   }
   return ok;
 }
 
 // C: exact top-k over the cluster's scores (or, dense, every channel) and this CTA's
 // share of it into M.mysel; then the first record copies.  Returns ok.
-__device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q, int rc, int nmine, int c0,
+__device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q, int rc, int nmine, int lgcs,
                                           bool ok) {
   Misc& M = misc(P);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, I = P.D.inter;
@@ -827,11 +853,14 @@ __device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q,
     MARK(7);
     select_topk(in_big<uint32_t>(P, P.o_keys), I, P.k, M.cmax, in_big<uint32_t>(P, P.o_hist), M);
     MARK(8);
-    if (warp == 0) positions(nw, I, c0, nmine, M, MYSEL(P), P.err);
+    if (warp == 0) positions_prefix(nw, P.k, nmine, M, MYSEL(P), P.err);
+    __syncthreads();
+    positions_place(I, q, lgcs, nmine, M, MYSEL(P));
+    __syncthreads();
   } else {
     if (warp == 0)
 #pragma unroll 1
-      for (int t = lane; t < nmine; t += 32) MYSEL(P)[t] = (uint16_t)(c0 + t);
+      for (int t = lane; t < nmine; t += 32) MYSEL(P)[t] = (uint16_t)(q + (t << lgcs));
     __syncthreads();  // (the dense path had no barrier since phase A: big is free now)
   }
   MARK(9);
@@ -887,23 +916,29 @@ __device__ __forceinline__ bool phase_records(const FusedParams& P, int e, int q
       if (ok) landed = i + nb;
     }
     {
-      // value 2j: gate_j . x, value 2j + 1: up_j . x (record j of the batch)
+      // value 2j: gate_j . x, value 2j + 1: up_j . x (record j of the batch; records past
+      // nb repeat record nb - 1, their sums dropped, so that all eight loads issue together)
       float v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      const uint16_t* rec[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (j < nb) {
-          const int sl = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
-          const uint16_t* rec = ring + (size_t)sl * P.rs;
+        const int jj = s0 + min(j, nb - 1);
+        rec[j] = ring + (size_t)(jj < P.ring ? jj : jj - P.ring) * P.rs;
+      }
 #pragma unroll
-          for (int it = 0; it < IT; ++it) {
-            const int el = (it * kFT + tid) * 8;
-            if (el < d) {
-              v[2 * j] = dot8xf(*reinterpret_cast<const uint4*>(rec + el), xf[it], v[2 * j]);
-              v[2 * j + 1] = dot8xf(*reinterpret_cast<const uint4*>(rec + d + el), xf[it], v[2 * j + 1]);
-            }
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kFT + tid) * 8;
+        if (el < d) {
+          uint4 a[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            a[2 * j] = *reinterpret_cast<const uint4*>(rec[j] + el);
+            a[2 * j + 1] = *reinterpret_cast<const uint4*>(rec[j] + d + el);
           }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = dot8xf(a[j], xf[it], v[j]);
         }
       }
       const float sw = warp_sum8(v);
@@ -930,20 +965,20 @@ __device__ __forceinline__ bool phase_records(const FusedParams& P, int e, int q
       M.h[tid] = __fdividef(g, 1.0f + __expf(-g)) * u;
     }
     __syncthreads();
-    // y += h_j * down_j over this thread's groups, two records at a time
+    // y += h_j * down_j over this thread's groups, two records at a time (a missing
+    // second record repeats the first with h = 0)
 #pragma unroll 1
     for (int j = 0; j < nb; j += 2) {
-      const int sa = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
-      const int sb = s0 + j + 1 < P.ring ? s0 + j + 1 : s0 + j + 1 - P.ring;
-      const uint16_t* reca = ring + (size_t)sa * P.rs + 2 * d;
-      const uint16_t* recb = ring + (size_t)sb * P.rs + 2 * d;
+      const int ja = s0 + j, jb = s0 + min(j + 1, nb - 1);
+      const uint16_t* reca = ring + (size_t)(ja < P.ring ? ja : ja - P.ring) * P.rs + 2 * d;
+      const uint16_t* recb = ring + (size_t)(jb < P.ring ? jb : jb - P.ring) * P.rs + 2 * d;
       const float ha = M.h[j], hb = j + 1 < nb ? M.h[j + 1] : 0.f;
 #pragma unroll
       for (int it = 0; it < IT; ++it) {
         const int el = (it * kFT + tid) * 8;
         if (el < d) {
           const uint4 va = *reinterpret_cast<const uint4*>(reca + el);
-          const uint4 vb = j + 1 < nb ? *reinterpret_cast<const uint4*>(recb + el) : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 vb = *reinterpret_cast<const uint4*>(recb + el);
           axpy8(y[it], ha, va);
           axpy8(y[it], hb, vb);
         }
@@ -999,12 +1034,10 @@ __device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int r
       red_add_v4(P.y_acc + q * P.slice + 4 * j, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
     }
   }
-  __threadfence();
+  // the CTA's reduction-adds precede (barrier, then the release of the counter's atomic)
+  // its count; the last contributor's acquire makes every other contribution visible
   __syncthreads();
-  if (tid == 0) {
-    M.last = (atomicAdd(P.slice_cnt + q, 1u) == (uint32_t)(K - 1));
-    if (M.last) __threadfence();
-  }
+  if (tid == 0) M.last = (atom_add_acq_rel_gpu(P.slice_cnt + q, 1u) == (uint32_t)(K - 1));
   __syncthreads();
   if (M.last) {
     // every contribution to this slice has arrived: convert, re-zero, reset
@@ -1063,11 +1096,12 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
 
   ok = phase_router<IT>(P, q, ok, xf);
   MARK(2);
-  router_rank(in_big<float>(P, P.o_logits), P.D.experts, P.epad, P.D.top_e, M, P.err);
-  int e = M.ids[rc];
-  if (e < 0) {  // a rank left empty (non-finite logits): keep a valid index, the call is flagged
+  router_rank(P, in_big<float>(P, P.o_logits), q);
+  ok = wait_phase(&M.bar[kBarIds], 0, P.err) && ok;
+  int e = (int)M.rk[rc].x;
+  if (e >= P.D.experts) {  // (only after an expired wait) keep a valid index; the call is flagged
     e = rc;
-    if (tid == 0) atomicOr(P.err, kErrNonFinite);
+    if (tid == 0) atomicOr(P.err, kErrInternal);
   }
   MARK(3);
   const int ntile_all = P.D.ipad / kRowTile;
@@ -1078,11 +1112,11 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
   // combine weights (warp 0; read in phase E, many barriers later)
   if (warp == 0) router_weights(in_big<float>(P, P.o_logits), P.D.experts, P.D.top_e, P.D.renorm, M);
 
-  ok = phase_scores(P, q, rc, nt, lt0, nz, ok);
+  ok = phase_scores<IT>(P, q, rc, nt, lt0, nz, ok, xf);
   MARK(6);
-  const int c0 = q * P.k / CS, c1 = (q + 1) * P.k / CS;
-  const int nmine = c1 - c0;
-  ok = phase_select(P, e, q, rc, nmine, c0, ok);
+  const int lgcs = CS == 16 ? 4 : 3;  // (the cluster size is 8 or 16)
+  const int nmine = P.k > q ? (P.k - q + CS - 1) >> lgcs : 0;
+  ok = phase_select(P, e, q, rc, nmine, lgcs, ok);
   // A_e z on this CTA's output slice while the first records fly (A_e from L2)
   if (r > 0) {
     ok = wait_phase(&M.bar[kBarZ], 0, P.err) && ok;
@@ -1091,7 +1125,10 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
   }
   MARK(10);
   ok = phase_records<IT>(P, e, q, nmine, ok, xf);
-  cluster_arrive();  // paired with the wait before exit: no CTA leaves while pushes may target it
+  // paired with the wait before exit: no CTA leaves before every CTA of the cluster has
+  // issued its pushes (each receiver waits for its own bytes; after an expired wait the
+  // quiesce below waits for them)
+  cluster_arrive_relaxed();
   __syncthreads();   // lr complete (a CTA may have had no records, hence no barrier since)
   ok = phase_combine(P, q, rc, ok);
   MARK(14);
