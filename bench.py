@@ -663,7 +663,10 @@ def main():
     oh = torch.empty_like(xh).pin_memory()
     ne = min(args.e2e_steps, args.steps)
     if args.top_e is None:
-        calls = [msb.HostCall(lay, args.k, B, stream=stream, general=general) for lay in layers]
+        # the host produces each step's x before the call (nothing on the stream writes
+        # it), so the calls declare it ready: the kernel fetches x across the host link
+        # while the previous launch still runs
+        calls = [msb.HostCall(lay, args.k, B, stream=stream, general=general, x_ready=True) for lay in layers]
         xp = [xh[i].data_ptr() for i in range(nseq)]
         op = [oh[i].data_ptr() for i in range(nseq)]
 

@@ -71,6 +71,11 @@ extern "C" {
 
 /* ------------------------------------------------------------------ flags */
 #define MSB_FLAG_GENERAL 1u    /* use the multi-kernel path even at B == 1 */
+#define MSB_FLAG_X_READY 2u    /* x is complete when the call is enqueued: nothing earlier on
+                                  the stream writes it (activations the host produced), so
+                                  the single-launch kernel may fetch it while the previous
+                                  launch on the stream still runs.  Wrong results if a
+                                  kernel or copy earlier on the stream does write x. */
 
 /* Block dimensions.  renorm = 1: the K kept router probabilities are rescaled
  * to sum to one; 0: they are used as they are. */
@@ -182,7 +187,7 @@ int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t f
  *  workspace, workspace_bytes: device scratch of at least
  *           msb_workspace_size(dims, batch) bytes, zero-filled before first use.
  *  trace    optional host struct of device pointers (NULL: no trace).
- *  flags    0 or MSB_FLAG_GENERAL.
+ *  flags    0, MSB_FLAG_GENERAL, MSB_FLAG_X_READY, or both.
  *  stream   cudaStream_t.
  * FP32 accumulation throughout; channel scores in FP32. */
 int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, const void* records,
@@ -206,11 +211,18 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
                                size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
                                void* stream);
 
-/* The block on activations in host memory: copies x_host to x_dev, runs
- * moe_sparse_block(x_dev -> out_dev) and copies out_dev to out_host, all enqueued on
- * `stream` with cudaMemcpyAsync (no synchronisation: the host buffers must stay
- * valid, and out_host unread, until the stream has passed the copies).  Use pinned
- * host memory (cudaHostAlloc / torch pin_memory) for asynchronous copies.
+/* The block on activations in host memory, everything enqueued on `stream` (no
+ * synchronisation: the host buffers must stay valid, and out_host unread, until the
+ * stream has passed the call).
+ *  - batch 1 on the single-launch path, with x_host and out_host pinned, mapped into
+ *    the current device's address space (cudaHostAlloc / torch pin_memory under
+ *    unified addressing) and 16-byte aligned: the kernel itself reads x_host and
+ *    writes out_host across
+ *    the host link, so consecutive calls keep their launch overlap; the staging
+ *    buffers are not touched.
+ *  - otherwise: copies x_host to x_dev, runs moe_sparse_block(x_dev -> out_dev) and
+ *    copies out_dev to out_host with cudaMemcpyAsync (pinned memory makes the copies
+ *    asynchronous).
  *  x_host, out_host  bf16 [batch][d] host memory, not overlapping each other.
  *  x_dev, out_dev    bf16 [batch][d] device staging buffers (as x and out of
  *                    moe_sparse_block: 16-byte aligned, not overlapping).

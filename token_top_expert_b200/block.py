@@ -358,9 +358,14 @@ class HostCall:
     The layer, k, batch, device staging buffers, workspace and stream are fixed and
     checked once, here; a call passes only the two host buffers (pinned host tensors of
     shape [batch][d], bf16), so the per-step cost on the host is one C call.  The call is
-    asynchronous: synchronise the stream before reading `out_host` or reusing `x_host`."""
+    asynchronous: synchronise the stream before reading `out_host` or reusing `x_host`.
 
-    def __init__(self, layer: PackedLayer, k: int, batch: int, stream=None, general: bool = False):
+    x_ready=True declares that nothing earlier on the stream writes x_host (the host
+    produced it before the call), so that the single-launch kernel fetches it while the
+    previous launch still runs (MSB_FLAG_X_READY)."""
+
+    def __init__(self, layer: PackedLayer, k: int, batch: int, stream=None, general: bool = False,
+                 x_ready: bool = False):
         import torch
         dims = layer.dims
         if not 1 <= k <= dims.inter:
@@ -377,8 +382,9 @@ class HostCall:
         self._head = (_ptr(self.x_dev), batch, _ptr(layer.router_t), _ptr(layer.records),
                       _ptr(layer.sketch), _ptr(layer.alpha), k, _ptr(layer.lr_a), _ptr(layer.lr_b),
                       _ptr(self.out_dev))
-        self._tail = (ctypes.byref(self._dims), self.workspace.ptr, self.workspace.nbytes,
-                      _lib.MSB_FLAG_GENERAL if general else 0, _stream(self.stream))
+        flags = (_lib.MSB_FLAG_GENERAL if general else 0) | (_lib.MSB_FLAG_X_READY if x_ready else 0)
+        self._tail = (ctypes.byref(self._dims), self.workspace.ptr, self.workspace.nbytes, flags,
+                      _stream(self.stream))
         self._layer = layer  # keep the weights alive
 
     def check_host(self, t):

@@ -178,7 +178,7 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
                  const uint32_t* sketch, const float* alpha, int32_t k, int mode, float tau,
                  const void* lr_a, const void* lr_b, void* out, const msb_dims* dims,
                  void* workspace, size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
-                 void* stream) {
+                 void* stream, bool x_mapped = false) {
   int rc = check_dims(dims);
   if (rc != MSB_OK) return rc;
   if (batch < 1) return MSB_EINVAL;
@@ -211,9 +211,10 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
   uint16_t* o = static_cast<uint16_t*>(out);
   if (mode == 0 && batch == 1 && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k)) {
     rc = launch_fused(xb, rt, rec, sketch, alpha, k, la, lb, o, D, ws.err, ws.counters, ws.y_acc,
-                      tr, st);
+                      tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0);
     if (rc != MSB_ENOTFUSED) return rc;
   }
+  if (x_mapped) return MSB_ENOTFUSED;  // the multi-kernel path takes device buffers only
   return launch_general(xb, batch, rt, rec, sketch, alpha, k, mode, tau, la, lb, o, D, ws, tr, st);
 }
 
@@ -300,6 +301,17 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
                       workspace, workspace_bytes, trace, flags, stream);
 }
 
+// Device address of pinned host memory that is mapped into the current device's address
+// space, or null (pageable memory, or not mapped).
+const void* mapped_address(const void* h) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, h) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
 int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, const void* router_t,
                               const void* records, const uint32_t* sketch, const float* alpha,
                               int32_t k, const void* lr_a, const void* lr_b, void* out_dev,
@@ -313,6 +325,17 @@ int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, co
   const size_t bytes = (size_t)batch * dims->d * 2;
   if (overlaps(x_host, bytes, out_host, bytes)) return MSB_EINVAL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // pinned, mapped host buffers on the single-launch path: the kernel itself reads x and
+  // writes the result across the host link (no copy-engine round trip between launches)
+  if (batch == 1 && !(flags & MSB_FLAG_GENERAL)) {
+    const void* xm = mapped_address(x_host);
+    void* om = const_cast<void*>(mapped_address(out_host));
+    if (xm && om && aligned16(xm) && aligned16(om)) {
+      rc = block_common(xm, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, om, dims,
+                        workspace, workspace_bytes, nullptr, flags, stream, true);
+      if (rc != MSB_ENOTFUSED) return rc;
+    }
+  }
   if (cudaMemcpyAsync(x_dev, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MSB_ECUDA;
   rc = block_common(x_dev, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out_dev,
                     dims, workspace, workspace_bytes, nullptr, flags, stream);

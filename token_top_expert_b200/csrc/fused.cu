@@ -93,6 +93,11 @@ struct FusedParams {
   int o_alpha, o_brows;                                  // inside big (phase B)
   int smem;
   uint32_t x1_bytes, sc_bytes, z_bytes, y_bytes;  // bytes each CTA expects per exchange
+  int x_ready;   // nothing earlier on the stream writes x: fetch it before the grid
+                 // dependency wait
+  int x_mapped;  // x and out are pinned host memory mapped into the device's address space:
+                 // each CTA reads its piece of x over the host link and pushes it to the
+                 // cluster; out is written across the link by the slices' last contributors
 };
 
 struct Misc {
@@ -172,6 +177,14 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v
   uint32_t old;
   asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
+}
+// 16-byte load that bypasses L1 (pinned host memory the host rewrites between calls:
+// a CTA never meets a line an earlier launch left in its SM); loads of a warp coalesce
+// into one transfer across the host link
+__device__ __forceinline__ uint4 ld_fresh16(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
 }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -1071,15 +1084,37 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
   __syncthreads();
   // barrier inits, cmax = 0 and the zero-fills above precede any remote access
   cluster_arrive();
-  // x and the accumulator may be written by the previous launch: wait for it here
-  pdl_wait();
-  pdl_trigger();  // the next launch may start its weight-only prologue
+  // x: one bulk copy, or (in mapped host memory) CTA q reads the q-th of CS equal pieces
+  // across the host link, one coalesced 16-byte load per thread, and pushes it to every
+  // CTA of the cluster once every CTA has initialised its barriers.  x and the
+  // accumulator may be written by the previous launch, so x is fetched after the grid
+  // dependency wait -- unless the caller declared x ready (nothing earlier on the stream
+  // writes it), in which case the fetch overlaps the previous launch.
   uint16_t* xs = in_big<uint16_t>(P, P.o_x);
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&M.bar[kBarX], 2u * d);
-    bulk_g2s(xs, P.x, 2u * d, &M.bar[kBarX]);
+  const int xv = d / (8 * CS);  // 16-byte vectors per piece
+  uint4 xpiece = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    if (pass == 1) {
+      pdl_wait();
+      pdl_trigger();  // the next launch may start its weight-only prologue
+    }
+    if (pass == (P.x_ready ? 0 : 1)) {
+      if (tid == 0) {
+        mbar_arrive_expect_tx(&M.bar[kBarX], 2u * d);
+        if (!P.x_mapped) bulk_g2s(xs, P.x, 2u * d, &M.bar[kBarX]);
+      }
+      if (P.x_mapped && tid < xv) xpiece = ld_fresh16(P.x + 8 * (q * xv + tid));
+      cluster_wait();  // every CTA of the cluster has initialised its barriers
+      if (P.x_mapped && tid < xv) {
+        const uint32_t la = smem_addr(xs + 8 * (q * xv + tid)), rb = smem_addr(&M.bar[kBarX]);
+#pragma unroll 1
+        for (int dst = 0; dst < CS; ++dst)
+          st_async4(mapa(la, dst), __uint_as_float(xpiece.x), __uint_as_float(xpiece.y),
+                    __uint_as_float(xpiece.z), __uint_as_float(xpiece.w), mapa(rb, dst));
+      }
+    }
   }
-  cluster_wait();  // every CTA of the cluster has initialised its barriers
   bool ok = wait_phase(&M.bar[kBarX], 0, P.err);
   ok = wait_phase(&M.bar[kBarRows], 0, P.err) && ok;
   MARK(1);
@@ -1329,8 +1364,11 @@ bool fused_supported(const Dims& D, int k) {
 int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* records,
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
                  const uint16_t* lr_b, uint16_t* out, const Dims& D, uint32_t* err,
-                 uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st) {
+                 uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st, bool x_mapped,
+                 bool x_ready) {
   FusedParams P{};
+  P.x_mapped = x_mapped ? 1 : 0;
+  P.x_ready = x_ready ? 1 : 0;
   P.x = x;
   P.router_t = router_t;
   P.records = records;

@@ -17,6 +17,7 @@ int fused_setup();
 int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* records,
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
                  const uint16_t* lr_b, uint16_t* out, const Dims& D, uint32_t* err,
-                 uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st);
+                 uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st,
+                 bool x_mapped = false, bool x_ready = false);
 
 }  // namespace msb

@@ -502,16 +502,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Issue the bulk copies of channels run[c0 .. c0 + n) (shared memory) into a stage buffer.
+// The stage's channel list into `list` and (copy) the bulk copies of its records.  The
+// list is always written: the consumer reads it whether or not the copies were issued.
 __device__ __forceinline__ void gather_issue(uint16_t* buf, const uint16_t* records, const int* run,
                                              int e, int c0, int n, int d, int I, int* list,
-                                             uint64_t* bar) {
+                                             uint64_t* bar, bool copy = true) {
   const int rs = 3 * d + 8;
-  fence_proxy_async();
-  mbar_arrive_expect_tx(bar, 6u * d * n);
+  if (copy) {
+    fence_proxy_async();
+    mbar_arrive_expect_tx(bar, 6u * d * n);
+  }
   for (int i = 0; i < n; ++i) {
     const int j = run[c0 + i];
     list[i] = j;
-    bulk_g2s(buf + (size_t)i * rs, records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
+    if (copy) bulk_g2s(buf + (size_t)i * rs, records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
   }
 }
 
@@ -635,12 +639,14 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
       }
       if (tid == 0)  // fill: stages 0 .. kGBufs - 2
-        for (int st = 0; st < min(kGBufs - 1, nst); ++st)
+        for (int st = 0; st < min(kGBufs - 1, nst); ++st) {
+          bool copy = true;
 #ifdef MSB_INSTRUMENTED
-          if (!(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0))
+          copy = !(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0);  // withhold the copies only
 #endif
           gather_issue(buf0 + st * bstride, records, s_run, e, st * CH, min(CH, nrun - st * CH), d, I,
-                       s_list[st], &bar[st]);
+                       s_list[st], &bar[st], copy);
+        }
       __syncthreads();  // s_tok, the fill's lists
       // B fragments (x of this lane's token g8) of this warp's k-steps
       uint32_t xb[KSW > 0 ? KSW : 1][2];
