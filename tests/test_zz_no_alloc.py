@@ -122,3 +122,22 @@ def test_noalloc_rejects_sizes_beyond_its_limit():
     rc = lib.moe_sparse_block_noalloc(fake, fake, fake, fake, fake, 138, fake, fake, fake * 2,
                                       ctypes.byref(big), None, None)
     assert rc == _lib.MSB_EUNSUPPORTED
+
+
+def test_noalloc_at_its_size_limit():
+    """d = MSB_NOALLOC_MAX_D = 8192: the static accumulator is used whole."""
+    msb = require_gpu()
+    import torch
+    from token_top_expert_b200 import _lib
+    lib = _lib.load()
+    w = synth.TINY.with_(name="wide_d8192_I512_E16_top4_k92_r16", d=8192, inter=512, experts=16,
+                         top_e=4, k=92, rank=16, seed=0x7E57 + 40)
+    dev = device_layer(w)
+    xb = synth.activations(w, 8)
+    x = to_bf16_tensor(xb)
+    out = torch.empty_like(x)
+    tr = msb.Trace(dev.dims, 1, w.k, scores=True)
+    assert call_noalloc(lib, x, dev, w.k, out, tr) == _lib.MSB_OK
+    torch.cuda.synchronize()
+    assert lib.msb_noalloc_check(torch.cuda.current_stream().cuda_stream) == _lib.MSB_OK
+    compare(xb, traced(tr, out), oracle.SynthLayer(w), w.top_e, w.k)
