@@ -70,7 +70,7 @@ extern "C" {
 #define MSB_MAX_BATCH 256      /* tokens per call B: 1..256 */
 
 /* ------------------------------------------------------------------ flags */
-#define MSB_FLAG_GENERAL 1u    /* use the multi-kernel path even at B == 1 */
+#define MSB_FLAG_GENERAL 1u    /* use the multi-kernel path at every batch size */
 #define MSB_FLAG_X_READY 2u    /* x is complete when the call is enqueued: nothing earlier on
                                   the stream writes it (activations the host produced), so
                                   the single-launch kernel may fetch it while the previous
@@ -160,7 +160,11 @@ int32_t msb_check(void* workspace, void* stream);
 const char* msb_strerror(int32_t status);
 
 /* Diagnostics: the path moe_sparse_block takes for these arguments on the
- * current device.  Fills info (host, 8 int32):
+ * current device.  Batches of up to 16 tokens run on the single-launch kernel
+ * when it fits (one cluster per (token, routed expert) pair, each pair reading
+ * its own k channels); larger batches, MSB_FLAG_GENERAL, and batches above 1
+ * whose trace asks for the per-expert union count take the multi-kernel path,
+ * which reads each expert's union of channels once.  Fills info (host, 8 int32):
  *   {path (1 = single launch, 2 = multi-kernel), cluster size, clusters per
  *    routed expert, channel-record ring slots, dynamic shared-memory bytes,
  *    resident 16-CTA clusters, resident 8-CTA clusters, 0}.

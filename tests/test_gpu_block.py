@@ -300,3 +300,31 @@ def test_workspace_reuse_across_batch_sizes(msb):
         for y in ys[1:]:
             assert np.linalg.norm(y - ys[0]) <= 1e-2 * np.linalg.norm(ys[0])
     assert np.linalg.norm(outs[1][0][0] - outs[16][0][0]) <= 1e-2 * np.linalg.norm(outs[1][0][0])
+
+
+# ------------------------------------------------------------------ small batches, one launch
+
+@pytest.mark.parametrize("workload,batch", [("qwen13", 2), ("qwen13", 4), ("qwen13", 16), ("tiny", 3)])
+def test_small_batch_single_launch(msb, workload, batch):
+    """Batches of up to 16 tokens on the single-launch kernel (one cluster per (token,
+    routed expert) pair): every token against the oracle; consecutive calls share the
+    workspace's accumulator and slice counters."""
+    import torch
+    from parity import from_bf16_tensor, to_bf16_tensor
+    w = synth.QWEN30B_BLOCK_13 if workload == "qwen13" else synth.TINY
+    dev = device_layer(w)
+    assert msb.path_info(dev.dims, batch, w.k)["path"] == "single_launch"
+    lay = oracle.SynthLayer(w)
+    ws = msb.Workspace(dev.dims, batch)
+    for step in range(2):
+        x = synth.activations(w, 60 + step, batch=batch)
+        tr = msb.Trace(dev.dims, batch, w.k, scores=True, union=False)
+        out = msb.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, trace=tr)
+        torch.cuda.synchronize()
+        ws.check()
+        g = {"y": oracle.bf16_to_f64(from_bf16_tensor(out)), "ids": tr.expert_ids.cpu().numpy(),
+             "w": tr.expert_w.cpu().numpy(), "sel": tr.sel.cpu().numpy().view(np.uint16),
+             "sel_count": tr.sel_count.cpu().numpy(), "union": None,
+             "scores": tr.scores.cpu().numpy()}
+        assert (g["sel_count"] == w.k).all()
+        print(batch, step, compare(x, g, lay, w.top_e, w.k))

@@ -202,7 +202,9 @@ class Trace:
     """Device buffers receiving a call's routing and selection."""
 
     def __init__(self, dims: Dims, batch: int, k: int, device="cuda", scores=False,
-                 threshold=False):
+                 threshold=False, union=True):
+        """union=False leaves out the per-expert union count (batches above 1 that trace it
+        take the multi-kernel path)."""
         import torch
         K = dims.top_e
         cap = dims.inter if threshold else k
@@ -210,7 +212,8 @@ class Trace:
         self.expert_w = torch.zeros((batch, K), dtype=torch.float32, device=device)
         self.sel = torch.zeros((batch, K, cap), dtype=torch.int16, device=device)
         self.sel_count = torch.zeros((batch, K), dtype=torch.int32, device=device)
-        self.union_count = torch.zeros((dims.experts,), dtype=torch.int32, device=device)
+        self.union_count = (torch.zeros((dims.experts,), dtype=torch.int32, device=device)
+                            if union else None)
         self.scores = (torch.zeros((batch, K, dims.ipad), dtype=torch.float32, device=device)
                        if scores else None)
 
@@ -274,7 +277,7 @@ def _check_call(x, layer: PackedLayer, out, trace, K: int, cap: int):
             raise ValueError("trace.%s is %s on %s; this call needs [>= %d]%s on %s"
                              % (name, tuple(t.shape), t.device, B, list(tail), dev))
     u = trace.union_count
-    if u.dim() != 1 or u.shape[0] < dims.experts or u.device != dev:
+    if u is not None and (u.dim() != 1 or u.shape[0] < dims.experts or u.device != dev):
         raise ValueError("trace.union_count needs >= %d entries on %s" % (dims.experts, dev))
 
 

@@ -209,9 +209,9 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
   const uint16_t* la = static_cast<const uint16_t*>(lr_a);
   const uint16_t* lb = static_cast<const uint16_t*>(lr_b);
   uint16_t* o = static_cast<uint16_t*>(out);
-  if (mode == 0 && batch == 1 && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k)) {
+  if (mode == 0 && batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k)) {
     rc = launch_fused(xb, rt, rec, sketch, alpha, k, la, lb, o, D, ws.err, ws.counters, ws.y_acc,
-                      tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0);
+                      tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0, batch);
     if (rc != MSB_ENOTFUSED) return rc;
   }
   if (x_mapped) return MSB_ENOTFUSED;  // the multi-kernel path takes device buffers only
@@ -366,8 +366,8 @@ int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t f
   if (rc != MSB_OK) return rc;
   const Dims D = to_dims(*dims);
   int p[6];
-  fused_plan_info(D, k, p);
-  const bool fused = batch == 1 && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k);
+  fused_plan_info(D, k, batch, p);
+  const bool fused = batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k);
   info[0] = fused ? 1 : 2;
   for (int i = 0; i < 6; ++i) info[1 + i] = p[i];
   info[7] = 0;

@@ -266,11 +266,14 @@ __device__ __noinline__ void router_weights(const float* logits, int E, int K, i
   if (lane < K) M.wk[lane] = __fdividef(pl, denom);
 }
 
-// Trace of the routing (one CTA): expert ids, weights, and the channels read per expert.
-__device__ __noinline__ void trace_routing(const TraceDev& tr, const Misc& M, int E, int K, int k) {
+// Trace of token tok's routing (one CTA): expert ids, weights, and the channels read per
+// expert.
+// (The per-expert union count is written for a single token; batches that trace it take
+// the multi-kernel path.)
+__device__ __noinline__ void trace_routing(const TraceDev& tr, const Misc& M, int E, int K, int k, int tok) {
   const int tid = threadIdx.x;
-  if (tid < K && tr.expert_ids) tr.expert_ids[tid] = (int)M.rk[tid].x;
-  if (tid < K && tr.expert_w) tr.expert_w[tid] = M.wk[tid];
+  if (tid < K && tr.expert_ids) tr.expert_ids[tok * K + tid] = (int)M.rk[tid].x;
+  if (tid < K && tr.expert_w) tr.expert_w[tok * K + tid] = M.wk[tid];
   if (tr.union_count)
 #pragma unroll 1
     for (int i = tid; i < E; i += kFT) {
@@ -493,8 +496,8 @@ __device__ __forceinline__ void positions_place(int n, int q, int lgcs, int nmin
   }
 }
 
-// Warp 0 of one CTA per cluster: the expert's whole ascending selected list (k entries)
-// and its size into the trace (dense: every channel).
+// Warp 0 of one CTA per cluster: the pair's whole ascending selected list (k entries)
+// and its size into trace row rc (dense: every channel).
 __device__ __noinline__ void trace_selection(const FusedParams& P, const Misc& M, int nw, int rc) {
   const int lane = threadIdx.x & 31, k = P.k;
   if (lane == 0 && P.tr.sel_count) P.tr.sel_count[rc] = k;
@@ -820,7 +823,7 @@ __device__ __forceinline__ void push_z(const FusedParams& P, int q, int nz, cons
 // B: the x permutation for scoring; sketch scores of this CTA's rows on the tensor
 // cores, pushed with the warps' largest keys; then z = B_e x rows, pushed.  Returns ok.
 template <int IT>
-__device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc, int nt, int lt0, int nz,
+__device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int pr, int nt, int lt0, int nz,
                                           bool ok, const float (&xf)[IT][8]) {
   Misc& M = misc(P);
   const int warp = threadIdx.x >> 5, KC = P.D.d / kColChunk;
@@ -844,7 +847,7 @@ __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc
     __syncthreads();
     MARK(5);
     push_scores(P, M, part, in_big<float>(P, P.o_alpha), in_big<uint32_t>(P, P.o_keys), nt * kRowTile, lt0,
-                rc, q);
+                pr, q);
   }
   // z = B_e x while the scores cross the cluster (B_e rows landed long ago)
   if (nz > 0) {
@@ -856,8 +859,8 @@ __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int rc
 
 // C: exact top-k over the cluster's scores (or, dense, every channel) and this CTA's
 // share of it into M.mysel; then the first record copies.  Returns ok.
-__device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q, int rc, int nmine, int lgcs,
-                                          bool ok) {
+__device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q, int pr, int tok, int nmine,
+                                          int lgcs, bool ok) {
   Misc& M = misc(P);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, I = P.D.inter;
   const int nw = (I + 31) / 32;
@@ -877,9 +880,9 @@ __device__ __forceinline__ bool phase_select(const FusedParams& P, int e, int q,
     __syncthreads();  // (the dense path had no barrier since phase A: big is free now)
   }
   MARK(9);
-  if (q == 0 && (P.tr.sel || P.tr.sel_count) && warp == 0) trace_selection(P, M, nw, rc);
-  if (blockIdx.x == 0 && (P.tr.expert_ids || P.tr.expert_w || P.tr.union_count))
-    trace_routing(P.tr, M, P.D.experts, P.D.top_e, P.k);
+  if (q == 0 && (P.tr.sel || P.tr.sel_count) && warp == 0) trace_selection(P, M, nw, pr);
+  if (q == 0 && pr == tok * P.D.top_e && (P.tr.expert_ids || P.tr.expert_w || P.tr.union_count))
+    trace_routing(P.tr, M, P.D.experts, P.D.top_e, P.k, tok);
   // the ring now takes over `big`: every thread is past its last use of phases A-C
   if (warp == 0 && ok) {
     fence_proxy_async();
@@ -1027,11 +1030,13 @@ __device__ __forceinline__ bool phase_records(const FusedParams& P, int e, int q
 // E: the owner of slice q sums the cluster's partials of it, adds A_e z, weights by
 // the router and reduction-adds into the FP32 accumulator; the last of the K
 // contributions converts the slice to BF16 and re-zeroes it.  Returns ok.
-__device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int rc, bool ok) {
+__device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int rc, int tok, bool ok) {
   Misc& M = misc(P);
   const int tid = threadIdx.x, K = P.D.top_e;
   const float* lr = reinterpret_cast<const float*>(g_sm + P.o_lr);
   const float* rbuf = reinterpret_cast<const float*>(g_sm + P.o_rbuf);
+  float* yacc = P.y_acc + (size_t)tok * P.D.d;     // token tok's accumulator row
+  uint32_t* cnt = P.slice_cnt + tok * P.cs;         // and its slices' arrival counters
   ok = wait_phase(&M.bar[kBarY], 0, P.err) && ok;
   MARK(13);
   const float we = M.wk[rc];
@@ -1044,28 +1049,28 @@ __device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int r
         const float4 v = *reinterpret_cast<const float4*>(rbuf + src * P.slice + 4 * j);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      red_add_v4(P.y_acc + q * P.slice + 4 * j, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
+      red_add_v4(yacc + q * P.slice + 4 * j, we * acc.x, we * acc.y, we * acc.z, we * acc.w);
     }
   }
   // the CTA's reduction-adds precede (barrier, then the release of the counter's atomic)
   // its count; the last contributor's acquire makes every other contribution visible
   __syncthreads();
-  if (tid == 0) M.last = (atom_add_acq_rel_gpu(P.slice_cnt + q, 1u) == (uint32_t)(K - 1));
+  if (tid == 0) M.last = (atom_add_acq_rel_gpu(cnt + q, 1u) == (uint32_t)(K - 1));
   __syncthreads();
   if (M.last) {
     // every contribution to this slice has arrived: convert, re-zero, reset
 #pragma unroll 1
     for (int j = tid; j < P.slice / 4; j += kFT) {
-      float4* p = reinterpret_cast<float4*>(P.y_acc + q * P.slice) + j;
+      float4* p = reinterpret_cast<float4*>(yacc + q * P.slice) + j;
       const float4 v = __ldcg(p);
       __stcg(p, make_float4(0.f, 0.f, 0.f, 0.f));
       const uint32_t lo = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.x)) |
                           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.y)) << 16);
       const uint32_t hi = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.z)) |
                           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(v.w)) << 16);
-      reinterpret_cast<uint2*>(P.out + q * P.slice)[j] = make_uint2(lo, hi);
+      reinterpret_cast<uint2*>(P.out + (size_t)tok * P.D.d + q * P.slice)[j] = make_uint2(lo, hi);
     }
-    if (tid == 0) P.slice_cnt[q] = 0u;
+    if (tid == 0) cnt[q] = 0u;
   }
   return ok;
 }
@@ -1074,7 +1079,11 @@ template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
 __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_constant__ FusedParams P) {
   const int CS = P.cs;
   const int q = (int)cluster_rank();
-  const int rc = blockIdx.x / CS;  // which routed expert (rank order)
+  // token tok, routed expert of rank rc: one cluster per (token, expert) pair; pr is the
+  // pair's row in the trace
+  const int tok = blockIdx.x / (CS * P.D.top_e);
+  const int rc = blockIdx.x / CS - tok * P.D.top_e;
+  const int pr = blockIdx.x / CS;
   const int tid = threadIdx.x, warp = tid >> 5;
   const int d = P.D.d, r = P.D.rank;
   Misc& M = misc(P);
@@ -1102,9 +1111,9 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
     if (pass == (P.x_ready ? 0 : 1)) {
       if (tid == 0) {
         mbar_arrive_expect_tx(&M.bar[kBarX], 2u * d);
-        if (!P.x_mapped) bulk_g2s(xs, P.x, 2u * d, &M.bar[kBarX]);
+        if (!P.x_mapped) bulk_g2s(xs, P.x + (size_t)tok * d, 2u * d, &M.bar[kBarX]);
       }
-      if (P.x_mapped && tid < xv) xpiece = ld_fresh16(P.x + 8 * (q * xv + tid));
+      if (P.x_mapped && tid < xv) xpiece = ld_fresh16(P.x + (size_t)tok * d + 8 * (q * xv + tid));
       cluster_wait();  // every CTA of the cluster has initialised its barriers
       if (P.x_mapped && tid < xv) {
         const uint32_t la = smem_addr(xs + 8 * (q * xv + tid)), rb = smem_addr(&M.bar[kBarX]);
@@ -1147,11 +1156,11 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
   // combine weights (warp 0; read in phase E, many barriers later)
   if (warp == 0) router_weights(in_big<float>(P, P.o_logits), P.D.experts, P.D.top_e, P.D.renorm, M);
 
-  ok = phase_scores<IT>(P, q, rc, nt, lt0, nz, ok, xf);
+  ok = phase_scores<IT>(P, q, pr, nt, lt0, nz, ok, xf);
   MARK(6);
   const int lgcs = CS == 16 ? 4 : 3;  // (the cluster size is 8 or 16)
   const int nmine = P.k > q ? (P.k - q + CS - 1) >> lgcs : 0;
-  ok = phase_select(P, e, q, rc, nmine, lgcs, ok);
+  ok = phase_select(P, e, q, pr, tok, nmine, lgcs, ok);
   // A_e z on this CTA's output slice while the first records fly (A_e from L2)
   if (r > 0) {
     ok = wait_phase(&M.bar[kBarZ], 0, P.err) && ok;
@@ -1165,7 +1174,7 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
   // quiesce below waits for them)
   cluster_arrive_relaxed();
   __syncthreads();   // lr complete (a CTA may have had no records, hence no barrier since)
-  ok = phase_combine(P, q, rc, ok);
+  ok = phase_combine(P, q, rc, tok, ok);
   MARK(14);
   cluster_wait();
   // every push aimed at this CTA has now been issued: if any wait of this CTA ran out,
@@ -1271,13 +1280,16 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int limit) {
 
 // Prefer 16-CTA clusters small enough to pair on an SM (all K clusters then fit the
 // GPCs), then 16-CTA clusters at any size when all K are resident, then 8-CTA
-// clusters; otherwise decline (the multi-kernel path runs).
-bool choose(FusedParams& P, const Dims& D, int k) {
+// clusters; otherwise decline (the multi-kernel path runs).  With several tokens (B K
+// clusters) 8-CTA clusters that pair on an SM come first: twice the work per CTA, but
+// the whole batch resident in one wave.
+bool choose(FusedParams& P, const Dims& D, int k, int batch = 1) {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64 || !g_ready[dev]) return false;
   const int K = D.top_e;
   const int pair = g_pair_smem[dev];
   const bool have16 = g_max_clusters16[dev] >= 1, have8 = g_max_clusters8[dev] >= 1;
+  if (batch > 1 && have8 && plan(P, D, k, 8, pair)) return true;
   if (have16 && plan(P, D, k, 16, pair)) return true;
   if (have16 && g_max_clusters16[dev] >= K && plan(P, D, k, 16, kSmemMax)) return true;
   if (have8 && plan(P, D, k, 8, pair)) return true;
@@ -1336,13 +1348,13 @@ int fused_setup() {
   return MSB_OK;
 }
 
-void fused_plan_info(const Dims& D, int k, int* info) {
+void fused_plan_info(const Dims& D, int k, int batch, int* info) {
   FusedParams P{};
   P.dense = (k == D.inter);
   const int dev = cur_dev();
 #pragma unroll 1
   for (int i = 0; i < 6; ++i) info[i] = 0;
-  if (choose(P, D, k)) {
+  if (choose(P, D, k, batch)) {
     info[0] = P.cs;
     info[1] = 1;
     info[2] = P.ring;
@@ -1365,7 +1377,8 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
                  const uint16_t* lr_b, uint16_t* out, const Dims& D, uint32_t* err,
                  uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st, bool x_mapped,
-                 bool x_ready) {
+                 bool x_ready, int batch) {
+  if (batch < 1 || batch > kFusedMaxBatch || (batch > 1 && (x_mapped || tr.union_count))) return MSB_ENOTFUSED;
   FusedParams P{};
   P.x_mapped = x_mapped ? 1 : 0;
   P.x_ready = x_ready ? 1 : 0;
@@ -1389,9 +1402,10 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
   P.D = D;
   P.k = k;
   P.dense = (k == D.inter);
-  if (!choose(P, D, k)) return MSB_ENOTFUSED;
+  if (!choose(P, D, k, batch)) return MSB_ENOTFUSED;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(P.cs * D.top_e, 1, 1);
+  if (kCntFusedSlices + batch * P.cs > kCounters) return MSB_ENOTFUSED;
+  cfg.gridDim = dim3(P.cs * D.top_e * batch, 1, 1);
   cfg.blockDim = dim3(kFT, 1, 1);
   cfg.dynamicSmemBytes = P.smem;
   cfg.stream = st;
