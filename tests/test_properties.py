@@ -136,3 +136,14 @@ def test_packers_match_the_oracle_on_random_layers(msb, seed, d, inter, experts,
         tq, aq = oracle.ternary_sketch(gq)
         np.testing.assert_array_equal(decode_sketch(pq["sketch"], dims, e)[:inter], tq)
         np.testing.assert_array_equal(pq["alpha"][e, :inter], aq)
+
+
+def test_calibrate_threshold_matches_oracle():
+    """The package's threshold calibration (selection) and the oracle's (sort) agree,
+    with and without ties, at budgets 0, 13%, 18%, 100%."""
+    import oracle
+    from token_top_expert_b200.block import calibrate_threshold
+    rng = np.random.default_rng(5)
+    for scores in (rng.random(4096), np.round(rng.random(4096) * 20) / 20, np.ones(7), rng.random(1)):
+        for budget in (0.0, 0.13, 0.18, 1.0):
+            assert calibrate_threshold(scores, budget) == oracle.calibrate_threshold(scores, budget)

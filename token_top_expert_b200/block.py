@@ -462,9 +462,15 @@ def residual_rmsnorm(h, y, x_next, eps: float = 1e-6, stream=None):
 
 
 def calibrate_threshold(scores: np.ndarray, budget: float) -> float:
-    """Offline calibration of the threshold comparator (not part of the decode path):
-    the score above which a fraction `budget` of the pooled calibration scores lie
-    (the (m+1)-th largest, m = floor(N * budget))."""
-    s = np.sort(np.asarray(scores, dtype=np.float64).ravel())[::-1]
-    m = int(np.floor(s.size * budget))
-    return float(s[min(m, s.size - 1)])
+    """Offline calibration of the threshold comparator (not part of the decode path).
+
+    The reading of "The threshold promises a budget but does not keep it": tau is the
+    pooled calibration score with exactly m = floor(N * budget) scores above it when
+    there are no ties, i.e. the (m+1)-th largest.  Found here by linear-time selection
+    (the element of ascending rank N - 1 - m), not by a full sort."""
+    s = np.asarray(scores, dtype=np.float64).ravel()
+    if s.size == 0:
+        raise ValueError("no calibration scores")
+    m = min(int(np.floor(s.size * budget)), s.size - 1)
+    r = s.size - 1 - m
+    return float(np.partition(s, r)[r])
