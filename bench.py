@@ -167,22 +167,29 @@ def block_launches(path, dense, rank):
     return 4 + (1 if (not dense or rank > 0) else 0) + (0 if dense else 1)
 
 
-def algorithmic_bytes(w, k, rank, union_sizes, dense):
+def q4_record_bytes(d):
+    """One 4-bit channel record: 3d codes at 4 bits, a BF16 scale and bias per group of 64
+    of the three vectors, padded to 16 bytes."""
+    return (3 * d // 2 + 3 * (d // 64) * 4 + 15) // 16 * 16
+
+
+def algorithmic_bytes(w, k, rank, union_sizes, dense, q4=False):
     """Bytes the method must read for one step: per used expert the sketch
-    (I*d/4), row scales (4I), the union of selected channel records (6d each)
-    and A_e, B_e (4dr).  The dense path (k = I) reads no sketch or scales; it still
-    adds the low-rank term when rank > 0."""
+    (I*d/4), row scales (4I), the union of selected channel records (6d each, or the
+    4-bit record size) and A_e, B_e (4dr).  The dense path (k = I) reads no sketch or
+    scales; it still adds the low-rank term when rank > 0."""
+    rec = q4_record_bytes(w.d) if q4 else 6 * w.d
     total = 0
     for u in union_sizes:
         if u == 0:
             continue
-        total += 6 * w.d * int(u) + 4 * w.d * rank
+        total += rec * int(u) + 4 * w.d * rank
         if not dense:
             total += w.inter * w.d // 4 + 4 * w.inter
     return total
 
 
-def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None, timed_s=12.0):
+def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None, timed_s=12.0, q4=False):
     """Time the FP64 CPU oracle, as it stands, on the first tokens of the step
     sequence: a warm pass (bounded by budget_s) fills its weight caches, then passes
     over the same tokens are timed until at least timed_s seconds of oracle work.
@@ -195,6 +202,9 @@ def oracle_sample(w, k, rank, xs, budget_s=15.0, max_tokens=None, top_e=None, ti
     except Exception:  # noqa: BLE001
         threads = 1
     lay = oracle.SynthLayer(w, max_cache=w.experts)
+    if q4:
+        from oracle import q4 as oq4
+        lay = oq4.Q4Layer(lay, max_cache=w.experts)
     toks = []
     t0 = time.time()
     n = 0
@@ -328,7 +338,8 @@ def config_of(w, args):
             "global_batch": args.batch * args.gpus, "batch_per_gpu": args.batch,
             "decode_steps": w.steps, "replicas": args.replicas,
             "l2": "inputs larger than L2: %d weight replicas rotated per step" % args.replicas,
-            "parallelism": "replicas" if args.gpus > 1 else "single"}
+            "parallelism": "replicas" if args.gpus > 1 else "single",
+            "records": "4-bit (group 64, affine)" if getattr(args, "q4", False) else "bf16"}
 
 
 def run_stack(args, w, world, rank, local):
@@ -532,6 +543,8 @@ def main():
                     help="stacked workload: run k in {13%%, 18%%, 100%%} x batch in {1, 32} on one set of layers")
     ap.add_argument("--threshold", action="store_true",
                     help="measure the calibrated-threshold comparator instead of top-k")
+    ap.add_argument("--q4", action="store_true",
+                    help="4-bit channel records (moe_sparse_block_q4; batches of at most 16 tokens)")
     ap.add_argument("--phase-marks", action="store_true",
                     help="per-phase timeline of the single-launch kernel (instrumented build)")
     args = ap.parse_args()
@@ -582,7 +595,7 @@ def main():
     # ---- weights: generate, pack (host C++ packer), upload, replicate
     lw = synth.layer_weights(w)
     dims = msb.Dims(w.d, w.inter, w.experts, w.top_e, args.rank, 1)
-    pk = msb.pack(lw.gate, lw.up, lw.down, lw.router, dims)
+    pk = (msb.pack_q4 if args.q4 else msb.pack)(lw.gate, lw.up, lw.down, lw.router, dims)
     base = msb.PackedLayer.from_host(dims, pk, lw.lr_a, lw.lr_b, device=dev)
     del lw, pk
     layers = [base] + [base.clone() for _ in range(args.replicas - 1)]
@@ -601,7 +614,11 @@ def main():
 
     # ---- union sizes of every step of the sequence (one traced pass) -> algorithmic bytes
     dense = args.k == w.inter
-    tr = msb.Trace(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B, args.k)
+    Kr = args.top_e or w.top_e
+    # (4-bit records run on the single launch, which leaves a batch's union count to the
+    # host: it is formed here from the traced selections)
+    host_union = args.q4 and B > 1
+    tr = msb.Trace(msb.Dims(w.d, w.inter, w.experts, Kr, args.rank, 1), B, args.k, union=not host_union)
     bytes_per_step = []
     with torch.cuda.stream(stream):
         for i in range(nseq):
@@ -610,8 +627,16 @@ def main():
                                  top_e=args.top_e)
             if i < 64 or not (B == 1 and not dense):
                 stream.synchronize()
-                bytes_per_step.append(algorithmic_bytes(w, args.k, args.rank,
-                                                        tr.union_count.cpu().tolist(), dense))
+                if host_union:
+                    ids, sel = tr.expert_ids.cpu().numpy(), tr.sel.cpu().numpy()
+                    sets = {}
+                    for t in range(B):
+                        for r in range(Kr):
+                            sets.setdefault(int(ids[t][r]), set()).update(sel[t][r].tolist())
+                    union = [len(v) for v in sets.values()]
+                else:
+                    union = tr.union_count.cpu().tolist()
+                bytes_per_step.append(algorithmic_bytes(w, args.k, args.rank, union, dense, args.q4))
     stream.synchronize()
     ws.check(stream)
     step_bytes = float(np.mean(bytes_per_step))
@@ -666,7 +691,7 @@ def main():
     xh = torch.from_numpy(np.stack(xs_host).view(np.int16)).view(torch.bfloat16).pin_memory()
     oh = torch.empty_like(xh).pin_memory()
     ne = min(args.e2e_steps, args.steps)
-    if args.top_e is None:
+    if args.top_e is None and not args.q4:
         # the host produces each step's x before the call (nothing on the stream writes
         # it), so the calls declare it ready: the kernel fetches x across the host link
         # while the previous launch still runs
@@ -709,7 +734,7 @@ def main():
     plan = msb.path_info(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B,
                          args.k, general=general)
     kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
-    traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else ""))
+    traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else "") + ("_q4" if args.q4 else ""))
     launches_per_step = block_launches(plan["path"], dense, args.rank)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world if world > 1 else 1,
@@ -731,7 +756,7 @@ def main():
     }
     if rank == 0 and not args.no_cpu_baseline:
         v, ntok, dt, threads = oracle_sample(w, args.k, args.rank, xs_host, budget_s=6.0,
-                                             top_e=args.top_e)
+                                             top_e=args.top_e, q4=args.q4)
         line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
                                 "sample": "%d token-blocks: passes over the first tokens of the "
                                           "same decode sequence (FP64 numpy oracle, weights "

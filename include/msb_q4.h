@@ -32,8 +32,8 @@
  * The sketch of a 4-bit layer is the ternary sketch of its dequantised gate rows, in
  * the format and with the rule of msb_pack (msb.h); router_t as msb_pack.
  *
- * Status: the block's kernels read BF16 records; none of msb.h's entry points reads
- * 4-bit records yet.
+ * moe_sparse_block_q4 runs the block on such records; the weights it computes with are
+ * the dequantised s * q + b (scores from the sketch of the dequantised gate rows).
  */
 #ifndef MSB_Q4_H_
 #define MSB_Q4_H_
@@ -65,6 +65,22 @@ int32_t msb_pack_q4(const uint16_t* gate_host, const uint16_t* up_host, const ui
                     const uint16_t* router_host, const msb_dims* dims, uint8_t* records_host,
                     uint32_t* sketch_host, float* alpha_host, uint16_t* router_t_host,
                     int32_t threads);
+
+/* The block of moe_sparse_block (msb.h: same arguments, same result, same workspace)
+ * on 4-bit channel records: records_q4 is the records array of msb_pack_q4 (device,
+ * 16-byte aligned), sketch and alpha those msb_pack_q4 wrote for the dequantised gate
+ * rows; router_t and the low-rank factors as msb_pack / moe_sparse_block.  Runs on the
+ * single-launch kernel only (batches up to 16 tokens whose shapes fit its plan): it
+ * gathers 3 d / 2 + 12 d / 64 bytes per channel (rounded up to 16) instead of 6 d, and
+ * forms gate.x per group of 64 weights as s * (q . x) + b * sum(x) in FP32.  Returns
+ * MSB_EUNSUPPORTED where the single launch declines (more than 16 tokens, a batch trace
+ * that asks for union counts, MSB_FLAG_GENERAL, shapes beyond its plan); other errors
+ * as moe_sparse_block. */
+int32_t moe_sparse_block_q4(const void* x, int32_t batch, const void* router_t, const void* records_q4,
+                            const uint32_t* sketch, const float* alpha, int32_t k, const void* lr_a,
+                            const void* lr_b, void* out, const msb_dims* dims, void* workspace,
+                            size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
+                            void* stream);
 
 #ifdef __cplusplus
 }

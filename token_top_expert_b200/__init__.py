@@ -17,6 +17,7 @@ from .block import (  # noqa: F401
     noalloc_check,
     pack,
     pack_q4,
+    q4_record_bytes,
     path_info,
     residual_rmsnorm,
     sketch_words,

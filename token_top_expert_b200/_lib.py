@@ -36,7 +36,7 @@ SYMBOLS = (
     "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
     "moe_sparse_block_noalloc", "msb_noalloc_check", "moe_sparse_block_top_e",
     "moe_sparse_block_host",
-    "msb_q4_record_bytes", "msb_pack_q4",
+    "msb_q4_record_bytes", "msb_pack_q4", "moe_sparse_block_q4",
 )
 MSB_Q4_GROUP = 64
 
@@ -85,6 +85,7 @@ def load() -> ctypes.CDLL:
         "msb_check": (I32, [P, P]),
         "msb_strerror": (ctypes.c_char_p, [I32]),
         "moe_sparse_block": (I32, [P, I32, P, P, P, P, I32, P, P, P, dims_p, P, SZ, trace_p, U32, P]),
+        "moe_sparse_block_q4": (I32, [P, I32, P, P, P, P, I32, P, P, P, dims_p, P, SZ, trace_p, U32, P]),
         "moe_sparse_block_threshold": (I32, [P, I32, P, P, P, P, F32, P, P, P, dims_p, P, SZ,
                                              trace_p, P]),
         "msb_residual_rmsnorm": (I32, [P, P, P, I32, I32, F32, P]),

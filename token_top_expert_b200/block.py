@@ -50,6 +50,11 @@ def sketch_words(dims: Dims) -> int:
     return _lib.load().msb_sketch_words(ctypes.byref(dims.c()))
 
 
+def q4_record_bytes(dims: Dims) -> int:
+    """Bytes of one 4-bit channel record (include/msb_q4.h)."""
+    return _lib.load().msb_q4_record_bytes(ctypes.byref(dims.c()))
+
+
 def pack(gate: np.ndarray, up: np.ndarray, down: np.ndarray, router: np.ndarray, dims: Dims,
          threads: int = 0) -> dict:
     """Pack model-layout BF16 weights (uint16 bit arrays) with libmsb's host packer.
@@ -113,10 +118,12 @@ def pack_q4(gate: np.ndarray, up: np.ndarray, down: np.ndarray, router: np.ndarr
 class PackedLayer:
     """One MoE layer's packed weights resident on a CUDA device."""
 
-    def __init__(self, dims: Dims, records, sketch, alpha, router_t, lr_a=None, lr_b=None):
+    def __init__(self, dims: Dims, records, sketch, alpha, router_t, lr_a=None, lr_b=None, q4=False):
+        """q4: records are 4-bit channel records (msb_pack_q4: uint8 [E][I][record bytes])."""
         self.dims = dims
         self.records, self.sketch, self.alpha, self.router_t = records, sketch, alpha, router_t
         self.lr_a, self.lr_b = lr_a, lr_b
+        self.q4 = q4
         self._check()
 
     def _check(self):
@@ -126,7 +133,8 @@ class PackedLayer:
         words = sketch_words(self.dims)
         if words == 0:
             raise ValueError("dims rejected by the library: %s" % (self.dims,))
-        want = [("records", self.records, E * I * 3 * d, 2), ("sketch", self.sketch, words, 4),
+        rec = ((E * I * q4_record_bytes(self.dims), 1) if self.q4 else (E * I * 3 * d, 2))
+        want = [("records", self.records) + rec, ("sketch", self.sketch, words, 4),
                 ("alpha", self.alpha, E * self.dims.ipad, 4), ("router_t", self.router_t, E * d, 2)]
         if r > 0:
             want += [("lr_a", self.lr_a, E * d * r, 2), ("lr_b", self.lr_b, E * r * d, 2)]
@@ -153,22 +161,23 @@ class PackedLayer:
         if r > 0 and lr_a is not None and lr_b is not None:
             # factors of a higher rank: the first r columns of A_e and rows of B_e
             lr_a, lr_b = lr_a[:, :, :r], lr_b[:, :r, :]
-        return cls(dims, t(packed["records"].view(np.int16)), t(packed["sketch"].view(np.int32)),
-                   t(packed["alpha"]), t(packed["router_t"].view(np.int16)),
+        q4 = packed["records"].dtype == np.uint8  # pack_q4 output
+        return cls(dims, t(packed["records"] if q4 else packed["records"].view(np.int16)),
+                   t(packed["sketch"].view(np.int32)), t(packed["alpha"]), t(packed["router_t"].view(np.int16)),
                    None if lr_a is None or r == 0 else t(lr_a.view(np.int16)),
-                   None if lr_b is None or r == 0 else t(lr_b.view(np.int16)))
+                   None if lr_b is None or r == 0 else t(lr_b.view(np.int16)), q4=q4)
 
     def clone(self) -> "PackedLayer":
         """A copy at different addresses (same values)."""
         c = lambda a: None if a is None else a.clone()
         return PackedLayer(self.dims, c(self.records), c(self.sketch), c(self.alpha),
-                           c(self.router_t), c(self.lr_a), c(self.lr_b))
+                           c(self.router_t), c(self.lr_a), c(self.lr_b), q4=self.q4)
 
     def without_lowrank(self) -> "PackedLayer":
         """The same weights (shared, not copied) with rank 0: no compensation term."""
         d = self.dims
         return PackedLayer(Dims(d.d, d.inter, d.experts, d.top_e, 0, d.renorm), self.records,
-                           self.sketch, self.alpha, self.router_t, None, None)
+                           self.sketch, self.alpha, self.router_t, None, None, q4=self.q4)
 
     def nbytes(self) -> int:
         return sum(a.numel() * a.element_size() for a in
@@ -316,7 +325,11 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
             _ptr(layer.alpha), k)
     rest = (_ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out), ctypes.byref(dims.c()), workspace.ptr,
             workspace.nbytes, ctypes.byref(tr) if tr is not None else None, flags, _stream(stream))
-    if top_e is None:
+    if layer.q4:
+        if top_e is not None:
+            raise ValueError("4-bit records: the expert-count override is not available")
+        rc = _lib.load().moe_sparse_block_q4(*args, *rest)
+    elif top_e is None:
         rc = _lib.load().moe_sparse_block(*args, *rest)
     else:
         rc = _lib.load().moe_sparse_block_top_e(*args, top_e, *rest)
@@ -335,6 +348,8 @@ def moe_sparse_block_noalloc(x, layer: PackedLayer, k: int, out=None, trace: Tra
     """The batch-1 block without a workspace (scratch is a static device array of
     the library), for callers that cannot allocate device memory.  Read the call's
     kernel status with noalloc_check() before the next such call."""
+    if layer.q4:
+        raise ValueError("4-bit records: use moe_sparse_block")
     import torch
     dims = layer.dims
     _act(x, dims)
@@ -369,6 +384,8 @@ class HostCall:
 
     def __init__(self, layer: PackedLayer, k: int, batch: int, stream=None, general: bool = False,
                  x_ready: bool = False):
+        if layer.q4:
+            raise ValueError("4-bit records: use moe_sparse_block")
         import torch
         dims = layer.dims
         if not 1 <= k <= dims.inter:
@@ -412,6 +429,8 @@ def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
                                workspace: Workspace | None = None, trace: Trace | None = None,
                                stream=None):
     """The calibrated-threshold comparator: channels with score > tau."""
+    if layer.q4:
+        raise ValueError("4-bit records: use moe_sparse_block")
     import torch
     dims = layer.dims
     _act(x, dims)

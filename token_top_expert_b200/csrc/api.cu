@@ -8,6 +8,7 @@
 #include "fused.h"
 #include "launch.h"
 #include "msb.h"
+#include "msb_q4.h"
 
 namespace msb {
 
@@ -178,7 +179,7 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
                  const uint32_t* sketch, const float* alpha, int32_t k, int mode, float tau,
                  const void* lr_a, const void* lr_b, void* out, const msb_dims* dims,
                  void* workspace, size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
-                 void* stream, bool x_mapped = false) {
+                 void* stream, bool x_mapped = false, bool q4 = false) {
   int rc = check_dims(dims);
   if (rc != MSB_OK) return rc;
   if (batch < 1) return MSB_EINVAL;
@@ -209,12 +210,13 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
   const uint16_t* la = static_cast<const uint16_t*>(lr_a);
   const uint16_t* lb = static_cast<const uint16_t*>(lr_b);
   uint16_t* o = static_cast<uint16_t*>(out);
-  if (mode == 0 && batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k)) {
+  if (mode == 0 && batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k, q4)) {
     rc = launch_fused(xb, rt, rec, sketch, alpha, k, la, lb, o, D, ws.err, ws.counters, ws.y_acc,
-                      tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0, batch);
+                      tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0, batch, q4);
     if (rc != MSB_ENOTFUSED) return rc;
   }
   if (x_mapped) return MSB_ENOTFUSED;  // the multi-kernel path takes device buffers only
+  if (q4) return MSB_EUNSUPPORTED;     // 4-bit records: the single-launch kernel only
   return launch_general(xb, batch, rt, rec, sketch, alpha, k, mode, tau, la, lb, o, D, ws, tr, st);
 }
 
@@ -285,6 +287,16 @@ int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, con
                          void* stream) {
   return block_common(x, batch, router_t, records, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out, dims,
                       workspace, workspace_bytes, trace, flags, stream);
+}
+
+int32_t moe_sparse_block_q4(const void* x, int32_t batch, const void* router_t, const void* records_q4,
+                            const uint32_t* sketch, const float* alpha, int32_t k, const void* lr_a,
+                            const void* lr_b, void* out, const msb_dims* dims, void* workspace,
+                            size_t workspace_bytes, const msb_trace* trace, uint32_t flags,
+                            void* stream) {
+  if (flags & MSB_FLAG_GENERAL) return MSB_EUNSUPPORTED;
+  return block_common(x, batch, router_t, records_q4, sketch, alpha, k, 0, 0.f, lr_a, lr_b, out, dims,
+                      workspace, workspace_bytes, trace, flags, stream, false, true);
 }
 
 int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_t,

@@ -93,6 +93,8 @@ struct FusedParams {
   int o_alpha, o_brows;                                  // inside big (phase B)
   int smem;
   uint32_t x1_bytes, sc_bytes, z_bytes, y_bytes;  // bytes each CTA expects per exchange
+  int q4;        // records are 4-bit (group-wise affine, 64 weights per group)
+  uint32_t rec_bytes;  // bytes of one channel record (6d for BF16)
   int x_ready;   // nothing earlier on the stream writes x: fetch it before the grid
                  // dependency wait
   int x_mapped;  // x and out are pinned host memory mapped into the device's address space:
@@ -612,10 +614,12 @@ __device__ __noinline__ void quiesce(Misc& M, int dense, uint32_t* err, uint64_t
 // Issue the bulk copy of channel `ch`'s record into ring slot `slot`.
 __device__ __forceinline__ void issue_record(const FusedParams& P, Misc& M, uint16_t* ring, int e,
                                              int ch, int slot) {
-  const uint32_t rb = 6u * (uint32_t)P.D.d;
+  const size_t idx = (size_t)e * P.D.inter + ch;
+  const uint32_t rb = P.rec_bytes;
+  const void* src = P.q4 ? static_cast<const void*>(reinterpret_cast<const uint8_t*>(P.records) + idx * rb)
+                         : static_cast<const void*>(P.records + idx * 3 * P.D.d);
   mbar_arrive_expect_tx(&M.bar[kBarRing + slot], rb);
-  bulk_g2s(ring + (size_t)slot * P.rs, P.records + ((size_t)e * P.D.inter + ch) * 3 * P.D.d, rb,
-           &M.bar[kBarRing + slot]);
+  bulk_g2s(ring + (size_t)slot * P.rs, src, rb, &M.bar[kBarRing + slot]);
 }
 
 
@@ -1027,6 +1031,174 @@ __device__ __forceinline__ bool phase_records(const FusedParams& P, int e, int q
   return ok;
 }
 
+// ---------------------------------------------------------------- 4-bit channel records
+// Record of one channel (group-wise affine, 64 weights per group): the nibble codes of the
+// gate row, the up row and the down column (byte i: element 2i in bits 0-3, 2i + 1 in bits
+// 4-7), then each vector's (scale, bias) BF16 pairs; the weight is s * q + b.
+
+// code k of a byte lane as an exact float: the byte placed in the mantissa of 2^23
+__device__ __forceinline__ float nib(uint32_t bytes, uint32_t sel) {
+  return __uint_as_float(__byte_perm(bytes, 0x4B000000u, sel)) - 8388608.0f;
+}
+
+// acc + sum of the 8 codes of c (elements 0..7 in order) times xf[0..8)
+__device__ __forceinline__ float dot8q(uint32_t c, const float (&xf)[8], float acc) {
+  const uint32_t lo = c & 0x0F0F0F0Fu, hi = (c >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc = fmaf(nib(lo, 0x7650u | i), xf[2 * i], acc);
+    acc = fmaf(nib(hi, 0x7650u | i), xf[2 * i + 1], acc);
+  }
+  return acc;
+}
+
+// y[0..8) += hs * (the 8 codes of c)
+__device__ __forceinline__ void axpy8q(float (&y)[8], float hs, uint32_t c) {
+  const uint32_t lo = c & 0x0F0F0F0Fu, hi = (c >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    y[2 * i] = fmaf(hs, nib(lo, 0x7650u | i), y[2 * i]);
+    y[2 * i + 1] = fmaf(hs, nib(hi, 0x7650u | i), y[2 * i + 1]);
+  }
+}
+
+// D on 4-bit records: the batches, waits, refills and pushes of phase_records; each
+// thread's 8 elements lie in one group, so gate.x over them is s * (q . x) + b * sum(x)
+// and the down update is (h s) q plus h b, the latter summed once per record.
+template <int IT>
+__device__ __forceinline__ bool phase_records_q4(const FusedParams& P, int e, int q, int nmine, bool ok,
+                                                 const float (&xf)[IT][8]) {
+  Misc& M = misc(P);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, d = P.D.d;
+  const uint8_t* ring8 = big_of(P);
+  const size_t slotb = 2u * (size_t)P.rs;                  // slot stride = record bytes
+  const int G = d / 64;
+  const uint32_t pb = 3u * (uint32_t)d / 2u;               // offset of the (scale, bias) pairs
+  const int bmax = max(1, min(4, P.ring / 2));
+  float xsum[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it)
+    xsum[it] = ((xf[it][0] + xf[it][1]) + (xf[it][2] + xf[it][3])) + ((xf[it][4] + xf[it][5]) + (xf[it][6] + xf[it][7]));
+  float y[IT][8], yb[IT];
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    yb[it] = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[it][i] = 0.f;
+  }
+  int s0 = 0, pb0 = 0, pnb = 0;
+  uint32_t par0 = 0;
+  int issued = ok ? min(P.ring, nmine) : 0, landed = 0;
+#pragma unroll 1
+  for (int i = 0; i < nmine;) {
+    const int nb = i == 0 ? 1 : min(bmax, nmine - i);
+    if (ok) {
+#pragma unroll 1
+      for (int j = 0; j < nb && ok; ++j) {
+        const int sl = s0 + j < P.ring ? s0 + j : s0 + j - P.ring;
+        ok = wait_phase(&M.bar[kBarRing + sl], s0 + j < P.ring ? par0 : par0 ^ 1u, P.err);
+      }
+      if (ok) landed = i + nb;
+    }
+    {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = 0.f;
+      const uint8_t* rec[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int jj = s0 + min(j, nb - 1);
+        rec[j] = ring8 + (size_t)(jj < P.ring ? jj : jj - P.ring) * slotb;
+      }
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kFT + tid) * 8;
+        if (el < d) {
+          const int g = el / 64;
+          uint32_t c[8], sb[8];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            c[2 * j] = *reinterpret_cast<const uint32_t*>(rec[j] + el / 2);
+            c[2 * j + 1] = *reinterpret_cast<const uint32_t*>(rec[j] + d / 2 + el / 2);
+            sb[2 * j] = *reinterpret_cast<const uint32_t*>(rec[j] + pb + 4 * g);
+            sb[2 * j + 1] = *reinterpret_cast<const uint32_t*>(rec[j] + pb + 4 * (G + g));
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            v[j] = fmaf(bf16_lo(sb[j]), dot8q(c[j], xf[it], 0.f), fmaf(bf16_hi(sb[j]), xsum[it], v[j]));
+        }
+      }
+      const float sw = warp_sum8(v);
+      if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
+    }
+    ok = __syncthreads_and(ok);
+    if (tid == 32 && ok && pnb > 0 && issued < nmine) {
+      uint16_t* wring = reinterpret_cast<uint16_t*>(big_of(P));
+      fence_proxy_async();
+#pragma unroll 1
+      for (int j = 0; j < pnb && issued < nmine; ++j, ++issued)
+        issue_record(P, M, wring, e, MYSEL(P)[issued], pb0 + j < P.ring ? pb0 + j : pb0 + j - P.ring);
+    }
+    if (i == 0) MARK(11);
+    if (tid < nb) {
+      float gs = 0.f, us = 0.f;
+#pragma unroll
+      for (int w = 0; w < kFW; ++w) {
+        gs += M.red8[w][2 * tid];
+        us += M.red8[w][2 * tid + 1];
+      }
+      M.h[tid] = __fdividef(gs, 1.0f + __expf(-gs)) * us;
+    }
+    __syncthreads();
+    // y += h_j * down_j: (h s) q per element, h b once per record
+#pragma unroll 1
+    for (int j = 0; j < nb; j += 2) {
+      const int ja = s0 + j, jb = s0 + min(j + 1, nb - 1);
+      const uint8_t* reca = ring8 + (size_t)(ja < P.ring ? ja : ja - P.ring) * slotb;
+      const uint8_t* recb = ring8 + (size_t)(jb < P.ring ? jb : jb - P.ring) * slotb;
+      const float ha = M.h[j], hb = j + 1 < nb ? M.h[j + 1] : 0.f;
+#pragma unroll
+      for (int it = 0; it < IT; ++it) {
+        const int el = (it * kFT + tid) * 8;
+        if (el < d) {
+          const int g = el / 64;
+          const uint32_t ca = *reinterpret_cast<const uint32_t*>(reca + d + el / 2);
+          const uint32_t cb = *reinterpret_cast<const uint32_t*>(recb + d + el / 2);
+          const uint32_t sa = *reinterpret_cast<const uint32_t*>(reca + pb + 4 * (2 * G + g));
+          const uint32_t sbb = *reinterpret_cast<const uint32_t*>(recb + pb + 4 * (2 * G + g));
+          axpy8q(y[it], ha * bf16_lo(sa), ca);
+          axpy8q(y[it], hb * bf16_lo(sbb), cb);
+          yb[it] = fmaf(ha, bf16_hi(sa), fmaf(hb, bf16_hi(sbb), yb[it]));
+        }
+      }
+    }
+    pb0 = s0;
+    pnb = nb;
+    s0 += nb;
+    if (s0 >= P.ring) { s0 -= P.ring; par0 ^= 1u; }
+    i += nb;
+  }
+#pragma unroll
+  for (int it = 0; it < IT; ++it)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) y[it][i] += yb[it];
+  if (!ok) drain_ring(M, issued, landed, P.ring, P.err, WAIT_LIMIT);
+  __syncthreads();
+  MARK(12);
+  const uint32_t rbuf = smem_addr(g_sm + P.o_rbuf), rbar_y = smem_addr(&M.bar[kBarY]);
+#pragma unroll
+  for (int it = 0; it < IT; ++it) {
+    const int el = (it * kFT + tid) * 8;
+    if (el < d) {
+      const int owner = el / P.slice, off = el - owner * P.slice;
+      const uint32_t ra = mapa(rbuf + 4u * (q * P.slice + off), owner), rb = mapa(rbar_y, owner);
+      st_async4(ra, y[it][0], y[it][1], y[it][2], y[it][3], rb);
+      st_async4(ra + 16u, y[it][4], y[it][5], y[it][6], y[it][7], rb);
+    }
+  }
+  return ok;
+}
+
 // E: the owner of slice q sums the cluster's partials of it, adds A_e z, weights by
 // the router and reduction-adds into the FP32 accumulator; the last of the K
 // contributions converts the slice to BF16 and re-zeroes it.  Returns ok.
@@ -1075,7 +1247,7 @@ __device__ __forceinline__ bool phase_combine(const FusedParams& P, int q, int r
   return ok;
 }
 
-template <int IT>  // IT = ceil(d / 2048): 8-element groups per thread
+template <int IT, bool Q4>  // IT = ceil(d / 2048): 8-element groups per thread; Q4: 4-bit records
 __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_constant__ FusedParams P) {
   const int CS = P.cs;
   const int q = (int)cluster_rank();
@@ -1168,7 +1340,10 @@ __global__ void __launch_bounds__(kFT, 2) fused_block_kernel(const __grid_consta
                   reinterpret_cast<float*>(g_sm + P.o_lr));
   }
   MARK(10);
-  ok = phase_records<IT>(P, e, q, nmine, ok, xf);
+  if (Q4)
+    ok = phase_records_q4<IT>(P, e, q, nmine, ok, xf);
+  else
+    ok = phase_records<IT>(P, e, q, nmine, ok, xf);
   // paired with the wait before exit: no CTA leaves before every CTA of the cluster has
   // issued its pushes (each receiver waits for its own bytes; after an expired wait the
   // quiesce below waits for them)
@@ -1208,11 +1383,10 @@ int align_up(int v, int a) { return (v + a - 1) / a * a; }
 
 using KernelFn = void (*)(FusedParams);
 
-KernelFn kernel_for(int d) {
+KernelFn kernel_for(int d, bool q4) {
   const int it = (d + 2047) / 2048;
-  if (it <= 1) return fused_block_kernel<1>;
-  if (it <= 2) return fused_block_kernel<2>;
-  return fused_block_kernel<4>;
+  if (q4) return it <= 1 ? fused_block_kernel<1, true> : it <= 2 ? fused_block_kernel<2, true> : fused_block_kernel<4, true>;
+  return it <= 1 ? fused_block_kernel<1, false> : it <= 2 ? fused_block_kernel<2, false> : fused_block_kernel<4, false>;
 }
 
 // Fill the carve-up for cluster size cs within `limit` bytes of shared memory.
@@ -1235,7 +1409,10 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int limit) {
   // phase A/B region at the start of big: router rows, then (reused) sketch tiles,
   // alpha and B_e rows
   P.rrs = d + 8;
-  P.rs = 3 * d + 8;
+  // ring slot stride in elements: BF16 records 16 bytes apart in the banks; 4-bit records
+  // are read 4 bytes per thread, conflict-free at their own (16-byte multiple) size
+  P.rec_bytes = P.q4 ? (uint32_t)(((size_t)3 * d / 2 + (size_t)3 * (d / 64) * 4 + 15) / 16 * 16) : 6u * d;
+  P.rs = P.q4 ? (int)(P.rec_bytes / 2) : 3 * d + 8;
   const int rows_b = align_up(P.rpc * 2 * P.rrs, 128);
   int b = P.dense ? 0 : P.tpc * (d / kColChunk) * kChunkWords * 4;
   b = align_up(b, 128);
@@ -1322,7 +1499,8 @@ int query_clusters(KernelFn fn, int cs, int smem) {
 int fused_setup() {
   const int dev = cur_dev();
   if (dev < 0 || dev >= 64) return MSB_ECUDA;
-  for (KernelFn fn : {fused_block_kernel<1>, fused_block_kernel<2>, fused_block_kernel<4>}) {
+  for (KernelFn fn : {fused_block_kernel<1, false>, fused_block_kernel<2, false>, fused_block_kernel<4, false>,
+                      fused_block_kernel<1, true>, fused_block_kernel<2, true>, fused_block_kernel<4, true>}) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) !=
         cudaSuccess)
       return MSB_ECUDA;
@@ -1342,8 +1520,8 @@ int fused_setup() {
   }
   g_pair_smem[dev] = per_sm / 2 - reserved;
   if (g_pair_smem[dev] > kSmemMax) g_pair_smem[dev] = kSmemMax;
-  g_max_clusters16[dev] = query_clusters(fused_block_kernel<1>, 16, kSmemMax);
-  g_max_clusters8[dev] = query_clusters(fused_block_kernel<1>, 8, kSmemMax);
+  g_max_clusters16[dev] = query_clusters(fused_block_kernel<1, false>, 16, kSmemMax);
+  g_max_clusters8[dev] = query_clusters(fused_block_kernel<1, false>, 8, kSmemMax);
   g_ready[dev] = true;
   return MSB_OK;
 }
@@ -1366,9 +1544,10 @@ void fused_plan_info(const Dims& D, int k, int batch, int* info) {
   }
 }
 
-bool fused_supported(const Dims& D, int k) {
+bool fused_supported(const Dims& D, int k, bool q4) {
   FusedParams P{};
   P.dense = (k == D.inter);
+  P.q4 = q4 ? 1 : 0;
   return choose(P, D, k);
 }
 
@@ -1377,9 +1556,10 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
                  const uint32_t* sketch, const float* alpha, int k, const uint16_t* lr_a,
                  const uint16_t* lr_b, uint16_t* out, const Dims& D, uint32_t* err,
                  uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st, bool x_mapped,
-                 bool x_ready, int batch) {
+                 bool x_ready, int batch, bool q4) {
   if (batch < 1 || batch > kFusedMaxBatch || (batch > 1 && (x_mapped || tr.union_count))) return MSB_ENOTFUSED;
   FusedParams P{};
+  P.q4 = q4 ? 1 : 0;
   P.x_mapped = x_mapped ? 1 : 0;
   P.x_ready = x_ready ? 1 : 0;
   P.x = x;
@@ -1420,7 +1600,7 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
   attr[2].val.clusterSchedulingPolicyPreference = cudaClusterSchedulingPolicySpread;
   cfg.attrs = attr;
   cfg.numAttrs = 3;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(D.d), P);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel_for(D.d, P.q4 != 0), P);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 
