@@ -573,16 +573,17 @@ __device__ __forceinline__ void axpy8(float (&y)[8], float h, uint4 v) {
 
 
 // score = alpha * |sum of the 8 warps' partials| / 2 for this CTA's nrows rows, pushed
-// to every CTA of the cluster (keys at rows lt0*16 ...), with one max per warp of rows
-// into each CTA's cmax.
+// to every CTA of the cluster (keys at rows lt0*16 ...; four threads per row, each
+// pushing to a quarter of the cluster), with one max per warp into each CTA's cmax.
 __device__ __forceinline__ void push_scores(const FusedParams& P, Misc& M, const float* part,
                                          const float* alpha_s, uint32_t* keys, int nrows, int lt0,
                                          int rc, int q) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, CS = P.cs;
+  const int per = CS / 4;  // destinations per thread: four threads share a row
   const uint32_t rbar_s = smem_addr(&M.bar[kBarScores]);
 #pragma unroll 1
-  for (int lr0 = 0; lr0 < nrows; lr0 += kFT) {
-    const int row = lr0 + tid;
+  for (int i0 = 0; i0 < 4 * nrows; i0 += kFT) {
+    const int item = i0 + tid, row = item >> 2, d0 = (item & 3) * per;
     uint32_t key = 0;
     if (row < nrows) {
       float sc = 0.f;
@@ -590,13 +591,13 @@ __device__ __forceinline__ void push_scores(const FusedParams& P, Misc& M, const
       for (int w = 1; w < kFW; ++w) sc += part[w * P.tpc * kRowTile + row];
       sc = alpha_s[row] * fabsf(sc + part[row]) * 0.5f;
       key = __float_as_uint(sc);
-      if (P.tr.scores) P.tr.scores[(size_t)rc * P.D.ipad + lt0 * kRowTile + row] = sc;
+      if (P.tr.scores && d0 == 0) P.tr.scores[(size_t)rc * P.D.ipad + lt0 * kRowTile + row] = sc;
       const uint32_t la = smem_addr(keys + lt0 * kRowTile + row);
 #pragma unroll 1
-      for (int dst = 0; dst < CS; ++dst) st_async(mapa(la, dst), key, mapa(rbar_s, dst));
+      for (int dst = d0; dst < d0 + per; ++dst) st_async(mapa(la, dst), key, mapa(rbar_s, dst));
     }
     const uint32_t m = __reduce_max_sync(0xffffffffu, key);
-    if (lr0 + warp * 32 < nrows && lane < CS)
+    if (i0 + warp * 32 < 4 * nrows && lane < CS)
       red_async_max(mapa(smem_addr(&M.cmax), lane), m, mapa(rbar_s, lane));
   }
 }
@@ -744,13 +745,12 @@ __device__ __forceinline__ bool phase_router(const FusedParams& P, int q, bool o
     const float sw = warp_sum8(v);
     if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
     __syncthreads();
-    if (tid < nb) {
+    if (tid < nb * P.cs) {  // one thread per (row, destination)
+      const int row = tid / P.cs, dst = tid - row * P.cs;
       float acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFW; ++w) acc += M.red8[w][tid];
-#pragma unroll 1
-      for (int dst = 0; dst < P.cs; ++dst)
-        st_async(mapa(la + 4u * (r0 + tid), dst), __float_as_uint(acc), mapa(rbar, dst));
+      for (int w = 0; w < kFW; ++w) acc += M.red8[w][row];
+      st_async(mapa(la + 4u * (r0 + row), dst), __float_as_uint(acc), mapa(rbar, dst));
     }
     __syncthreads();
   }
@@ -764,6 +764,12 @@ __device__ __forceinline__ void issue_expert(const FusedParams& P, int e, int q,
   const int d = P.D.d, r = P.D.rank, KC = d / kColChunk, CS = P.cs;
   const int ntile_all = P.D.ipad / kRowTile;
   fence_proxy_async();  // the router rows were read through the generic proxy
+  // the B_e rows first: z is formed while the (larger) sketch tiles are in flight
+  mbar_arrive_expect_tx(&M.bar[kBarLow], (uint32_t)nz * 2u * d);
+  uint16_t* brows = in_big<uint16_t>(P, P.o_brows);
+#pragma unroll 1
+  for (int i = 0; i < nz; ++i)
+    bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[kBarLow]);
   if (!P.dense) {
     const uint32_t code_bytes = (uint32_t)nt * KC * kChunkWords * 4u;
     mbar_arrive_expect_tx(&M.bar[kBarSketch], code_bytes + (uint32_t)nt * kRowTile * 4u);
@@ -774,11 +780,6 @@ __device__ __forceinline__ void issue_expert(const FusedParams& P, int e, int q,
                nt * kRowTile * 4u, &M.bar[kBarSketch]);
     }
   }
-  mbar_arrive_expect_tx(&M.bar[kBarLow], (uint32_t)nz * 2u * d);
-  uint16_t* brows = in_big<uint16_t>(P, P.o_brows);
-#pragma unroll 1
-  for (int i = 0; i < nz; ++i)
-    bulk_g2s(brows + (size_t)i * d, P.lr_b + ((size_t)e * r + q + i * CS) * d, 2u * d, &M.bar[kBarLow]);
   if (r > 0) prefetch_l2(P.lr_a + ((size_t)e * d + (size_t)q * P.slice) * r, 2u * P.slice * r);
 }
 
@@ -812,20 +813,20 @@ __device__ __forceinline__ void push_z(const FusedParams& P, int q, int nz, cons
     const float sw = warp_sum8(v);
     if ((lane & 3) == 0) M.red8[warp][lane >> 2] = sw;
     __syncthreads();
-    if (tid < nb) {
+    if (tid < nb * CS) {  // one thread per (row, destination)
+      const int row = tid / CS, dst = tid - row * CS;
       float acc = 0.f;
 #pragma unroll
-      for (int w = 0; w < kFW; ++w) acc += M.red8[w][tid];
-      const uint32_t za = smem_addr(&M.z[q + (r0 + tid) * CS]);
-#pragma unroll 1
-      for (int dst = 0; dst < CS; ++dst) st_async(mapa(za, dst), __float_as_uint(acc), mapa(rbar, dst));
+      for (int w = 0; w < kFW; ++w) acc += M.red8[w][row];
+      st_async(mapa(smem_addr(&M.z[q + (r0 + row) * CS]), dst), __float_as_uint(acc), mapa(rbar, dst));
     }
     __syncthreads();
   }
 }
 
-// B: the x permutation for scoring; sketch scores of this CTA's rows on the tensor
-// cores, pushed with the warps' largest keys; then z = B_e x rows, pushed.  Returns ok.
+// B: the x permutation for scoring and z = B_e x (pushed) while the sketch tiles fly;
+// then the sketch scores of this CTA's rows on the tensor cores, pushed with the warps'
+// largest keys.  Returns ok.
 template <int IT>
 __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int pr, int nt, int lt0, int nz,
                                           bool ok, const float (&xf)[IT][8]) {
@@ -842,6 +843,13 @@ __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int pr
       const int kc = i >> 5, c = (i >> 3) & 3, q8 = i & 7;
       xperm[i] = x32[kc * 32 + 8 * (q8 >> 1) + c + 4 * (q8 & 1)];
     }
+  }
+  // z = B_e x, pushed, while the sketch tiles are still in flight
+  if (nz > 0) {
+    ok = wait_phase(&M.bar[kBarLow], 0, P.err) && ok;
+    push_z<IT>(P, q, nz, xf);
+  }
+  if (!P.dense) {
     ok = wait_phase(&M.bar[kBarSketch], 0, P.err) && ok;
     __syncthreads();  // xperm complete
     MARK(4);
@@ -852,11 +860,6 @@ __device__ __forceinline__ bool phase_scores(const FusedParams& P, int q, int pr
     MARK(5);
     push_scores(P, M, part, in_big<float>(P, P.o_alpha), in_big<uint32_t>(P, P.o_keys), nt * kRowTile, lt0,
                 pr, q);
-  }
-  // z = B_e x while the scores cross the cluster (B_e rows landed long ago)
-  if (nz > 0) {
-    ok = wait_phase(&M.bar[kBarLow], 0, P.err) && ok;
-    push_z<IT>(P, q, nz, xf);
   }
   return ok;
 }
@@ -1445,7 +1448,7 @@ bool plan(FusedParams& P, const Dims& D, int k, int cs, int limit) {
     const int t0 = qq * P.tpc < ntile_all ? qq * P.tpc : ntile_all;
     const int t1 = t0 + P.tpc < ntile_all ? t0 + P.tpc : ntile_all;
     const int nrows = (t1 - t0) * kRowTile;
-    maxmsgs += (uint32_t)((nrows + 31) / 32);
+    maxmsgs += (uint32_t)((4 * nrows + 31) / 32);  // one max per warp of (row, quarter) items
   }
   P.x1_bytes = 4u * (uint32_t)E;
   P.sc_bytes = P.dense ? 0u : 4u * ((uint32_t)ipad + maxmsgs);
