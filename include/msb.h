@@ -218,12 +218,11 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
 /* The block on activations in host memory, everything enqueued on `stream` (no
  * synchronisation: the host buffers must stay valid, and out_host unread, until the
  * stream has passed the call).
- *  - batch 1 on the single-launch path, with x_host and out_host pinned, mapped into
- *    the current device's address space (cudaHostAlloc / torch pin_memory under
- *    unified addressing) and 16-byte aligned: the kernel itself reads x_host and
- *    writes out_host across
- *    the host link, so consecutive calls keep their launch overlap; the staging
- *    buffers are not touched.
+ *  - batches on the single-launch path (up to 16 tokens) with x_host and out_host
+ *    pinned, mapped into the current device's address space (cudaHostAlloc / torch
+ *    pin_memory under unified addressing) and 16-byte aligned: the kernel itself
+ *    reads x_host and writes out_host across the host link, so consecutive calls
+ *    keep their launch overlap; the staging buffers are not touched.
  *  - otherwise: copies x_host to x_dev, runs moe_sparse_block(x_dev -> out_dev) and
  *    copies out_dev to out_host with cudaMemcpyAsync (pinned memory makes the copies
  *    asynchronous).

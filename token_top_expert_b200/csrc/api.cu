@@ -339,7 +339,7 @@ int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, co
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // pinned, mapped host buffers on the single-launch path: the kernel itself reads x and
   // writes the result across the host link (no copy-engine round trip between launches)
-  if (batch == 1 && !(flags & MSB_FLAG_GENERAL)) {
+  if (batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL)) {
     const void* xm = mapped_address(x_host);
     void* om = const_cast<void*>(mapped_address(out_host));
     if (xm && om && aligned16(xm) && aligned16(om)) {

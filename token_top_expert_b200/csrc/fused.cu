@@ -1560,7 +1560,7 @@ int launch_fused(const uint16_t* x, const uint16_t* router_t, const uint16_t* re
                  const uint16_t* lr_b, uint16_t* out, const Dims& D, uint32_t* err,
                  uint32_t* counters, float* y_acc, const TraceDev& tr, cudaStream_t st, bool x_mapped,
                  bool x_ready, int batch, bool q4) {
-  if (batch < 1 || batch > kFusedMaxBatch || (batch > 1 && (x_mapped || tr.union_count))) return MSB_ENOTFUSED;
+  if (batch < 1 || batch > kFusedMaxBatch || (batch > 1 && tr.union_count)) return MSB_ENOTFUSED;
   FusedParams P{};
   P.q4 = q4 ? 1 : 0;
   P.x_mapped = x_mapped ? 1 : 0;
