@@ -1,36 +1,38 @@
-// Single-launch batch-1 sparse-MoE block (the decode hot path).
+// Single-launch sparse-MoE block for decode batches of up to 16 tokens (the hot path).
 //
-// One 16-CTA thread-block cluster per routed expert.  Every exchange inside a
-// cluster is a one-way push: the producer writes into the consumers' shared memory
-// with st.async / red.async, and each consumer waits on its own mbarrier for the
-// exact byte count it expects, so no exchange costs a cluster-wide barrier.
-// Across clusters only FP32 reduction-adds into a small accumulator meet; the last
-// contribution to an output slice writes it as BF16.
+// One thread-block cluster per (token, routed expert) pair: 16 CTAs for one token, 8
+// for several (so that a batch is resident in about one wave).  Every exchange inside a
+// cluster is a one-way push: the producer writes into the consumers' shared memory with
+// st.async / red.async, and each consumer waits on its own mbarrier for the exact byte
+// count it expects, so no exchange costs a cluster-wide barrier.  Across clusters only
+// FP32 reduction-adds into the token's accumulator row meet; the last contribution to an
+// output slice writes it as BF16.
 //
-//  A  router: each CTA computes E/16 logits x . W_router[e] (rows staged by a
-//     bulk copy before the grid dependency wait) and pushes them to every CTA of
-//     the cluster; every CTA ranks the E logits and cluster c takes the c-th expert.
-//  B  sketch scores: each CTA stages its 16-row tiles of the packed 2-bit sketch,
-//     scores them on the tensor cores (the packed codes are the bf16 A fragment)
-//     and pushes alpha*|T.x| and its largest key to every CTA of the cluster.
-//  C  exact top-k: every CTA selects the same k channels (histogram below the
-//     cluster's largest score, the k-th key's bin ranked directly; ties to the
-//     lower index) and issues bulk copies of its share of the channel records.
-//  D  records: as each 6d-byte record lands, its gate.x and up.x are reduced over
-//     the CTA, h = silu(gate.x) * up.x, and every thread adds h * down over its
-//     8-element groups of the output; z = B_e x (pushed like the scores) and
-//     A_e z on this CTA's output slice run while the records stream.
-//  E  combine: each CTA pushes its partial output, slice by slice, to the slice's
-//     owner; the owner sums the 16 partials, adds A_e z, scales by the router
-//     weight and reduction-adds into the FP32 accumulator; the last of the K
-//     contributions to a slice converts it to BF16 and re-zeroes it.
+//  A  router: each CTA computes its E/cs logits x . W_router[e] (rows staged by bulk
+//     copies before the grid dependency wait) and pushes them to every CTA; the CTA
+//     owning a logit ranks it exactly against all E and pushes the K winners into every
+//     CTA's rank table; cluster c of the token takes its c-th expert.
+//  B  z = B_e x (pushed) while the sketch tiles are in flight; then the sketch scores of
+//     the CTA's 16-row tiles on the tensor cores (the packed codes are the bf16 A
+//     fragment), pushed with one max per warp to every CTA.
+//  C  exact top-k: every CTA selects the same k channels (histogram below the cluster's
+//     largest score, ballot prefixes, the k-th key's bin ranked directly when it is not
+//     taken whole; ties to the lower index); the CTAs interleave over the ascending list
+//     and issue bulk copies of their channel records; A_e z on the CTA's output slice.
+//  D  records in batches as they land (BF16 or 4-bit group-affine records): gate.x and
+//     up.x on the CUDA cores with one transposed warp reduction per batch, h =
+//     silu(gate.x) * up.x, and every thread adds h * down over its 8-element groups.
+//  E  combine: each CTA pushes its partial output, slice by slice, to the slice's owner;
+//     the owner sums the partials, adds A_e z, scales by the router weight and
+//     reduction-adds into the FP32 accumulator; the last of the K contributions to a
+//     slice converts it to BF16 and re-zeroes it.
 //
-// The kernel's code is kept small (rolled loops, rare paths out of line): on B200
-// a kernel whose executed code fits the SM's instruction cache stays warm from one
-// launch to the next, while one that does not pays instruction fetches every launch.
-//
-// The launch uses programmatic stream serialisation: barrier set-up and the router
-// rows' copy run before griddepcontrol.wait, overlapping the previous launch.
+// x comes from device memory (one bulk copy) or, for pinned and mapped host buffers,
+// from the host link (each CTA reads a piece and pushes it to the cluster).  The launch
+// uses programmatic stream serialisation: barrier set-up and the router rows' copy (and
+// x, when the caller declared it ready) run before griddepcontrol.wait.  Every wait is
+// bounded; an expired wait sets the sticky error word and the CTA still takes every
+// exchange and barrier step.
 //
 // "KAIST drops calibration from MoE decoding ...": "Top-k instead of a threshold"
 // (fixed read budget), "A reader built from weights alone" (ternary sketch filter
