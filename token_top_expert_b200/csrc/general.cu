@@ -21,11 +21,13 @@ constexpr int kNT = 256;          // threads per CTA in every general kernel
 constexpr int kRouterTok = 8;     // tokens per router CTA
 constexpr int kScoreRows = 64;    // sketch rows per score CTA (4 tensor-core row tiles)
 constexpr int kScoreTok = 8;      // tokens per MMA n-tile
-constexpr int kLrRows = 256;      // A_e rows per low-rank work item
+constexpr int kLrPass = 4;        // low-rank work item: passes of kNT / qs rows of A_e
+static_assert(MSB_MAX_RANK % 8 == 0 && (MSB_MAX_RANK & (MSB_MAX_RANK - 1)) == 0,
+              "the low-rank z stride 8 qs must fit 8 * MSB_MAX_RANK floats per token group");
 constexpr int kGCh = 8;           // gather: channels per stage at most (one m-tile of gate/up rows)
 constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in flight)
 constexpr int kGRunStages = 8;    // gather: stages per work item at most
-constexpr int kGAccTiles = 32;    // gather: output column tiles per warp held in registers
+constexpr int kGAccTiles = 16;    // gather: 16-column output tiles per warp held in registers
 
 // =====================================================================================
 // router
@@ -472,6 +474,8 @@ __global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch
 struct GatherCfg {
   int ch;       // channels per work item (<= kGCh)
   int nlr;      // low-rank work items per slot
+  int lr_qs;    // low-rank: 8-element pieces per row of A_e, rounded up to a power of two
+  int lr_vec;   // low-rank: rows are 16-byte aligned (r % 8 == 0)
   int dense;    // 1: every channel is selected (no sketch)
   uint64_t wait_ns;  // bounded-wait limit
 #ifdef MSB_INSTRUMENTED
@@ -501,21 +505,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
          ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(hi)) << 16);
 }
 
-// Issue the bulk copies of channels run[c0 .. c0 + n) (shared memory) into a stage buffer.
-// The stage's channel list into `list` and (copy) the bulk copies of its records.  The
-// list is always written: the consumer reads it whether or not the copies were issued.
+// Reduction-add of one down tile D[16 columns][8 tokens] (columns m0 + row, the mma.sync
+// accumulator layout) into the FP32 accumulator y[token][column].  Lanes g and g ^ 1 of a
+// column pair swap one value so that each lane adds two adjacent columns of one token;
+// `hi`: rows 8-15 are real columns too.
+__device__ __forceinline__ void gather_red_tile(float* y, const int* s_tok, int ntg, int d, int m0,
+                                                const float (&acc)[4], int lane, bool hi) {
+  const int g8 = lane >> 2, c4 = lane & 3;
+  const bool odd = g8 & 1;
+  const int t = 2 * c4 + (odd ? 1 : 0);  // token of this lane's pair after the swap
+  const int col = m0 + (g8 & ~1);
+  const float s0 = __shfl_xor_sync(0xffffffffu, odd ? acc[0] : acc[1], 4);
+  const float s1 = __shfl_xor_sync(0xffffffffu, odd ? acc[2] : acc[3], 4);
+  if (t < ntg) {
+    float* row = y + (size_t)s_tok[t] * d + col;
+    red_add_v2(row, odd ? s0 : acc[0], odd ? acc[1] : s0);
+    if (hi) red_add_v2(row + 8, odd ? s1 : acc[2], odd ? acc[3] : s1);
+  }
+}
+
+// One warp issues a stage: the channel list of run[c0 .. c0 + n) (shared memory) into
+// `list` and (copy) the bulk copies of their records into a stage buffer, lane i taking
+// channel i (n <= 32).  The list is always written: the consumer reads it whether or not
+// the copies were issued.
 __device__ __forceinline__ void gather_issue(uint16_t* buf, const uint16_t* records, const int* run,
                                              int e, int c0, int n, int d, int I, int* list,
                                              uint64_t* bar, bool copy = true) {
-  const int rs = 3 * d + 8;
-  if (copy) {
+  const int lane = threadIdx.x & 31;
+  if (copy && lane == 0) {
     fence_proxy_async();
     mbar_arrive_expect_tx(bar, 6u * d * n);
   }
-  for (int i = 0; i < n; ++i) {
-    const int j = run[c0 + i];
-    list[i] = j;
-    if (copy) bulk_g2s(buf + (size_t)i * rs, records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
+  __syncwarp();
+  if (lane < n) {
+    const int j = run[c0 + lane];
+    list[lane] = j;
+    if (copy) bulk_g2s(buf + (size_t)lane * (3 * d + 8), records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
   }
 }
 
@@ -538,6 +563,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   __shared__ float s_w[8];
   __shared__ float s_red[kNT / 32][16][8];
   __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels >= ch zero
+  __shared__ __align__(16) float s_lz[8 * MSB_MAX_RANK];  // low-rank: [token][8 qs] z times weight
+  __shared__ int s_ltok[8];
   // slot tables, copied once: run offsets, union sizes, experts, pair offsets
   __shared__ int s_coff[MSB_MAX_EXPERTS + 1], s_ucnt[MSB_MAX_EXPERTS], s_se[MSB_MAX_EXPERTS],
       s_so[MSB_MAX_EXPERTS + 1];
@@ -569,8 +596,10 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   const int c4 = lane & 3, g8 = lane >> 2;
   const int KS = d / 16;
   const int ks0 = warp * KS / (kNT / 32), ks1 = (warp + 1) * KS / (kNT / 32);
-  const int NTW = d / 64;  // 8-column output tiles per warp
-  const int nt0 = warp * NTW;
+  // down columns of this warp: [c0w, c0w + d / 8), NT16 tiles of 16 and one of 8 if d / 64 is odd
+  const int c0w = warp * (d / 8);
+  const int NT16 = d / 128;
+  const bool tail8 = (d / 64) & 1;
   const int nmw = mask_words(ipad);
   // h step ownership: thread tid < 8 * CH takes (token tid / CH, channel tid % CH)
   const int hc = tid % CH, ht = tid / CH;
@@ -602,19 +631,72 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
     if (item >= nitems || !ok) break;
 
     // ----------------------------------------------------------- low-rank item
+    // kLrPass passes of kNT / qs rows of A_e: thread (row, piece) holds 8 elements of the
+    // row per pass (one 16-byte load when r % 8 == 0), all loads issued before the
+    // tokens' z (times the router weight) are staged in shared memory 8 tokens at a time;
+    // the row's pieces meet by shuffles and lane `piece` adds tokens piece, piece + qs, ...
     if (item >= nchunks) {
       const int q = item - nchunks, u = q / cfg.nlr;
-      const int row = (q - u * cfg.nlr) * kLrRows + tid;
       const int e = s_se[u];
       const int off = s_so[u], cnt = s_so[u + 1] - off;
-      if (row < d && r > 0) {
-        const uint16_t* arow = lr_a + ((size_t)e * d + row) * r;
-        for (int ti = 0; ti < cnt; ++ti) {
-          const int p = off + ti;
-          const float* z = ws.z + (size_t)p * r;
-          float acc = 0.f;
-          for (int qq = 0; qq < r; ++qq) acc = fmaf(bf16_lo(arow[qq]), __ldcg(z + qq), acc);
-          atomicAdd(&ws.y_acc[(size_t)ws.pair_tok[p] * d + row], ws.pair_w[p] * acc);
+      const int qs = cfg.lr_qs, zs = 8 * qs;  // pieces per row (a power of two), z stride
+      const int rpp = kNT / qs;               // rows per pass
+      const int lrow = tid / qs, piece = tid - lrow * qs;
+      const int row0 = (q - u * cfg.nlr) * (kLrPass * rpp);
+      uint4 av[kLrPass];
+#pragma unroll
+      for (int ps = 0; ps < kLrPass; ++ps) {
+        const int row = row0 + ps * rpp + lrow;
+        av[ps] = make_uint4(0u, 0u, 0u, 0u);
+        if (row < d && piece * 8 < r) {
+          const uint16_t* src = lr_a + ((size_t)e * d + row) * r + piece * 8;
+          if (cfg.lr_vec) {
+            av[ps] = __ldg(reinterpret_cast<const uint4*>(src));
+          } else {
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              if (piece * 8 + i < r) w[i >> 1] |= (uint32_t)__ldg(src + i) << (16 * (i & 1));
+            av[ps] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      for (int tg = 0; tg < cnt; tg += 8) {
+        const int ntg = min(8, cnt - tg);
+        if (tg > 0) __syncthreads();  // the previous group's reads of s_lz
+        for (int i = tid; i < 8 * zs; i += kNT) {
+          const int t = i / zs, c = i - t * zs;
+          float v = 0.f;
+          if (t < ntg && c < r) v = __ldcg(ws.z + (size_t)(off + tg + t) * r + c) * ws.pair_w[off + tg + t];
+          s_lz[i] = v;
+        }
+        if (tid < 8) s_ltok[tid] = tid < ntg ? ws.pair_tok[off + tg + tid] : 0;
+        __syncthreads();
+#pragma unroll
+        for (int ps = 0; ps < kLrPass; ++ps) {
+          const int row = row0 + ps * rpp + lrow;
+          const uint32_t aw[4] = {av[ps].x, av[ps].y, av[ps].z, av[ps].w};
+          float acc[8];
+#pragma unroll
+          for (int t = 0; t < 8; ++t) {
+            const float4 z0 = *reinterpret_cast<const float4*>(s_lz + t * zs + piece * 8);
+            const float4 z1 = *reinterpret_cast<const float4*>(s_lz + t * zs + piece * 8 + 4);
+            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              a = fmaf(__uint_as_float(aw[i] << 16), zz[2 * i], a);
+              a = fmaf(__uint_as_float(aw[i] & 0xffff0000u), zz[2 * i + 1], a);
+            }
+            acc[t] = a;
+          }
+          for (int o = 1; o < qs; o <<= 1)
+#pragma unroll
+            for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+          if (row < d)
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              if ((t & (qs - 1)) == piece && t < ntg) atomicAdd(&ws.y_acc[(size_t)s_ltok[t] * d + row], acc[t]);
         }
       }
       continue;
@@ -638,7 +720,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         s_tok[tid] = ws.pair_tok[p];
         s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
       }
-      if (tid == 0)  // fill: stages 0 .. kGBufs - 2
+      if (warp == 0)  // fill: stages 0 .. kGBufs - 2
         for (int st = 0; st < min(kGBufs - 1, nst); ++st) {
           bool copy = true;
 #ifdef MSB_INSTRUMENTED
@@ -657,15 +739,11 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
           xb[i][0] = __ldg(xrow + (ks0 + i) * 8 + c4);
           xb[i][1] = __ldg(xrow + (ks0 + i) * 8 + 4 + c4);
         }
-      // selection bit of this thread's (token, channel) in stage 0
-      uint32_t selw = 1u;
-      if (!cfg.dense && tid < 8 * CH && ht < ntg && hc < min(CH, nrun)) {
-        const int j = s_list[0][hc];
-        selw = __ldcg(&ws.selmask[(size_t)(off + tg0 + ht) * nmw + (j >> 5)]) >> (j & 31);
-      }
-      float yacc[REGACC ? kGAccTiles : 1][2];
+      float yacc[REGACC ? kGAccTiles : 1][4];
 #pragma unroll
-      for (int i = 0; i < (REGACC ? kGAccTiles : 1); ++i) { yacc[i][0] = 0.f; yacc[i][1] = 0.f; }
+      for (int i = 0; i < (REGACC ? kGAccTiles : 1); ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) yacc[i][j] = 0.f;
 
 #pragma unroll 1
       for (int stg = 0; stg < nst; ++stg) {
@@ -673,7 +751,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         const int nch = min(CH, nrun - stg * CH);
         // keep kGBufs - 1 stages in flight: stage stg + kGBufs - 1 goes into the buffer
         // that stage stg - 1 has just released
-        if (tid == 0 && stg + kGBufs - 1 < nst) {
+        if (warp == 0 && stg + kGBufs - 1 < nst) {
           const int sn = stg + kGBufs - 1, bn = sn % kGBufs;
           gather_issue(buf0 + bn * bstride, records, s_run, e, sn * CH, min(CH, nrun - sn * CH), d, I,
                        s_list[bn], &bar[bn]);
@@ -686,6 +764,13 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
           break;
         }
         phases ^= 1u << b;
+        // selection bit of this thread's (token, channel), loaded here so that its latency
+        // overlaps gate/up (the stage's list was written before the barrier above)
+        uint32_t selw = 1u;
+        if (!cfg.dense && tid < 8 * CH && ht < ntg && hc < nch) {
+          const int j = s_list[b][hc];
+          selw = __ldcg(&ws.selmask[(size_t)(off + tg0 + ht) * nmw + (j >> 5)]) >> (j & 31);
+        }
         const uint16_t* rec = buf0 + b * bstride;
         // gate/up ldmatrix row: channel lane % 8 (channels past nch read channel 0;
         // their rows are dropped), gate (lanes 0-7, 16-23) or up, k offset 8 (lane / 16)
@@ -693,8 +778,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         uint32_t a_addr =
             smem_addr(rec + (size_t)gch * rs + ((lane >> 3) & 1) * d + 8 * (lane >> 4)) + 32u * ks0;
         // down ldmatrix.trans row: channel lane % 8 (channels past nch read channel 0;
-        // their h is zero), element block 8 (lane / 16)
-        const uint32_t b_base = smem_addr(rec + (size_t)gch * rs + 2 * d + 8 * (lane >> 4));
+        // their h is zero); lane / 8 picks the 8-column block
+        const uint32_t b_base = smem_addr(rec + (size_t)gch * rs + 2 * d);
         // ---- gate/up partials over this warp's k-steps
         {
           float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -746,72 +831,74 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
             h = silu(g) * uu * s_w[ht];
           }
           s_h[ht][hc] = h;
-          // the next stage's selection bit (its list was written when it was issued)
-          selw = 1u;
-          if (!cfg.dense && stg + 1 < nst && ht < ntg && hc < min(CH, nrun - (stg + 1) * CH)) {
-            const int j = s_list[(stg + 1) % kGBufs][hc];
-            selw = __ldcg(&ws.selmask[(size_t)(off + tg0 + ht) * nmw + (j >> 5)]) >> (j & 31);
-          }
         }
         __syncthreads();
-        // ---- down: A = [h_hi ; h_lo] (token rows), B = down columns, this warp's column tiles
+        // ---- down: D[16 columns][8 tokens] += A x B with A = this warp's down columns
+        // (rows) over k = [channels 0-7 | channels 0-7 again] and B = [h_hi ; h_lo] of the
+        // tokens, so that one MMA carries both halves of h
         const float2 hp = *reinterpret_cast<const float2*>(&s_h[g8][2 * c4]);
-        const uint32_t ahi = pack_bf16x2(hp.x, hp.y);
-        const float hx = __uint_as_float(ahi << 16), hy = __uint_as_float(ahi & 0xffff0000u);
-        const uint32_t alo = pack_bf16x2(hp.x - hx, hp.y - hy);
+        const uint32_t hhi = pack_bf16x2(hp.x, hp.y);
+        const float hx = __uint_as_float(hhi << 16), hy = __uint_as_float(hhi & 0xffff0000u);
+        const uint32_t hlo = pack_bf16x2(hp.x - hx, hp.y - hy);
         if (REGACC) {
+          // (register indices stay compile-time: the tile loop is unrolled)
 #pragma unroll
-          for (int nt = 0; nt < kGAccTiles; nt += 2) {
-            if (nt < NTW) {
-              const int m0 = (nt0 + nt) * 8;
-              uint32_t b0, b1, b2, b3;
-              if (nt + 1 < NTW) {
-                ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
-              } else {
-                ldsm_x2_t(b_base + 2u * m0, b0, b1);
-                b2 = b0; b3 = b1;
+          for (int t = 0; t < kGAccTiles; t += 2) {
+            const int m0 = c0w + 16 * t;
+            if (t + 1 < NT16) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(b_base + 2u * (m0 + 8 * (lane >> 3)), a0, a1, a2, a3);
+              mma_bf16(yacc[t], a0, a1, a0, a1, hhi, hlo);
+              mma_bf16(yacc[t + 1], a2, a3, a2, a3, hhi, hlo);
+            } else if (t < NT16) {  // one 16-column tile, then perhaps 8 columns
+              uint32_t a0, a1;
+              ldsm_x2_t(b_base + 2u * (m0 + 8 * ((lane >> 3) & 1)), a0, a1);
+              mma_bf16(yacc[t], a0, a1, a0, a1, hhi, hlo);
+              if (tail8) {
+                ldsm_x2_t(b_base + 2u * (m0 + 16), a0, a1);
+                mma_bf16(yacc[t + 1], a0, a0, a0, a0, hhi, hlo);
               }
-              float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
-              mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
-              yacc[nt][0] += dA[0] + dA[2];
-              yacc[nt][1] += dA[1] + dA[3];
-              yacc[nt + 1][0] += dB[0] + dB[2];
-              yacc[nt + 1][1] += dB[1] + dB[3];
+            } else if (t == NT16 && tail8) {  // 8 columns: rows 8-15 repeat rows 0-7, dropped
+              uint32_t a0, a1;
+              ldsm_x2_t(b_base + 2u * m0, a0, a1);
+              mma_bf16(yacc[t], a0, a0, a0, a0, hhi, hlo);
             }
           }
         } else {
-          float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
-          const bool tok_ok = g8 < ntg;
-          int nt = 0;
-          for (; nt + 2 <= NTW; nt += 2) {
-            const int m0 = (nt0 + nt) * 8;
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(b_base + 2u * m0, b0, b1, b2, b3);
+          int t = 0;
+          for (; t + 2 <= NT16; t += 2) {
+            const int m0 = c0w + 16 * t;
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_t(b_base + 2u * (m0 + 8 * (lane >> 3)), a0, a1, a2, a3);
             float dA[4] = {0.f, 0.f, 0.f, 0.f}, dB[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
-            mma_bf16(dB, ahi, alo, 0u, 0u, b2, b3);
-            if (tok_ok) {
-              red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
-              red_add_v2(yrow + m0 + 8 + 2 * c4, dB[0] + dB[2], dB[1] + dB[3]);
-            }
+            mma_bf16(dA, a0, a1, a0, a1, hhi, hlo);
+            mma_bf16(dB, a2, a3, a2, a3, hhi, hlo);
+            gather_red_tile(ws.y_acc, s_tok, ntg, d, m0, dA, lane, true);
+            gather_red_tile(ws.y_acc, s_tok, ntg, d, m0 + 16, dB, lane, true);
           }
-          if (nt < NTW) {
-            const int m0 = (nt0 + nt) * 8;
-            uint32_t b0, b1;
-            ldsm_x2_t(b_base + 2u * m0, b0, b1);
+          if (t < NT16) {
+            const int m0 = c0w + 16 * t;
+            uint32_t a0, a1;
+            ldsm_x2_t(b_base + 2u * (m0 + 8 * ((lane >> 3) & 1)), a0, a1);
             float dA[4] = {0.f, 0.f, 0.f, 0.f};
-            mma_bf16(dA, ahi, alo, 0u, 0u, b0, b1);
-            if (tok_ok) red_add_v2(yrow + m0 + 2 * c4, dA[0] + dA[2], dA[1] + dA[3]);
+            mma_bf16(dA, a0, a1, a0, a1, hhi, hlo);
+            gather_red_tile(ws.y_acc, s_tok, ntg, d, m0, dA, lane, true);
+          }
+          if (tail8) {
+            uint32_t a0, a1;
+            ldsm_x2_t(b_base + 2u * (c0w + 16 * NT16), a0, a1);
+            float dA[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16(dA, a0, a0, a0, a0, hhi, hlo);
+            gather_red_tile(ws.y_acc, s_tok, ntg, d, c0w + 16 * NT16, dA, lane, false);
           }
         }
         __syncthreads();  // this stage's buffer, s_red and s_h are free
       }
-      if (REGACC && ok && g8 < ntg) {  // one reduction-add per output of the run
-        float* yrow = ws.y_acc + (size_t)s_tok[g8] * d;
+      if (REGACC && ok) {  // one reduction-add per output of the run
 #pragma unroll
-        for (int nt = 0; nt < kGAccTiles; ++nt)
-          if (nt < NTW) red_add_v2(yrow + (nt0 + nt) * 8 + 2 * c4, yacc[nt][0], yacc[nt][1]);
+        for (int t = 0; t < kGAccTiles; ++t)
+          if (t < NT16 + (tail8 ? 1 : 0))
+            gather_red_tile(ws.y_acc, s_tok, ntg, d, c0w + 16 * t, yacc[t], lane, t < NT16);
       }
     }
   }
@@ -890,7 +977,13 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
   GatherCfg cfg;
   cfg.ch = max(1, min(kGCh, (196 * 1024 / kGBufs) / (6 * d + 16)));
-  cfg.nlr = D.rank > 0 ? (d + kLrRows - 1) / kLrRows : 0;
+  cfg.lr_qs = 1;
+  while (cfg.lr_qs * 8 < D.rank) cfg.lr_qs *= 2;
+  cfg.lr_vec = D.rank % 8 == 0;
+  {
+    const int rows = kLrPass * (kNT / cfg.lr_qs);
+    cfg.nlr = D.rank > 0 ? (d + rows - 1) / rows : 0;
+  }
   cfg.dense = dense;
   cfg.wait_ns = kWaitLimitNs;
 #ifdef MSB_INSTRUMENTED
