@@ -65,3 +65,18 @@ def test_widest_hidden_size(msb, batch, general):
     assert (g["sel_count"] == w.k).all()
     check_union(g, w.top_e)
     print(batch, general, compare(x, g, lay, w.top_e, w.k))
+
+
+@pytest.mark.parametrize("rank", [8, 12, 128])
+def test_low_rank_term_ranks(msb, rank):
+    """A_e z on the multi-kernel path for ranks whose rows of A_e are 16-byte multiples
+    (staged through shared memory: 8, and 128, the largest accepted) and one that is not
+    (12: read from registers)."""
+    w = synth.TINY.with_(name="tiny_r%d" % rank, rank=rank)
+    dev = device_layer(w)
+    assert msb.path_info(dev.dims, 24, w.k)["path"] != "single_launch"
+    lay = oracle.SynthLayer(w)
+    x = synth.activations(w, 19, batch=24)
+    g = run_gpu(x, dev, w.k)
+    assert (g["sel_count"] == w.k).all()
+    print(rank, compare(x, g, lay, w.top_e, w.k, rank=rank, tokens=_sampled(24)))

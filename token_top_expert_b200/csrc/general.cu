@@ -19,6 +19,7 @@ namespace msb {
 
 constexpr int kNT = 256;          // threads per CTA in every general kernel
 constexpr int kRouterTok = 8;     // tokens per router CTA
+constexpr int kRouterExp = 8;     // experts per router CTA
 constexpr int kScoreRows = 64;    // sketch rows per score CTA (4 tensor-core row tiles)
 constexpr int kScoreTok = 8;      // tokens per MMA n-tile
 constexpr int kLrPass = 4;        // low-rank work item: passes of kNT / qs rows of A_e
@@ -48,26 +49,42 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
       for (int c = c0 + threadIdx.x; c < c1; c += kNT) ws.y_acc[(size_t)(t0 + t) * d + c] = 0.f;
   }
 
-  const int e = blockIdx.x * (kNT / 32) + warp;
-  if (e < E) {
-    float acc[kRouterTok];
+  // logits of this CTA's 8 experts for its tokens: thread i takes the 16-byte groups
+  // i, i + kNT, ... of d for every (expert, token), so that each row of the router and of
+  // x is read once; the 64 partial sums meet across the warp (transposed) and the warps
+  {
+    const int e0 = blockIdx.x * kRouterExp;
+    float acc[kRouterExp * kRouterTok];
 #pragma unroll
-    for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
-    const uint4* wrow = reinterpret_cast<const uint4*>(router_t + (size_t)e * d);
-#pragma unroll 8
-    for (int i = lane; i < d / 8; i += 32) {
-      const uint4 wv = __ldg(wrow + i);
+    for (int i = 0; i < kRouterExp * kRouterTok; ++i) acc[i] = 0.f;
+    for (int v = threadIdx.x; v < d / 8; v += kNT) {
+      uint4 wv[kRouterExp], xv[kRouterTok];
+#pragma unroll
+      for (int i = 0; i < kRouterExp; ++i)
+        wv[i] = e0 + i < E ? __ldg(reinterpret_cast<const uint4*>(router_t + (size_t)(e0 + i) * d) + v)
+                           : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int t = 0; t < kRouterTok; ++t)
-        if (t < nt) {
-          const uint4 xv = __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d) + i);
-          acc[t] = dot8(wv, xv, acc[t]);
-        }
-    }
+        xv[t] = t < nt ? __ldg(reinterpret_cast<const uint4*>(x + (size_t)(t0 + t) * d) + v)
+                       : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int t = 0; t < kRouterTok; ++t) {
-      const float s = warp_sum(acc[t]);
-      if (t < nt && lane == 0) ws.logits[(size_t)(t0 + t) * E + e] = s;
+      for (int i = 0; i < kRouterExp; ++i)
+#pragma unroll
+        for (int t = 0; t < kRouterTok; ++t) acc[i * kRouterTok + t] = dot8(wv[i], xv[t], acc[i * kRouterTok + t]);
+    }
+    warp_sum_transposed(acc, lane);  // lane l: totals of (expert, token) 2l and 2l + 1
+    __shared__ float2 s_part[kNT / 32][32];
+    s_part[warp][lane] = make_float2(acc[0], acc[1]);
+    __syncthreads();
+    if (threadIdx.x < kRouterExp * kRouterTok) {
+      const int q = threadIdx.x, i = q / kRouterTok, t = q % kRouterTok;
+      float sum = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNT / 32; ++w) {
+        const float2 pp = s_part[w][q >> 1];
+        sum += (q & 1) ? pp.y : pp.x;
+      }
+      if (e0 + i < E && t < nt) ws.logits[(size_t)(t0 + t) * E + e0 + i] = sum;
     }
   }
 
@@ -214,14 +231,34 @@ __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict_
 // =====================================================================================
 // sketch scores (tensor cores) and z = B_e x
 // =====================================================================================
+// One 64-column chunk of a 16-row tile: the codes pair w (2 bits per weight, placed at
+// the sign and exponent bits of a BF16 +-2 or 0) x the staged x fragments, into sum.
+__device__ __forceinline__ void score_chunk(uint2 w, const uint32_t* xp, float (&sum)[4]) {
+  const uint4 xa = *reinterpret_cast<const uint4*>(xp);
+  const uint4 xb = *reinterpret_cast<const uint4*>(xp + 4);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  mma_bf16(acc, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
+           (w.y << 2) & kSketchMask, xa.x, xa.y);
+  mma_bf16(acc, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
+           (w.y << 6) & kSketchMask, xa.z, xa.w);
+  mma_bf16(acc, (w.x << 8) & kSketchMask, (w.y << 8) & kSketchMask, (w.x << 10) & kSketchMask,
+           (w.y << 10) & kSketchMask, xb.x, xb.y);
+  mma_bf16(acc, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask,
+           (w.x << 14) & kSketchMask, (w.y << 14) & kSketchMask, xb.z, xb.w);
+  sum[0] += acc[0];
+  sum[1] += acc[1];
+  sum[2] += acc[2];
+  sum[3] += acc[3];
+}
+
 // Dynamic shared memory: xperm [kScoreTok][KC*32 + 4] uint32, then part [4][64] floats.
 // xperm holds, per token n, chunk kc and lane column c, the eight bf16 pairs
 // (s, p) = B-fragment registers of the four 16-column steps of that chunk.
-__global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__ x,
+__global__ void __launch_bounds__(kNT, 3) score_kernel(const uint16_t* __restrict__ x,
                                                     const uint32_t* __restrict__ sketch,
                                                     const float* __restrict__ alpha,
                                                     const uint16_t* __restrict__ lr_b, Dims D,
-                                                    Workspace ws, TraceDev tr, int z_only) {
+                                                    Workspace ws, TraceDev tr, int nsb) {
   extern __shared__ __align__(16) uint32_t smem[];
   const int u = blockIdx.y;
   if (u >= *ws.nused) return;
@@ -234,25 +271,33 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
   uint32_t* xperm = smem;
   float* part = reinterpret_cast<float*>(smem + kScoreTok * xstride);
 
-  // ---- z = B_e x for the rows of this CTA (row rho handled by CTA rho % gridDim.x)
-  if (D.rank > 0) {
-    for (int item = warp; ; item += kNT / 32) {
-      const int per = cnt;
-      const int local = item / per, ti = item % per;
-      const int rho = blockIdx.x + local * gridDim.x;
-      if (rho >= D.rank) break;
-      const int p = off + ti;
-      const int t = ws.pair_tok[p];
-      const uint4* brow = reinterpret_cast<const uint4*>(lr_b + ((size_t)e * D.rank + rho) * d);
-      const uint4* xr = reinterpret_cast<const uint4*>(x + (size_t)t * d);
-      float acc = 0.f;
-#pragma unroll 8
-      for (int i = lane; i < d / 8; i += 32) acc = dot8(__ldg(brow + i), __ldg(xr + i), acc);
-      acc = warp_sum(acc);
-      if (lane == 0) ws.z[(size_t)p * D.rank + rho] = acc;
+  // ---- CTAs nsb.. of a slot: z = B_e x, one row of B_e per warp, 4 tokens at a time (they
+  // run beside the score CTAs instead of ahead of them)
+  if ((int)blockIdx.x >= nsb) {
+    const int rho = ((int)blockIdx.x - nsb) * (kNT / 32) + warp;
+    if (rho >= D.rank) return;
+    const uint4* brow = reinterpret_cast<const uint4*>(lr_b + ((size_t)e * D.rank + rho) * d);
+    for (int tq = 0; tq < cnt; tq += 4) {
+      const int n = min(4, cnt - tq);
+      const uint4* xr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        xr[j] = reinterpret_cast<const uint4*>(x + (size_t)ws.pair_tok[off + tq + min(j, n - 1)] * d);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int i = lane; i < d / 8; i += 32) {
+        const uint4 bv = __ldg(brow + i);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = dot8(bv, __ldg(xr[j] + i), acc[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float v = warp_sum(acc[j]);
+        if (lane == 0 && j < n) ws.z[(size_t)(off + tq + j) * D.rank + rho] = v;
+      }
     }
+    return;
   }
-  if (z_only) return;
 
   const int tile0 = blockIdx.x * (kScoreRows / kRowTile);
   const int ntiles = min(kScoreRows / kRowTile, ipad / kRowTile - tile0);
@@ -261,6 +306,17 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
   const int kc0 = kh ? KC / 2 : 0, kc1 = kh ? KC : KC / 2;
   const uint2* codes =
       reinterpret_cast<const uint2*>(sketch) + ((size_t)(e * (ipad / kRowTile) + tile0 + rt) * KC) * 32 + lane;
+
+  // this warp's codes (chunks kc0 .. kc1 of its tile, contiguous) are brought into L2 and
+  // its rows' alpha loaded before x is staged, so that the latencies overlap
+  if (rt < ntiles && lane == 0)
+    prefetch_l2(codes - lane + (size_t)kc0 * 32, (uint32_t)(kc1 - kc0) * 32u * 8u);
+  float al[2] = {0.f, 0.f};
+  if (kh == 0 && rt < ntiles) {
+    const int row0 = (tile0 + rt) * kRowTile + g;
+    al[0] = __ldg(alpha + (size_t)e * ipad + row0);
+    al[1] = __ldg(alpha + (size_t)e * ipad + row0 + 8);
+  }
 
   __shared__ int s_tk[kScoreTok];
   for (int tt = 0; tt < cnt; tt += kScoreTok) {
@@ -289,24 +345,7 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
     if (rt < ntiles) {
       const uint32_t* xp = xperm + g * xstride + c * 8;
 #pragma unroll 8
-      for (int kc = kc0; kc < kc1; ++kc) {
-        const uint2 w = __ldg(codes + (size_t)kc * 32);
-        const uint4 xa = *reinterpret_cast<const uint4*>(xp + kc * 32);
-        const uint4 xb = *reinterpret_cast<const uint4*>(xp + kc * 32 + 4);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16(acc, w.x & kSketchMask, w.y & kSketchMask, (w.x << 2) & kSketchMask,
-                 (w.y << 2) & kSketchMask, xa.x, xa.y);
-        mma_bf16(acc, (w.x << 4) & kSketchMask, (w.y << 4) & kSketchMask, (w.x << 6) & kSketchMask,
-                 (w.y << 6) & kSketchMask, xa.z, xa.w);
-        mma_bf16(acc, (w.x << 8) & kSketchMask, (w.y << 8) & kSketchMask, (w.x << 10) & kSketchMask,
-                 (w.y << 10) & kSketchMask, xb.x, xb.y);
-        mma_bf16(acc, (w.x << 12) & kSketchMask, (w.y << 12) & kSketchMask,
-                 (w.x << 14) & kSketchMask, (w.y << 14) & kSketchMask, xb.z, xb.w);
-        sum[0] += acc[0];
-        sum[1] += acc[1];
-        sum[2] += acc[2];
-        sum[3] += acc[3];
-      }
+      for (int kc = kc0; kc < kc1; ++kc) score_chunk(__ldg(codes + (size_t)kc * 32), xp + kc * 32, sum);
     }
     // combine the two k-halves: kh == 1 writes, kh == 0 adds
     if (kh == 1 && rt < ntiles) {
@@ -324,7 +363,7 @@ __global__ void __launch_bounds__(kNT) score_kernel(const uint16_t* __restrict__
         const int row = row0 + (i >> 1) * 8;
         if (n < ntok) {
           const int p = off + tt + n;
-          const float s = __ldg(alpha + (size_t)e * ipad + row) * fabsf(sum[i]) * 0.5f;
+          const float s = al[i >> 1] * fabsf(sum[i]) * 0.5f;
           ws.scores[(size_t)p * ipad + row] = s;
           if (tr.scores) {
             const int t = ws.pair_tok[p];
@@ -476,6 +515,7 @@ struct GatherCfg {
   int nlr;      // low-rank work items per slot
   int lr_qs;    // low-rank: 8-element pieces per row of A_e, rounded up to a power of two
   int lr_vec;   // low-rank: rows are 16-byte aligned (r % 8 == 0)
+  int lr_rows;  // low-rank: rows of A_e per item copied into a stage buffer (0: registers)
   int dense;    // 1: every channel is selected (no sketch)
   uint64_t wait_ns;  // bounded-wait limit
 #ifdef MSB_INSTRUMENTED
@@ -524,6 +564,33 @@ __device__ __forceinline__ void gather_red_tile(float* y, const int* s_tok, int 
   }
 }
 
+// acc[t] = (8 bf16 of a row of A_e) . z[t][0..8) for the 8 tokens of a group, z at stride zs
+__device__ __forceinline__ void gather_lr_dot(uint4 av, const float* z, int zs, float (&acc)[8]) {
+  const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float4 z0 = *reinterpret_cast<const float4*>(z + t * zs);
+    const float4 z1 = *reinterpret_cast<const float4*>(z + t * zs + 4);
+    const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+    float a = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a = fmaf(__uint_as_float(aw[i] << 16), zz[2 * i], a);
+      a = fmaf(__uint_as_float(aw[i] & 0xffff0000u), zz[2 * i + 1], a);
+    }
+    acc[t] = a;
+  }
+}
+
+// Thread 0 copies rows [row0, row0 + nrow) of A_e (r bf16 each, r % 8 == 0) into `buf`.
+__device__ __forceinline__ void gather_lr_issue(uint16_t* buf, const uint16_t* lr_a, int e, int row0,
+                                                int nrow, int d, int r, uint64_t* bar) {
+  const uint32_t bytes = (uint32_t)nrow * 2u * (uint32_t)r;
+  fence_proxy_async();
+  mbar_arrive_expect_tx(bar, bytes);
+  bulk_g2s(buf, lr_a + ((size_t)e * d + row0) * r, bytes, bar);
+}
+
 // One warp issues a stage: the channel list of run[c0 .. c0 + n) (shared memory) into
 // `list` and (copy) the bulk copies of their records into a stage buffer, lane i taking
 // channel i (n <= 32).  The list is always written: the consumer reads it whether or not
@@ -565,6 +632,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   __shared__ __align__(16) float s_h[8][2 * kGCh];  // [token][channel], channels >= ch zero
   __shared__ __align__(16) float s_lz[8 * MSB_MAX_RANK];  // low-rank: [token][8 qs] z times weight
   __shared__ int s_ltok[8];
+  __shared__ int s_lr_next[2];
   // slot tables, copied once: run offsets, union sizes, experts, pair offsets
   __shared__ int s_coff[MSB_MAX_EXPERTS + 1], s_ucnt[MSB_MAX_EXPERTS], s_se[MSB_MAX_EXPERTS],
       s_so[MSB_MAX_EXPERTS + 1];
@@ -630,8 +698,85 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
     const int item = s_item;
     if (item >= nitems || !ok) break;
 
+    // ----------------------------------------------------------- low-rank items, staged
+    // Every later item is a low-rank item too, so the CTA stays here: thread 0 copies the
+    // next item's rows of A_e (cfg.lr_rows rows of r bf16, contiguous) into the other stage
+    // buffer while the current item is computed from shared memory.
+    if (item >= nchunks && cfg.lr_rows > 0) {
+      const int qs = cfg.lr_qs, zs = 8 * qs, rpp = kNT / qs;
+      const int lrow = tid / qs, piece = tid - lrow * qs;
+      const int R = cfg.lr_rows;
+      const uint32_t rowb = 2u * (uint32_t)r;
+      int cur = item, bsel = 0, par = 0;
+      if (tid == 0) {
+        const int q = cur - nchunks, u = q / cfg.nlr, row0 = (q - u * cfg.nlr) * R;
+        gather_lr_issue(buf0, lr_a, s_se[u], row0, min(R, d - row0), d, r, &bar[0]);
+      }
+      for (;;) {
+        if (tid == 0) {  // claim the item after next and start the next one's copy
+          const int nx = next_item;
+          if (nx < nitems) {
+            next_item = (int)atomicAdd(&ws.counters[kCntGatherWork], 1u);
+            const int q = nx - nchunks, u = q / cfg.nlr, row0 = (q - u * cfg.nlr) * R;
+            gather_lr_issue(buf0 + (bsel ^ 1) * bstride, lr_a, s_se[u], row0, min(R, d - row0), d, r,
+                            &bar[bsel ^ 1]);
+          }
+          s_lr_next[par] = nx;
+        }
+        const int q = cur - nchunks, u = q / cfg.nlr;
+        const int off = s_so[u], cnt = s_so[u + 1] - off;
+        const int row0 = (q - u * cfg.nlr) * R, nrow = min(R, d - row0);
+        const uint8_t* abuf = reinterpret_cast<const uint8_t*>(buf0 + bsel * bstride);
+        for (int tg = 0; tg < cnt; tg += 8) {
+          const int ntg = min(8, cnt - tg);
+          if (tg > 0) __syncthreads();  // the previous group's reads of s_lz
+          for (int i = tid; i < 8 * zs; i += kNT) {
+            const int t = i / zs, c = i - t * zs;
+            float v = 0.f;
+            if (t < ntg && c < r) v = __ldcg(ws.z + (size_t)(off + tg + t) * r + c) * ws.pair_w[off + tg + t];
+            s_lz[i] = v;
+          }
+          if (tid < 8) s_ltok[tid] = tid < ntg ? ws.pair_tok[off + tg + tid] : 0;
+          if (tg == 0) {  // the rows' copy, and s_lz / s_ltok / s_lr_next visible
+            const bool okw = mbar_wait(&bar[bsel], (phases >> bsel) & 1u, ws.err, cfg.wait_ns);
+            if (!__syncthreads_and(okw)) {  // sticky error set; let the copies in flight land
+              mbar_wait(&bar[bsel], (phases >> bsel) & 1u, ws.err, cfg.wait_ns);
+              if (s_lr_next[par] < nitems)
+                mbar_wait(&bar[bsel ^ 1], (phases >> (bsel ^ 1)) & 1u, ws.err, cfg.wait_ns);
+              ok = false;
+              break;
+            }
+            phases ^= 1u << bsel;
+          } else {
+            __syncthreads();
+          }
+          for (int lr = lrow; lr < R; lr += rpp) {  // trip count uniform: R is a multiple of rpp
+            uint4 av = make_uint4(0u, 0u, 0u, 0u);
+            if (lr < nrow && piece * 8 < r) av = *reinterpret_cast<const uint4*>(abuf + lr * rowb + piece * 16);
+            float acc[8];
+            gather_lr_dot(av, s_lz + piece * 8, zs, acc);
+            for (int o = 1; o < qs; o <<= 1)
+#pragma unroll
+              for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
+            if (lr < nrow)
+#pragma unroll
+              for (int t = 0; t < 8; ++t)
+                if ((t & (qs - 1)) == piece && t < ntg)
+                  atomicAdd(&ws.y_acc[(size_t)s_ltok[t] * d + row0 + lr], acc[t]);
+          }
+        }
+        if (!ok) break;
+        __syncthreads();  // buffer bsel and s_lz are free
+        cur = s_lr_next[par];
+        par ^= 1;
+        bsel ^= 1;
+        if (cur >= nitems) break;
+      }
+      break;
+    }
+
     // ----------------------------------------------------------- low-rank item
-    // kLrPass passes of kNT / qs rows of A_e: thread (row, piece) holds 8 elements of the
+    // (rows not 16-byte aligned) kLrPass passes of kNT / qs rows of A_e: thread (row, piece) holds 8 elements of the
     // row per pass (one 16-byte load when r % 8 == 0), all loads issued before the
     // tokens' z (times the router weight) are staged in shared memory 8 tokens at a time;
     // the row's pieces meet by shuffles and lane `piece` adds tokens piece, piece + qs, ...
@@ -675,21 +820,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
 #pragma unroll
         for (int ps = 0; ps < kLrPass; ++ps) {
           const int row = row0 + ps * rpp + lrow;
-          const uint32_t aw[4] = {av[ps].x, av[ps].y, av[ps].z, av[ps].w};
           float acc[8];
-#pragma unroll
-          for (int t = 0; t < 8; ++t) {
-            const float4 z0 = *reinterpret_cast<const float4*>(s_lz + t * zs + piece * 8);
-            const float4 z1 = *reinterpret_cast<const float4*>(s_lz + t * zs + piece * 8 + 4);
-            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-            float a = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              a = fmaf(__uint_as_float(aw[i] << 16), zz[2 * i], a);
-              a = fmaf(__uint_as_float(aw[i] & 0xffff0000u), zz[2 * i + 1], a);
-            }
-            acc[t] = a;
-          }
+          gather_lr_dot(av[ps], s_lz + piece * 8, zs, acc);
           for (int o = 1; o < qs; o <<= 1)
 #pragma unroll
             for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
@@ -965,14 +1097,17 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   const int dense = (mode == 0 && k == D.inter);
   const int maxslots = min(E, B * K);
   {
-    dim3 grid((E + 7) / 8, (B + kRouterTok - 1) / kRouterTok);
+    dim3 grid((E + kRouterExp - 1) / kRouterExp, (B + kRouterTok - 1) / kRouterTok);
     router_kernel<<<grid, kNT, 0, st>>>(x, B, router_t, D, ws, tr);
   }
   const int KC = d / kColChunk;
   const size_t score_smem = (size_t)kScoreTok * (KC * 32 + 4) * 4 + 4 * 32 * 4 * 4;
   if (!dense || D.rank > 0) {
-    dim3 grid((D.ipad + kScoreRows - 1) / kScoreRows, maxslots);
-    score_kernel<<<grid, kNT, score_smem, st>>>(x, sketch, alpha, lr_b, D, ws, tr, dense);
+    // per slot: nsb score CTAs of kScoreRows rows, then the z CTAs of kNT / 32 rows of B_e
+    const int nsb = dense ? 0 : (D.ipad + kScoreRows - 1) / kScoreRows;
+    const int nzb = (D.rank + kNT / 32 - 1) / (kNT / 32);
+    dim3 grid(nsb + nzb, maxslots);
+    score_kernel<<<grid, kNT, score_smem, st>>>(x, sketch, alpha, lr_b, D, ws, tr, nsb);
   }
   if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
   GatherCfg cfg;
@@ -981,7 +1116,17 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   while (cfg.lr_qs * 8 < D.rank) cfg.lr_qs *= 2;
   cfg.lr_vec = D.rank % 8 == 0;
   {
-    const int rows = kLrPass * (kNT / cfg.lr_qs);
+    // staged items: about 32 KB of A_e each, within one stage buffer, a multiple of the
+    // rows one pass covers; otherwise kLrPass passes from registers
+    const int rpp = kNT / cfg.lr_qs;
+    int rows = 0;
+    if (D.rank > 0 && cfg.lr_vec) {
+      const int fit = (int)(((size_t)cfg.ch * (6 * d + 16)) / (2 * D.rank));
+      rows = min(fit, max(rpp, 32768 / (2 * D.rank)));
+      rows = min(rows, (d + rpp - 1) / rpp * rpp) / rpp * rpp;
+    }
+    cfg.lr_rows = rows;
+    if (rows == 0) rows = kLrPass * rpp;
     cfg.nlr = D.rank > 0 ? (d + rows - 1) / rows : 0;
   }
   cfg.dense = dense;
