@@ -29,6 +29,7 @@ constexpr int kGCh = 8;           // gather: channels per stage at most (one m-t
 constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in flight)
 constexpr int kGRunStages = 8;    // gather: stages per work item at most
 constexpr int kGAccTiles = 16;    // gather: 16-column output tiles per warp held in registers
+static_assert(kGCh <= kNT / 32, "gather: one warp issues each channel of a stage");
 
 // =====================================================================================
 // router
@@ -591,24 +592,30 @@ __device__ __forceinline__ void gather_lr_issue(uint16_t* buf, const uint16_t* l
   bulk_g2s(buf, lr_a + ((size_t)e * d + row0) * r, bytes, bar);
 }
 
-// One warp issues a stage: the channel list of run[c0 .. c0 + n) (shared memory) into
-// `list` and (copy) the bulk copies of their records into a stage buffer, lane i taking
-// channel i (n <= 32).  The list is always written: the consumer reads it whether or not
-// the copies were issued.
+// Every thread calls, after thread 0 has armed `bar` with the stage's bytes (gather_arm)
+// and a barrier of the CTA has ordered that before this call: the channel list of
+// run[c0 .. c0 + n) (shared memory) into `list` and (copy) the bulk copies of their
+// records into a stage buffer, lane 0 of warp i taking channel i (n <= warps), so that no
+// warp waits for all the issues.  The list is always written: the consumer reads it
+// whether or not the copies were issued.
 __device__ __forceinline__ void gather_issue(uint16_t* buf, const uint16_t* records, const int* run,
                                              int e, int c0, int n, int d, int I, int* list,
                                              uint64_t* bar, bool copy = true) {
-  const int lane = threadIdx.x & 31;
-  if (copy && lane == 0) {
-    fence_proxy_async();
-    mbar_arrive_expect_tx(bar, 6u * d * n);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0 && warp < n) {
+    const int j = run[c0 + warp];
+    list[warp] = j;
+    if (copy) {
+      fence_proxy_async();  // the buffer's earlier reads (generic proxy) before the copy
+      bulk_g2s(buf + (size_t)warp * (3 * d + 8), records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
+    }
   }
-  __syncwarp();
-  if (lane < n) {
-    const int j = run[c0 + lane];
-    list[lane] = j;
-    if (copy) bulk_g2s(buf + (size_t)lane * (3 * d + 8), records + ((size_t)e * I + j) * 3 * d, 6u * d, bar);
-  }
+}
+
+// Thread 0: arrive on a stage barrier whose previous phase has completed, expecting the
+// bytes of n records (the stage's copies are issued later by gather_issue).
+__device__ __forceinline__ void gather_arm(uint64_t* bar, int n, int d) {
+  mbar_arrive_expect_tx(bar, 6u * d * n);
 }
 
 // REGACC: d <= 64 * kGAccTiles, outputs held in registers over a run.
@@ -846,21 +853,30 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
 
     for (int tg0 = 0; tg0 < cnt && ok; tg0 += 8) {  // (records are streamed again per 8 tokens)
       const int ntg = min(8, cnt - tg0);
+      // every stage barrier's last phase has completed: thread 0 arms those of stages
+      // 0 .. kGBufs - 1 (the fill's, and the one iteration 0 issues)
+      if (tid == 0)
+        for (int st = 0; st < min(kGBufs, nst); ++st) {
+          bool copy = true;
+#ifdef MSB_INSTRUMENTED
+          copy = !(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0);  // withhold the stage
+#endif
+          if (copy) gather_arm(&bar[st], min(CH, nrun - st * CH), d);
+        }
       __syncthreads();  // s_run; s_tok, s_w, s_h and every stage buffer are free
       if (tid < 8) {
         const int p = off + tg0 + min(tid, ntg - 1);
         s_tok[tid] = ws.pair_tok[p];
         s_w[tid] = tid < ntg ? ws.pair_w[p] : 0.f;
       }
-      if (warp == 0)  // fill: stages 0 .. kGBufs - 2
-        for (int st = 0; st < min(kGBufs - 1, nst); ++st) {
-          bool copy = true;
+      for (int st = 0; st < min(kGBufs - 1, nst); ++st) {  // fill: stages 0 .. kGBufs - 2
+        bool copy = true;
 #ifdef MSB_INSTRUMENTED
-          copy = !(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0);  // withhold the copies only
+        copy = !(cfg.skip == 2u && item == 0 && tg0 == 0 && st == 0);  // withhold the stage
 #endif
-          gather_issue(buf0 + st * bstride, records, s_run, e, st * CH, min(CH, nrun - st * CH), d, I,
-                       s_list[st], &bar[st], copy);
-        }
+        gather_issue(buf0 + st * bstride, records, s_run, e, st * CH, min(CH, nrun - st * CH), d, I,
+                     s_list[st], &bar[st], copy);
+      }
       __syncthreads();  // s_tok, the fill's lists
       // B fragments (x of this lane's token g8) of this warp's k-steps
       uint32_t xb[KSW > 0 ? KSW : 1][2];
@@ -882,8 +898,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         const int b = stg % kGBufs;
         const int nch = min(CH, nrun - stg * CH);
         // keep kGBufs - 1 stages in flight: stage stg + kGBufs - 1 goes into the buffer
-        // that stage stg - 1 has just released
-        if (warp == 0 && stg + kGBufs - 1 < nst) {
+        // that stage stg - 1 has just released (its barrier armed before that release)
+        if (stg + kGBufs - 1 < nst) {
           const int sn = stg + kGBufs - 1, bn = sn % kGBufs;
           gather_issue(buf0 + bn * bstride, records, s_run, e, sn * CH, min(CH, nrun - sn * CH), d, I,
                        s_list[bn], &bar[bn]);
@@ -1024,6 +1040,8 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
             gather_red_tile(ws.y_acc, s_tok, ntg, d, c0w + 16 * NT16, dA, lane, false);
           }
         }
+        // the stage that reuses this buffer: arm its barrier (this phase has completed)
+        if (tid == 0 && stg + kGBufs < nst) gather_arm(&bar[b], min(CH, nrun - (stg + kGBufs) * CH), d);
         __syncthreads();  // this stage's buffer, s_red and s_h are free
       }
       if (REGACC && ok) {  // one reduction-add per output of the run
