@@ -28,7 +28,6 @@ static_assert(MSB_MAX_RANK % 8 == 0 && (MSB_MAX_RANK & (MSB_MAX_RANK - 1)) == 0,
 constexpr int kGCh = 8;           // gather: channels per stage at most (one m-tile of gate/up rows)
 constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in flight)
 constexpr int kGRunStages = 8;    // gather: stages per work item at most
-constexpr int kGAccTiles = 16;    // gather: 16-column output tiles per warp held in registers
 static_assert(kGCh <= kNT / 32, "gather: one warp issues each channel of a stage");
 
 // =====================================================================================
@@ -618,16 +617,18 @@ __device__ __forceinline__ void gather_arm(uint64_t* bar, int n, int d) {
   mbar_arrive_expect_tx(bar, 6u * d * n);
 }
 
-// REGACC: d <= 64 * kGAccTiles, outputs held in registers over a run.
+// NACC > 0: d <= 128 NACC, each warp's outputs (NACC tiles of 16 columns) held in
+// registers over a run; 0: reduction-adds after every stage.
 // KSW: the x B-fragments of this warp's k-steps held in registers per token group
 // (d <= 128 * KSW); 0: read through L1/L2 at every stage.
 // Stages of cfg.ch channels stream through kGBufs buffers, kGBufs - 1 of them in flight
 // while one is computed.
-template <bool REGACC, int KSW>
+template <int NACC, int KSW>
 __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restrict__ x,
                                                         const uint16_t* __restrict__ records,
                                                         const uint16_t* __restrict__ lr_a, Dims D,
                                                         Workspace ws, GatherCfg cfg) {
+  constexpr bool REGACC = NACC > 0;
   extern __shared__ __align__(128) uint8_t gsm[];
   __shared__ __align__(8) uint64_t bar[kGBufs];
   __shared__ int s_item, s_u;
@@ -887,9 +888,9 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
           xb[i][0] = __ldg(xrow + (ks0 + i) * 8 + c4);
           xb[i][1] = __ldg(xrow + (ks0 + i) * 8 + 4 + c4);
         }
-      float yacc[REGACC ? kGAccTiles : 1][4];
+      float yacc[REGACC ? NACC : 1][4];
 #pragma unroll
-      for (int i = 0; i < (REGACC ? kGAccTiles : 1); ++i)
+      for (int i = 0; i < (REGACC ? NACC : 1); ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) yacc[i][j] = 0.f;
 
@@ -928,45 +929,44 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         // down ldmatrix.trans row: channel lane % 8 (channels past nch read channel 0;
         // their h is zero); lane / 8 picks the 8-column block
         const uint32_t b_base = smem_addr(rec + (size_t)gch * rs + 2 * d);
-        // ---- gate/up partials over this warp's k-steps
+        // ---- gate/up partials over this warp's k-steps (four accumulator chains)
         {
-          float acc0[4] = {0.f, 0.f, 0.f, 0.f}, acc1[4] = {0.f, 0.f, 0.f, 0.f};
+          float acc[4][4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
           int ks = ks0;
           if (KSW > 0) {
 #pragma unroll
-            for (int i = 0; i < KSW; i += 2) {
-              if (ks0 + i + 1 < ks1) {
-                uint32_t a[2][4];
-                ldsm_x4(a_addr + 32u * i, a[0][0], a[0][1], a[0][2], a[0][3]);
-                ldsm_x4(a_addr + 32u * (i + 1), a[1][0], a[1][1], a[1][2], a[1][3]);
-                mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], xb[i][0], xb[i][1]);
-                mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], xb[i + 1][0], xb[i + 1][1]);
-              } else if (ks0 + i < ks1) {
+            for (int i = 0; i < KSW; ++i)
+              if (ks0 + i < ks1) {
                 uint32_t a0, a1, a2, a3;
                 ldsm_x4(a_addr + 32u * i, a0, a1, a2, a3);
-                mma_bf16(acc0, a0, a1, a2, a3, xb[i][0], xb[i][1]);
+                mma_bf16(acc[i & 3], a0, a1, a2, a3, xb[i][0], xb[i][1]);
               }
-            }
             ks = ks1;
           }
-          for (; ks + 2 <= ks1; ks += 2, a_addr += 64u) {
-            uint32_t a[2][4];
-            ldsm_x4(a_addr, a[0][0], a[0][1], a[0][2], a[0][3]);
-            ldsm_x4(a_addr + 32u, a[1][0], a[1][1], a[1][2], a[1][3]);
-            const uint32_t b00 = __ldg(xrow + ks * 8 + c4), b01 = __ldg(xrow + ks * 8 + 4 + c4);
-            const uint32_t b10 = __ldg(xrow + ks * 8 + 8 + c4), b11 = __ldg(xrow + ks * 8 + 12 + c4);
-            mma_bf16(acc0, a[0][0], a[0][1], a[0][2], a[0][3], b00, b01);
-            mma_bf16(acc1, a[1][0], a[1][1], a[1][2], a[1][3], b10, b11);
+          for (; ks + 4 <= ks1; ks += 4, a_addr += 128u) {
+            uint32_t a[4][4], bb[4][2];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              ldsm_x4(a_addr + 32u * i, a[i][0], a[i][1], a[i][2], a[i][3]);
+              bb[i][0] = __ldg(xrow + (ks + i) * 8 + c4);
+              bb[i][1] = __ldg(xrow + (ks + i) * 8 + 4 + c4);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mma_bf16(acc[i], a[i][0], a[i][1], a[i][2], a[i][3], bb[i][0], bb[i][1]);
           }
-          if (ks < ks1) {
+          for (; ks < ks1; ++ks, a_addr += 32u) {
             uint32_t a0, a1, a2, a3;
             ldsm_x4(a_addr, a0, a1, a2, a3);
-            mma_bf16(acc0, a0, a1, a2, a3, __ldg(xrow + ks * 8 + c4), __ldg(xrow + ks * 8 + 4 + c4));
+            mma_bf16(acc[0], a0, a1, a2, a3, __ldg(xrow + ks * 8 + c4), __ldg(xrow + ks * 8 + 4 + c4));
           }
-          s_red[warp][g8][2 * c4] = acc0[0] + acc1[0];
-          s_red[warp][g8][2 * c4 + 1] = acc0[1] + acc1[1];
-          s_red[warp][g8 + 8][2 * c4] = acc0[2] + acc1[2];
-          s_red[warp][g8 + 8][2 * c4 + 1] = acc0[3] + acc1[3];
+          s_red[warp][g8][2 * c4] = (acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]);
+          s_red[warp][g8][2 * c4 + 1] = (acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1]);
+          s_red[warp][g8 + 8][2 * c4] = (acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2]);
+          s_red[warp][g8 + 8][2 * c4 + 1] = (acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3]);
         }
         __syncthreads();
         // ---- h[token][channel] = silu(g) u, times the selection bit and the router weight
@@ -991,7 +991,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
         if (REGACC) {
           // (register indices stay compile-time: the tile loop is unrolled)
 #pragma unroll
-          for (int t = 0; t < kGAccTiles; t += 2) {
+          for (int t = 0; t < NACC; t += 2) {
             const int m0 = c0w + 16 * t;
             if (t + 1 < NT16) {
               uint32_t a0, a1, a2, a3;
@@ -1046,7 +1046,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
       }
       if (REGACC && ok) {  // one reduction-add per output of the run
 #pragma unroll
-        for (int t = 0; t < kGAccTiles; ++t)
+        for (int t = 0; t < NACC; ++t)
           if (t < NT16 + (tail8 ? 1 : 0))
             gather_red_tile(ws.y_acc, s_tok, ntg, d, c0w + 16 * t, yacc[t], lane, t < NT16);
       }
@@ -1158,12 +1158,12 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   const int ngrid = sm_count();
   union_kernel<<<maxslots, kNT, 0, st>>>(D, ws, cfg.ch, ngrid, dense);
   const size_t gsmem = (size_t)kGBufs * cfg.ch * (6 * d + 16);
-  if (d <= 2048)
-    gather_kernel<true, 16><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
-  else if (d <= 4096)
-    gather_kernel<false, 32><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+  if (d <= 2048)  // outputs and x fragments in registers
+    gather_kernel<16, 16><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+  else if (d <= 4096)  // outputs in registers, x fragments through L1
+    gather_kernel<32, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
   else
-    gather_kernel<false, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+    gather_kernel<0, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
   {
     const size_t n8 = (size_t)B * d / 8;
     const size_t nb = (n8 + kNT - 1) / kNT;
@@ -1178,11 +1178,11 @@ int general_set_smem_limits() {
   cudaError_t e = cudaSuccess;
   e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<true, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  e = cudaFuncSetAttribute(gather_kernel<16, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<false, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  e = cudaFuncSetAttribute(gather_kernel<32, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   if (e != cudaSuccess) return MSB_ECUDA;
-  e = cudaFuncSetAttribute(gather_kernel<false, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+  e = cudaFuncSetAttribute(gather_kernel<0, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, big);
   return e == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 
