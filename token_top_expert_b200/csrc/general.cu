@@ -534,6 +534,10 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+
 __device__ __forceinline__ void ldsm_x2_t(uint32_t addr, uint32_t& r0, uint32_t& r1) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];"
                : "=r"(r0), "=r"(r1)
@@ -580,6 +584,14 @@ __device__ __forceinline__ void gather_lr_dot(uint4 av, const float* z, int zs, 
     }
     acc[t] = a;
   }
+}
+
+// B fragment of the low-rank MMA: z[t][i], z[t][i + 1] (FP32, times the router weight) as
+// a BF16 pair (zhi) and the pair of what BF16 rounding left over (zlo)
+__device__ __forceinline__ void lr_zfrag(const float* z, uint32_t& zhi, uint32_t& zlo) {
+  const float2 v = *reinterpret_cast<const float2*>(z);
+  zhi = pack_bf16x2(v.x, v.y);
+  zlo = pack_bf16x2(v.x - __uint_as_float(zhi << 16), v.y - __uint_as_float(zhi & 0xffff0000u));
 }
 
 // Thread 0 copies rows [row0, row0 + nrow) of A_e (r bf16 each, r % 8 == 0) into `buf`.
@@ -711,8 +723,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
     // next item's rows of A_e (cfg.lr_rows rows of r bf16, contiguous) into the other stage
     // buffer while the current item is computed from shared memory.
     if (item >= nchunks && cfg.lr_rows > 0) {
-      const int qs = cfg.lr_qs, zs = 8 * qs, rpp = kNT / qs;
-      const int lrow = tid / qs, piece = tid - lrow * qs;
+      const int zs = 8 * cfg.lr_qs;  // z stride: r rounded up to 8 times a power of two
       const int R = cfg.lr_rows;
       const uint32_t rowb = 2u * (uint32_t)r;
       int cur = item, bsel = 0, par = 0;
@@ -758,19 +769,28 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
           } else {
             __syncthreads();
           }
-          for (int lr = lrow; lr < R; lr += rpp) {  // trip count uniform: R is a multiple of rpp
-            uint4 av = make_uint4(0u, 0u, 0u, 0u);
-            if (lr < nrow && piece * 8 < r) av = *reinterpret_cast<const uint4*>(abuf + lr * rowb + piece * 16);
-            float acc[8];
-            gather_lr_dot(av, s_lz + piece * 8, zs, acc);
-            for (int o = 1; o < qs; o <<= 1)
-#pragma unroll
-              for (int t = 0; t < 8; ++t) acc[t] += __shfl_xor_sync(0xffffffffu, acc[t], o);
-            if (lr < nrow)
-#pragma unroll
-              for (int t = 0; t < 8; ++t)
-                if ((t & (qs - 1)) == piece && t < ntg)
-                  atomicAdd(&ws.y_acc[(size_t)s_ltok[t] * d + row0 + lr], acc[t]);
+          // D[16 rows][8 tokens] += rows of A_e x [z_hi ; z_lo]: the two BF16 halves of z lie
+          // along k against the same 8 values of r repeated, 8 values of r per MMA; a warp
+          // takes every (kNT / 32)-th tile of 16 rows (nrow is a multiple of 16)
+          for (int tl = warp; tl < nrow / 16; tl += kNT / 32) {
+            const uint8_t* tb = abuf + (size_t)tl * 16 * rowb + (size_t)(lane & 15) * rowb;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            int rc = 0;
+            for (; rc + 16 <= r; rc += 16) {  // lanes 16-31 address the next 8 values of r
+              uint32_t a0, a1, a2, a3, z0, z1, z2, z3;
+              ldsm_x4(smem_addr(tb + 2 * (rc + 8 * (lane >> 4))), a0, a1, a2, a3);
+              lr_zfrag(s_lz + g8 * zs + rc + 2 * c4, z0, z1);
+              lr_zfrag(s_lz + g8 * zs + rc + 8 + 2 * c4, z2, z3);
+              mma_bf16(acc, a0, a1, a0, a1, z0, z1);
+              mma_bf16(acc, a2, a3, a2, a3, z2, z3);
+            }
+            if (rc < r) {  // 8 values of r left
+              uint32_t a0, a1, z0, z1;
+              ldsm_x2(smem_addr(tb + 2 * rc), a0, a1);
+              lr_zfrag(s_lz + g8 * zs + rc + 2 * c4, z0, z1);
+              mma_bf16(acc, a0, a1, a0, a1, z0, z1);
+            }
+            gather_red_tile(ws.y_acc, s_ltok, ntg, d, row0 + 16 * tl, acc, lane, true);
           }
         }
         if (!ok) break;
