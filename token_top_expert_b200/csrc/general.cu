@@ -30,12 +30,21 @@ constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in
 constexpr int kGRunStages = 8;    // gather: stages per work item at most
 static_assert(kGCh <= kNT / 32, "gather: one warp issues each channel of a stage");
 
+// Every kernel of this path is launched with programmatic stream serialization and begins
+// here: wait until the kernels before it on the stream have completed and their writes are
+// visible, then let the next kernel be scheduled while this one runs (it waits in turn).
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // =====================================================================================
 // router
 // =====================================================================================
 __global__ void __launch_bounds__(kNT) router_kernel(const uint16_t* __restrict__ x, int B,
                                                      const uint16_t* __restrict__ router_t, Dims D,
                                                      Workspace ws, TraceDev tr) {
+  pdl_begin();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = D.d, E = D.experts, K = D.top_e;
   const int t0 = blockIdx.y * kRouterTok;
@@ -259,6 +268,7 @@ __global__ void __launch_bounds__(kNT, 3) score_kernel(const uint16_t* __restric
                                                     const float* __restrict__ alpha,
                                                     const uint16_t* __restrict__ lr_b, Dims D,
                                                     Workspace ws, TraceDev tr, int nsb) {
+  pdl_begin();
   extern __shared__ __align__(16) uint32_t smem[];
   const int u = blockIdx.y;
   if (u >= *ws.nused) return;
@@ -382,6 +392,7 @@ __global__ void __launch_bounds__(kNT, 3) score_kernel(const uint16_t* __restric
 // =====================================================================================
 __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau, Dims D,
                                                      Workspace ws, TraceDev tr) {
+  pdl_begin();
   __shared__ uint32_t keys[MSB_MAX_INTER];
   __shared__ uint16_t sel_s[MSB_MAX_INTER];
   __shared__ uint32_t words[MSB_MAX_INTER / 32];
@@ -444,6 +455,7 @@ __global__ void __launch_bounds__(kNT) select_kernel(int k, int mode, float tau,
 // slots' channel chunks (the gather kernel's work items)
 // =====================================================================================
 __global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch, int ngrid, int dense) {
+  pdl_begin();
   __shared__ uint32_t s_tmp[kNT / 32 + 1];
   __shared__ int s_last;
   const int tid = threadIdx.x;
@@ -640,6 +652,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
                                                         const uint16_t* __restrict__ records,
                                                         const uint16_t* __restrict__ lr_a, Dims D,
                                                         Workspace ws, GatherCfg cfg) {
+  pdl_begin();
   constexpr bool REGACC = NACC > 0;
   extern __shared__ __align__(128) uint8_t gsm[];
   __shared__ __align__(8) uint64_t bar[kGBufs];
@@ -1079,6 +1092,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
 // =====================================================================================
 __global__ void __launch_bounds__(kNT) finalize_kernel(uint16_t* __restrict__ out, int B, Dims D,
                                                        Workspace ws, TraceDev tr, int dense) {
+  pdl_begin();
   const size_t n8 = (size_t)B * D.d / 8;
   for (size_t i = blockIdx.x * (size_t)kNT + threadIdx.x; i < n8; i += (size_t)gridDim.x * kNT) {
     float4* src = reinterpret_cast<float4*>(ws.y_acc) + 2 * i;
@@ -1127,6 +1141,23 @@ int sm_count() {
   return n[dev];
 }
 
+// Launch one kernel of this path, kNT threads per CTA, with programmatic stream
+// serialization (the kernel begins with pdl_begin()).
+template <typename... KArgs, typename... Args>
+bool launch_pdl(void (*kernel)(KArgs...), dim3 grid, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kNT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess;
+}
+
 int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uint16_t* records,
                    const uint32_t* sketch, const float* alpha, int k, int mode, float tau,
                    const uint16_t* lr_a, const uint16_t* lr_b, uint16_t* out, const Dims& D,
@@ -1134,9 +1165,10 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   const int E = D.experts, K = D.top_e, d = D.d;
   const int dense = (mode == 0 && k == D.inter);
   const int maxslots = min(E, B * K);
+  bool ok = true;
   {
     dim3 grid((E + kRouterExp - 1) / kRouterExp, (B + kRouterTok - 1) / kRouterTok);
-    router_kernel<<<grid, kNT, 0, st>>>(x, B, router_t, D, ws, tr);
+    ok = ok && launch_pdl(router_kernel, grid, 0, st, x, B, router_t, D, ws, tr);
   }
   const int KC = d / kColChunk;
   const size_t score_smem = (size_t)kScoreTok * (KC * 32 + 4) * 4 + 4 * 32 * 4 * 4;
@@ -1145,22 +1177,22 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
     const int nsb = dense ? 0 : (D.ipad + kScoreRows - 1) / kScoreRows;
     const int nzb = (D.rank + kNT / 32 - 1) / (kNT / 32);
     dim3 grid(nsb + nzb, maxslots);
-    score_kernel<<<grid, kNT, score_smem, st>>>(x, sketch, alpha, lr_b, D, ws, tr, nsb);
+    ok = ok && launch_pdl(score_kernel, grid, score_smem, st, x, sketch, alpha, lr_b, D, ws, tr, nsb);
   }
-  if (!dense) select_kernel<<<B * K, kNT, 0, st>>>(k, mode, tau, D, ws, tr);
+  if (!dense) ok = ok && launch_pdl(select_kernel, dim3(B * K), 0, st, k, mode, tau, D, ws, tr);
   GatherCfg cfg;
   cfg.ch = max(1, min(kGCh, (196 * 1024 / kGBufs) / (6 * d + 16)));
   cfg.lr_qs = 1;
   while (cfg.lr_qs * 8 < D.rank) cfg.lr_qs *= 2;
   cfg.lr_vec = D.rank % 8 == 0;
   {
-    // staged items: about 32 KB of A_e each, within one stage buffer, a multiple of the
+    // staged items: about 64 KB of A_e each, within one stage buffer, a multiple of the
     // rows one pass covers; otherwise kLrPass passes from registers
     const int rpp = kNT / cfg.lr_qs;
     int rows = 0;
     if (D.rank > 0 && cfg.lr_vec) {
       const int fit = (int)(((size_t)cfg.ch * (6 * d + 16)) / (2 * D.rank));
-      rows = min(fit, max(rpp, 32768 / (2 * D.rank)));
+      rows = min(fit, max(rpp, 65536 / (2 * D.rank)));
       rows = min(rows, (d + rpp - 1) / rpp * rpp) / rpp * rpp;
     }
     cfg.lr_rows = rows;
@@ -1176,21 +1208,21 @@ int launch_general(const uint16_t* x, int B, const uint16_t* router_t, const uin
   // persistent CTAs, one per SM, taking work items (runs of union channels, then
   // low-rank row blocks) off a counter
   const int ngrid = sm_count();
-  union_kernel<<<maxslots, kNT, 0, st>>>(D, ws, cfg.ch, ngrid, dense);
+  ok = ok && launch_pdl(union_kernel, dim3(maxslots), 0, st, D, ws, cfg.ch, ngrid, dense);
   const size_t gsmem = (size_t)kGBufs * cfg.ch * (6 * d + 16);
   if (d <= 2048)  // outputs and x fragments in registers
-    gather_kernel<16, 16><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+    ok = ok && launch_pdl(gather_kernel<16, 16>, dim3(ngrid), gsmem, st, x, records, lr_a, D, ws, cfg);
   else if (d <= 4096)  // outputs in registers, x fragments through L1
-    gather_kernel<32, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+    ok = ok && launch_pdl(gather_kernel<32, 0>, dim3(ngrid), gsmem, st, x, records, lr_a, D, ws, cfg);
   else
-    gather_kernel<0, 0><<<ngrid, kNT, gsmem, st>>>(x, records, lr_a, D, ws, cfg);
+    ok = ok && launch_pdl(gather_kernel<0, 0>, dim3(ngrid), gsmem, st, x, records, lr_a, D, ws, cfg);
   {
     const size_t n8 = (size_t)B * d / 8;
     const size_t nb = (n8 + kNT - 1) / kNT;
     const int blocks = (int)(nb < 148 * 4 ? nb : 148 * 4);
-    finalize_kernel<<<blocks, kNT, 0, st>>>(out, B, D, ws, tr, dense);
+    ok = ok && launch_pdl(finalize_kernel, dim3(blocks), 0, st, out, B, D, ws, tr, dense);
   }
-  return cudaGetLastError() == cudaSuccess ? MSB_OK : MSB_ECUDA;
+  return ok && cudaGetLastError() == cudaSuccess ? MSB_OK : MSB_ECUDA;
 }
 
 int general_set_smem_limits() {
