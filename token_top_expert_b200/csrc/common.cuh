@@ -167,26 +167,6 @@ __device__ __forceinline__ float dot8(uint4 a, uint4 b, float acc) {
   return acc;
 }
 
-// Sums of v[0..N) over the warp, transposed: afterwards lane l holds in v[0 .. N/32) the
-// totals of the values N/32 l .. N/32 l + N/32 - 1 (N a power of two, N >= 32).  Each round
-// halves the values a lane keeps: the lane whose bit o is set keeps the upper half and adds
-// its partner's copy of it.
-template <int N>
-__device__ __forceinline__ void warp_sum_transposed(float (&v)[N], int lane) {
-  static_assert(N >= 32 && (N & (N - 1)) == 0, "N: a power of two, at least 32");
-#pragma unroll
-  for (int s = 0; s < 5; ++s) {
-    const int o = 16 >> s, half = N >> (s + 1);
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = up ? v[i] : v[i + half];
-      const float keep = up ? v[i + half] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-}
-
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

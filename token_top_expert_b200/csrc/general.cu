@@ -27,8 +27,28 @@ static_assert(MSB_MAX_RANK % 8 == 0 && (MSB_MAX_RANK & (MSB_MAX_RANK - 1)) == 0,
               "the low-rank z stride 8 qs must fit 8 * MSB_MAX_RANK floats per token group");
 constexpr int kGCh = 8;           // gather: channels per stage at most (one m-tile of gate/up rows)
 constexpr int kGBufs = 2;         // gather: stage buffers (kGBufs - 1 stages in flight)
-constexpr int kGRunStages = 8;    // gather: stages per work item at most
+constexpr int kGRunCh = 64;       // gather: channels per work item at most (a multiple of stages)
 static_assert(kGCh <= kNT / 32, "gather: one warp issues each channel of a stage");
+
+// Sums of v[0..N) over the warp, transposed: afterwards lane l holds in v[0 .. N/32) the
+// totals of the values N/32 l .. N/32 l + N/32 - 1 (N a power of two, N >= 32).  Each round
+// halves the values a lane keeps: the lane whose bit o is set keeps the upper half and adds
+// its partner's copy of it.
+template <int N>
+__device__ __forceinline__ void warp_sum_transposed(float (&v)[N], int lane) {
+  static_assert(N >= 32 && (N & (N - 1)) == 0, "N: a power of two, at least 32");
+#pragma unroll
+  for (int s = 0; s < 5; ++s) {
+    const int o = 16 >> s, half = N >> (s + 1);
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = up ? v[i] : v[i + half];
+      const float keep = up ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
 
 // Every kernel of this path is launched with programmatic stream serialization and begins
 // here: wait until the kernels before it on the stream have completed and their writes are
@@ -483,7 +503,8 @@ __global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch
   if (!s_last) return;
   __threadfence();
   // run length: a multiple of the stage size ch, about two runs per CTA of the grid,
-  // at most kGRunStages stages (longer runs mean fewer reduction-adds per output)
+  // at most kGRunCh channels (longer runs mean fewer reduction-adds per output and less
+  // per-item overhead, shorter ones a more even finish)
   uint32_t n2[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -491,7 +512,7 @@ __global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch
   uint32_t all;
   block_excl_scan<kNT>(n2[0] + n2[1], s_tmp, &all);
   int run = (int)((all + 2u * ngrid - 1) / (2u * ngrid));
-  run = min(kGRunStages * ch, max(ch, (run + ch - 1) / ch * ch));
+  run = min(kGRunCh / ch * ch, max(ch, (run + ch - 1) / ch * ch));
   uint32_t c[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 2; ++i) c[i] = (n2[i] + run - 1) / run;
@@ -658,7 +679,7 @@ __global__ void __launch_bounds__(kNT, 1) gather_kernel(const uint16_t* __restri
   __shared__ __align__(8) uint64_t bar[kGBufs];
   __shared__ int s_item, s_u;
   __shared__ int s_list[kGBufs][kGCh];
-  __shared__ int s_run[kGRunStages * kGCh];  // channel indices of the current run
+  __shared__ int s_run[kGRunCh];  // channel indices of the current run
   __shared__ int s_tok[8];
   __shared__ float s_w[8];
   __shared__ float s_red[kNT / 32][16][8];
