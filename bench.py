@@ -732,7 +732,7 @@ def main():
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     plan = msb.path_info(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B,
-                         args.k, general=general)
+                         args.k, general=general, single=bool(args.q4))  # 4-bit: single launch only
     kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
     traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else "") + ("_q4" if args.q4 else ""))
     launches_per_step = block_launches(plan["path"], dense, args.rank)

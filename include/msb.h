@@ -71,6 +71,9 @@ extern "C" {
 
 /* ------------------------------------------------------------------ flags */
 #define MSB_FLAG_GENERAL 1u    /* use the multi-kernel path at every batch size */
+#define MSB_FLAG_SINGLE 4u     /* batches up to 16 tokens: the single-launch kernel even
+                                  where the multi-kernel path is faster (ignored with
+                                  MSB_FLAG_GENERAL) */
 #define MSB_FLAG_X_READY 2u    /* x is complete when the call is enqueued: nothing earlier on
                                   the stream writes it (activations the host produced), so
                                   the single-launch kernel may fetch it while the previous
@@ -160,11 +163,13 @@ int32_t msb_check(void* workspace, void* stream);
 const char* msb_strerror(int32_t status);
 
 /* Diagnostics: the path moe_sparse_block takes for these arguments on the
- * current device.  Batches of up to 16 tokens run on the single-launch kernel
- * when it fits (one cluster per (token, routed expert) pair, each pair reading
- * its own k channels); larger batches, MSB_FLAG_GENERAL, and batches above 1
- * whose trace asks for the per-expert union count take the multi-kernel path,
- * which reads each expert's union of channels once.  Fills info (host, 8 int32):
+ * current device.  Small batches run on the single-launch kernel when it fits
+ * (one cluster per (token, routed expert) pair, each pair reading its own k
+ * channels): up to 12 (2048 / d)^2 tokens (1..16; the measured crossover: 12 at
+ * d = 2048, 3 at d = 4096), up to 16 with MSB_FLAG_SINGLE or 4-bit records.
+ * Larger batches, MSB_FLAG_GENERAL, and batches above 1 whose trace asks for the
+ * per-expert union count take the multi-kernel path, which reads each expert's
+ * union of channels once.  Fills info (host, 8 int32):
  *   {path (1 = single launch, 2 = multi-kernel), cluster size, clusters per
  *    routed expert, channel-record ring slots, dynamic shared-memory bytes,
  *    resident 16-CTA clusters, resident 8-CTA clusters, 0}.
@@ -191,7 +196,7 @@ int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t f
  *  workspace, workspace_bytes: device scratch of at least
  *           msb_workspace_size(dims, batch) bytes, zero-filled before first use.
  *  trace    optional host struct of device pointers (NULL: no trace).
- *  flags    0, MSB_FLAG_GENERAL, MSB_FLAG_X_READY, or both.
+ *  flags    0 or an OR of MSB_FLAG_GENERAL, MSB_FLAG_SINGLE, MSB_FLAG_X_READY.
  *  stream   cudaStream_t.
  * FP32 accumulation throughout; channel scores in FP32. */
 int32_t moe_sparse_block(const void* x, int32_t batch, const void* router_t, const void* records,
@@ -218,7 +223,7 @@ int32_t moe_sparse_block_top_e(const void* x, int32_t batch, const void* router_
 /* The block on activations in host memory, everything enqueued on `stream` (no
  * synchronisation: the host buffers must stay valid, and out_host unread, until the
  * stream has passed the call).
- *  - batches on the single-launch path (up to 16 tokens) with x_host and out_host
+ *  - batches on the single-launch path (see msb_path_info) with x_host and out_host
  *    pinned, mapped into the current device's address space (cudaHostAlloc / torch
  *    pin_memory under unified addressing) and 16-byte aligned: the kernel itself
  *    reads x_host and writes out_host across the host link, so consecutive calls

@@ -307,19 +307,20 @@ def test_workspace_reuse_across_batch_sizes(msb):
 @pytest.mark.parametrize("workload,batch", [("qwen13", 2), ("qwen13", 4), ("qwen13", 16), ("tiny", 3)])
 def test_small_batch_single_launch(msb, workload, batch):
     """Batches of up to 16 tokens on the single-launch kernel (one cluster per (token,
-    routed expert) pair): every token against the oracle; consecutive calls share the
+    routed expert) pair; asked for, since 16 tokens at d = 2048 default to the
+    multi-kernel path): every token against the oracle; consecutive calls share the
     workspace's accumulator and slice counters."""
     import torch
     from parity import from_bf16_tensor, to_bf16_tensor
     w = synth.QWEN30B_BLOCK_13 if workload == "qwen13" else synth.TINY
     dev = device_layer(w)
-    assert msb.path_info(dev.dims, batch, w.k)["path"] == "single_launch"
+    assert msb.path_info(dev.dims, batch, w.k, single=True)["path"] == "single_launch"
     lay = oracle.SynthLayer(w)
     ws = msb.Workspace(dev.dims, batch)
     for step in range(2):
         x = synth.activations(w, 60 + step, batch=batch)
         tr = msb.Trace(dev.dims, batch, w.k, scores=True, union=False)
-        out = msb.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, trace=tr)
+        out = msb.moe_sparse_block(to_bf16_tensor(x), dev, w.k, workspace=ws, trace=tr, single=True)
         torch.cuda.synchronize()
         ws.check()
         g = {"y": oracle.bf16_to_f64(from_bf16_tensor(out)), "ids": tr.expert_ids.cpu().numpy(),
@@ -328,3 +329,19 @@ def test_small_batch_single_launch(msb, workload, batch):
              "scores": tr.scores.cpu().numpy()}
         assert (g["sel_count"] == w.k).all()
         print(batch, step, compare(x, g, lay, w.top_e, w.k))
+
+
+@pytest.mark.parametrize("workload,batch,path", [
+    ("qwen13", 12, "single_launch"), ("qwen13", 16, "multi_kernel"),
+    ("large", 3, "single_launch"), ("large", 4, "multi_kernel"), ("wide", 1, "single_launch"),
+    ("wide", 2, "multi_kernel"), ("tiny", 16, "single_launch")])
+def test_default_path_follows_the_crossover(msb, workload, batch, path):
+    """The default path: the single launch up to 12 (2048 / d)^2 tokens (1..16), the
+    multi-kernel path above; MSB_FLAG_SINGLE keeps the single launch up to 16 tokens."""
+    # the shapes of the workloads the parity tests run (d, I, E, K, r) and their k
+    shape, k = {"qwen13": ((2048, 768, 128, 8, 32), 100), "large": ((4096, 1536, 128, 8, 64), 276),
+                "wide": ((8192, 512, 16, 4, 16), 92), "tiny": ((256, 512, 8, 2, 16), 92)}[workload]
+    dims = msb.Dims(*shape, 1)
+    assert msb.path_info(dims, batch, k)["path"] == path
+    assert msb.path_info(dims, batch, k, single=True)["path"] == "single_launch"
+    assert msb.path_info(dims, batch, k, general=True, single=True)["path"] == "multi_kernel"

@@ -21,6 +21,7 @@ MSB_ENONFINITE = -5
 MSB_EINTERNAL = -6
 MSB_FLAG_GENERAL = 1
 MSB_FLAG_X_READY = 2
+MSB_FLAG_SINGLE = 4
 
 MSB_MAX_D = 8192
 MSB_MAX_INTER = 4096

@@ -301,10 +301,12 @@ def _act(x, dims: Dims):
 
 def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspace | None = None,
                      trace: Trace | None = None, general: bool = False, stream=None,
-                     top_e: int | None = None):
+                     top_e: int | None = None, single: bool = False):
     """One sparse-MoE block decode step: out[t] = sum_e w_te * (gathered SwiGLU over the
     k top-scoring channels + A_e B_e x_t).  x: bf16 [B][d] on the GPU.  top_e: route each
     token to this many experts instead of the trained layer.dims.top_e (at most that).
+    general / single: the multi-kernel path at any batch / the single-launch kernel up to
+    16 tokens (default: whichever the measured crossover for d prefers; see path_info).
     out and workspace are allocated when not given (pass both for repeated calls and for
     a raw stream handle); the call is asynchronous on `stream` (default: torch's current
     stream)."""
@@ -320,7 +322,7 @@ def moe_sparse_block(x, layer: PackedLayer, k: int, out=None, workspace: Workspa
         workspace = new_ws = Workspace(dims, B, x.device)
     _temporaries_on(stream, [new_out, new_ws.buf if new_ws else None])
     tr = trace.c() if trace is not None else None
-    flags = _lib.MSB_FLAG_GENERAL if general else 0
+    flags = (_lib.MSB_FLAG_GENERAL if general else 0) | (_lib.MSB_FLAG_SINGLE if single else 0)
     args = (_ptr(x), B, _ptr(layer.router_t), _ptr(layer.records), _ptr(layer.sketch),
             _ptr(layer.alpha), k)
     rest = (_ptr(layer.lr_a), _ptr(layer.lr_b), _ptr(out), ctypes.byref(dims.c()), workspace.ptr,
@@ -452,11 +454,11 @@ def moe_sparse_block_threshold(x, layer: PackedLayer, tau: float, out=None,
     return out
 
 
-def path_info(dims: Dims, batch: int, k: int, general: bool = False) -> dict:
+def path_info(dims: Dims, batch: int, k: int, general: bool = False, single: bool = False) -> dict:
     """Which path moe_sparse_block takes on the current device, and its plan."""
     info = (ctypes.c_int32 * 8)()
-    rc = _lib.load().msb_path_info(ctypes.byref(dims.c()), batch, k,
-                                   _lib.MSB_FLAG_GENERAL if general else 0, info)
+    flags = (_lib.MSB_FLAG_GENERAL if general else 0) | (_lib.MSB_FLAG_SINGLE if single else 0)
+    rc = _lib.load().msb_path_info(ctypes.byref(dims.c()), batch, k, flags, info)
     _check(rc, "msb_path_info")
     v = list(info)
     return {"path": "single_launch" if v[0] == 1 else "multi_kernel", "cluster_size": v[1],

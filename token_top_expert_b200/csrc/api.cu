@@ -210,7 +210,8 @@ int block_common(const void* x, int32_t batch, const void* router_t, const void*
   const uint16_t* la = static_cast<const uint16_t*>(lr_a);
   const uint16_t* lb = static_cast<const uint16_t*>(lr_b);
   uint16_t* o = static_cast<uint16_t*>(out);
-  if (mode == 0 && batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k, q4)) {
+  if (mode == 0 && batch <= single_launch_max_batch(D, (flags & MSB_FLAG_SINGLE) != 0, q4) &&
+      !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k, q4)) {
     rc = launch_fused(xb, rt, rec, sketch, alpha, k, la, lb, o, D, ws.err, ws.counters, ws.y_acc,
                       tr, st, x_mapped, (flags & MSB_FLAG_X_READY) != 0, batch, q4);
     if (rc != MSB_ENOTFUSED) return rc;
@@ -339,7 +340,8 @@ int32_t moe_sparse_block_host(const void* x_host, void* x_dev, int32_t batch, co
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // pinned, mapped host buffers on the single-launch path: the kernel itself reads x and
   // writes the result across the host link (no copy-engine round trip between launches)
-  if (batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL)) {
+  if (batch <= single_launch_max_batch(to_dims(*dims), (flags & MSB_FLAG_SINGLE) != 0, false) &&
+      !(flags & MSB_FLAG_GENERAL)) {
     const void* xm = mapped_address(x_host);
     void* om = const_cast<void*>(mapped_address(out_host));
     if (xm && om && aligned16(xm) && aligned16(om)) {
@@ -379,7 +381,8 @@ int32_t msb_path_info(const msb_dims* dims, int32_t batch, int32_t k, uint32_t f
   const Dims D = to_dims(*dims);
   int p[6];
   fused_plan_info(D, k, batch, p);
-  const bool fused = batch <= kFusedMaxBatch && !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k);
+  const bool fused = batch <= single_launch_max_batch(D, (flags & MSB_FLAG_SINGLE) != 0, false) &&
+                     !(flags & MSB_FLAG_GENERAL) && fused_supported(D, k);
   info[0] = fused ? 1 : 2;
   for (int i = 0; i < 6; ++i) info[1 + i] = p[i];
   info[7] = 0;

@@ -9,11 +9,22 @@
 namespace msb {
 
 constexpr int MSB_ENOTFUSED = 1;  // internal: the fused path declines, use the general path
-// Batches up to this size run on the single-launch kernel, one cluster per (token,
-// routed expert) pair, each pair reading its own channels; larger ones take the
-// multi-kernel path, which reads each expert's union of channels once.  (Measured on
-// B200 with d = 2048 and 4096: the single launch is ahead up to 16 tokens, behind at 32.)
+// The single-launch kernel takes batches up to this size, one cluster per (token, routed
+// expert) pair, each pair reading its own channels; the multi-kernel path reads each
+// expert's union of channels once.
 constexpr int kFusedMaxBatch = 16;
+
+// Largest batch that runs on the single launch by default.  Its records traffic grows
+// with every (token, expert) pair while the union's saturates, so the crossover falls
+// as d grows: measured on B200, the single launch is ahead up to 12 tokens and behind
+// at 16 at d = 2048, ahead at 2 and behind from 4 at d = 4096; the limit is
+// 12 (2048 / d)^2 tokens, 1..kFusedMaxBatch.  `single` (the caller asked for the
+// single launch) and 4-bit records (the single launch only) raise it to kFusedMaxBatch.
+inline int single_launch_max_batch(const Dims& D, bool single, bool q4) {
+  if (single || q4) return kFusedMaxBatch;
+  const long long v = 12LL * 2048 * 2048 / ((long long)D.d * D.d);
+  return v < 1 ? 1 : (v > kFusedMaxBatch ? kFusedMaxBatch : (int)v);
+}
 
 bool fused_supported(const Dims& D, int k, bool q4 = false);
 // {cluster size, clusters per expert, ring slots, smem bytes, max 16-clusters, max 8-clusters}
