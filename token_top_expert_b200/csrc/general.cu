@@ -1,10 +1,17 @@
-// Multi-kernel sparse-MoE block path, any batch size 1..256.
+// Multi-kernel sparse-MoE block path, any batch size 1..256 (the default for batches past
+// the single launch's crossover), every kernel launched with programmatic stream
+// serialization:
 //
-//   router_kernel   logits, softmax, top-K, grouping of (token, expert) pairs by expert
-//   score_kernel    ternary-sketch channel scores on the tensor cores (+ z = B_e x)
+//   router_kernel   logits (each router and x row read once per CTA), softmax, top-K,
+//                   grouping of (token, expert) pairs by expert
+//   score_kernel    ternary-sketch channel scores on the tensor cores; z = B_e x on CTAs
+//                   of their own in the same grid
 //   select_kernel   exact top-k (or threshold) per pair, per-expert union bitmap
-//   gather_kernel   gathered channel records -> SwiGLU -> down, A_e z, router-weighted
-//                   reduction into an FP32 accumulator
+//   union_kernel    per-expert union lists, runs of at most 64 channels as work items
+//   gather_kernel   persistent: gathered channel records -> SwiGLU -> down on the tensor
+//                   cores, outputs held in registers over a run; then A_e z on the tensor
+//                   cores from bulk-copied rows of A_e; router-weighted reduction into an
+//                   FP32 accumulator
 //   finalize_kernel FP32 accumulator -> BF16 output (and re-zeroing)
 //
 // Each step follows the block definition of "KAIST drops calibration from MoE
