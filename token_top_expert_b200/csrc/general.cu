@@ -538,17 +538,23 @@ __global__ void __launch_bounds__(kNT) union_kernel(Dims D, Workspace ws, int ch
 // =====================================================================================
 // gathered channel records -> SwiGLU -> down; low-rank A_e z; weighted reduction
 // =====================================================================================
-// Each chunk CTA takes up to kGCh channels of one expert's union list and every token
-// routed to that expert, 8 tokens at a time, on the tensor cores:
+// Persistent CTAs (one per SM) take work items off a counter: first runs of at most
+// kGRunCh channels of one expert's union list, then low-rank row blocks.  A run streams
+// through stages of up to kGCh channels for every token routed to the expert, 8 tokens at
+// a time, on the tensor cores:
 //   gate/up   D[16 rows][8 tokens] = [gate rows | up rows] (ldmatrix from the records
-//             in shared memory) x the tokens' x rows (B fragments read through L1);
-//             warp w takes k-steps [w KS/8, (w+1) KS/8), the warps' partials meet in
-//             shared memory;
+//             in shared memory) x the tokens' x rows (B fragments in registers, or read
+//             through L1); warp w takes k-steps [w KS/8, (w+1) KS/8) over four
+//             accumulator chains, the warps' partials meet in shared memory;
 //   h         silu(g) u, times the pair's selection bit and router weight;
-//   down      D[16][8 columns] = [h_hi ; h_lo] (8 tokens x 16 channels, h split into
-//             two bf16 halves so that the product keeps ~16 significant bits) x the
-//             records' down columns (ldmatrix.trans), rows t and t+8 summed into the
-//             FP32 accumulator of token t with 8-byte reduction-adds.
+//   down      D[16 columns][8 tokens] += the records' down columns (ldmatrix.trans) x
+//             [h_hi ; h_lo]: h split into two bf16 halves laid along k against the same
+//             8 channels repeated, so that one MMA keeps ~16 significant bits of h; the
+//             run's outputs stay in registers (NACC > 0) and reach the FP32 accumulator
+//             once per run, two adjacent columns per 8-byte reduction-add.
+// Low-rank items: A_e z for a block of rows of A_e, on the tensor cores the same way
+// (z's halves along k), from rows bulk-copied into a stage buffer while the previous item
+// is computed.
 // Dynamic shared memory: records [ch][3d + 8] bf16 (16 bytes of stagger per slot).
 struct GatherCfg {
   int ch;       // channels per work item (<= kGCh)
