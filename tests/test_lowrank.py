@@ -20,6 +20,30 @@ def _expert(d, inter, seed, scale):
             rng.normal(0, scale, (d, inter)))
 
 
+def test_sketch_is_the_packers_rule():
+    """The estimate's sketch comes from the packer (msb_ternary_rows); it equals the
+    oracle's ternarisation, including entries exactly at the 0.7 mean |W| threshold
+    (strict inequality: not kept), signs, and an all-zero row (alpha 0)."""
+    rng = np.random.default_rng(9)
+    w = rng.normal(0, 0.02, (24, 80)).astype(np.float32)
+    w[3] = 0.0
+    w[5] = 1.0
+    w[5, :20] = 5.0   # mean |W| = 2, threshold 1.4: the 1.0 entries drop, the 5.0 stay
+    w[6, :40] = 13.0  # mean |W| = 10, threshold exactly 7: the 7.0 entries are not kept
+    w[6, 40:] = 7.0
+    w[7] = -w[6]
+    t, alpha = lowrank._ternary(w)
+    rt, ra = oracle.ternary_sketch(w.astype(np.float64))
+    np.testing.assert_array_equal(t, rt)
+    np.testing.assert_allclose(alpha, ra, rtol=1e-6, atol=0)
+    assert alpha[3] == 0.0 and (t[3] == 0).all()
+    assert (t[5, :20] == 1).all() and (t[5, 20:] == 0).all() and alpha[5] == 5.0
+    assert (t[6, :40] == 1).all() and (t[6, 40:] == 0).all() and alpha[6] == 13.0
+    assert (t[7, :40] == -1).all() and (t[7, 40:] == 0).all() and alpha[7] == 13.0
+    with pytest.raises(ValueError):
+        lowrank._ternary(np.zeros((0, 8), np.float32))
+
+
 def test_channel_moments_match_the_oracle_selection():
     d, inter, k = 64, 48, 12
     gate, up, down = _expert(d, inter, 1, 0.2)

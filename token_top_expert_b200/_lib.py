@@ -32,7 +32,7 @@ MSB_MAX_BATCH = 256
 
 # every function include/msb.h and include/msb_q4.h declare
 SYMBOLS = (
-    "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_workspace_size",
+    "msb_sketch_words", "msb_alpha_count", "msb_pack", "msb_ternary_rows", "msb_workspace_size",
     "msb_workspace_init", "msb_check", "msb_strerror", "moe_sparse_block",
     "moe_sparse_block_threshold", "msb_residual_rmsnorm", "msb_path_info",
     "moe_sparse_block_noalloc", "msb_noalloc_check", "moe_sparse_block_top_e",
@@ -79,6 +79,7 @@ def load() -> ctypes.CDLL:
         "msb_sketch_words": (SZ, [dims_p]),
         "msb_alpha_count": (SZ, [dims_p]),
         "msb_pack": (I32, [P, P, P, P, dims_p, P, P, P, P, I32]),
+        "msb_ternary_rows": (I32, [P, I32, I32, P, P]),
         "msb_q4_record_bytes": (SZ, [dims_p]),
         "msb_pack_q4": (I32, [P, P, P, P, dims_p, P, P, P, P, I32]),
         "msb_workspace_size": (SZ, [dims_p, I32]),

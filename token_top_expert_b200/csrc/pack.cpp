@@ -232,6 +232,17 @@ extern "C" int32_t msb_pack(const uint16_t* gate_host, const uint16_t* up_host,
   return MSB_OK;
 }
 
+extern "C" int32_t msb_ternary_rows(const float* w_host, int32_t rows, int32_t d, int8_t* t_host,
+                                    float* alpha_host) {
+  if (!w_host || !t_host || !alpha_host || rows < 1 || d < 1) return MSB_EINVAL;
+  std::vector<double> w((size_t)d);
+  for (int j = 0; j < rows; ++j) {
+    for (int i = 0; i < d; ++i) w[i] = w_host[(size_t)j * d + i];
+    alpha_host[j] = ternary_row(w.data(), d, t_host + (size_t)j * d);
+  }
+  return MSB_OK;
+}
+
 extern "C" size_t msb_q4_record_bytes(const msb_dims* dims) {
   if (!dims || dims->d < 64 || dims->d % 64 != 0 || dims->d > MSB_MAX_D) return 0;
   return q4_record_bytes(dims->d);

@@ -27,13 +27,18 @@ prior the SwiGLU output is close to a quadratic form in x, whose best linear pre
 small: on the Qwen3-30B-A3B-shaped synthetic block the map removes 1.4-2 % of the sparse
 block's error against the dense one.
 
-The selection inside the estimate follows the block's own rule: ternary sketch of the gate
-rows (threshold 0.7 * mean |W|, scale = mean |W| of the kept entries), scores
-alpha_j * |T_j . x|, the k highest kept (ties to the lower index).
+The selection inside the estimate follows the block's own rule: the ternary sketch of the
+gate rows comes from the packer (msb_ternary_rows: threshold 0.7 * mean |W|, scale = mean
+|W| of the kept entries), the scores are alpha_j * |T_j . x| and the k highest are kept
+(ties to the lower index) over the Monte Carlo samples.
 """
 from __future__ import annotations
 
+import ctypes
+
 import numpy as np
+
+from . import _lib
 
 
 def _f32(a) -> np.ndarray:
@@ -52,14 +57,19 @@ def _bf16_bits(x: np.ndarray) -> np.ndarray:
 
 
 def _ternary(gate: np.ndarray):
-    """Per-row ternary sketch of gate [I][d]: T in {-1, 0, 1}, alpha [I]."""
-    a = np.abs(gate.astype(np.float64))
-    d = gate.shape[1]
-    keep = 10.0 * d * a > 7.0 * a.sum(axis=1, keepdims=True)  # |W| > 0.7 mean |W|, exactly
-    t = np.where(keep, np.sign(gate), 0.0).astype(np.float32)
-    n = keep.sum(axis=1)
-    alpha = np.where(n > 0, (a * keep).sum(axis=1) / np.maximum(n, 1), 0.0).astype(np.float32)
-    return t, alpha
+    """Per-row ternary sketch of gate [I][d] (float32): T in {-1, 0, 1} (as float32) and
+    alpha [I], computed by the packer itself (msb_ternary_rows), so the selection inside
+    the estimate is the one the block's sketch makes."""
+    w = np.ascontiguousarray(gate, dtype=np.float32)
+    rows, d = w.shape
+    t = np.empty((rows, d), np.int8)
+    alpha = np.empty(rows, np.float32)
+    rc = _lib.load().msb_ternary_rows(w.ctypes.data_as(ctypes.c_void_p), rows, d,
+                                      t.ctypes.data_as(ctypes.c_void_p),
+                                      alpha.ctypes.data_as(ctypes.c_void_p))
+    if rc != 0:
+        raise ValueError("msb_ternary_rows: status %d" % rc)
+    return t.astype(np.float32), alpha
 
 
 def channel_moments(gate, up, down, k: int, x: np.ndarray, sketch=None):
