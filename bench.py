@@ -534,6 +534,9 @@ def main():
     ap.add_argument("--replicas", type=int, default=8,
                     help="weight copies rotated per step so that every step reads HBM")
     ap.add_argument("--general", action="store_true", help="force the multi-kernel path")
+    ap.add_argument("--single", action="store_true",
+                    help="ask for the single-launch kernel (batches up to 16 tokens), even past "
+                         "the measured crossover where the multi-kernel path is the default")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU-oracle timing")
     ap.add_argument("--e2e-steps", type=int, default=2000,
                     help="steps of the end-to-end measurement (host copies in the timed region)")
@@ -606,11 +609,12 @@ def main():
     outs = torch.empty_like(xs)
     ws = msb.Workspace(dims, B, dev)
     stream = torch.cuda.Stream(dev)
-    general = args.general
+    general, single = args.general, args.single
 
     def step(i, s):
         msb.moe_sparse_block(xs[i % nseq], layers[i % args.replicas], args.k, out=outs[i % nseq],
-                             workspace=ws, general=general, stream=s, top_e=args.top_e)
+                             workspace=ws, general=general, stream=s, top_e=args.top_e,
+                             single=single)
 
     # ---- union sizes of every step of the sequence (one traced pass) -> algorithmic bytes
     dense = args.k == w.inter
@@ -695,7 +699,8 @@ def main():
         # the host produces each step's x before the call (nothing on the stream writes
         # it), so the calls declare it ready: the kernel fetches x across the host link
         # while the previous launch still runs
-        calls = [msb.HostCall(lay, args.k, B, stream=stream, general=general, x_ready=True) for lay in layers]
+        calls = [msb.HostCall(lay, args.k, B, stream=stream, general=general, x_ready=True, single=single)
+                 for lay in layers]
         xp = [xh[i].data_ptr() for i in range(nseq)]
         op = [oh[i].data_ptr() for i in range(nseq)]
 
@@ -708,7 +713,7 @@ def main():
         def e2e_step(i):
             xd.copy_(xh[i % nseq], non_blocking=True)
             msb.moe_sparse_block(xd, layers[i % args.replicas], args.k, out=od, workspace=ws,
-                                 general=general, stream=stream, top_e=args.top_e)
+                                 general=general, stream=stream, top_e=args.top_e, single=single)
             oh[i % nseq].copy_(od, non_blocking=True)
     with torch.cuda.stream(stream):
         for i in range(min(50, ne)):
@@ -732,7 +737,7 @@ def main():
     peak, peak_kind = peaks()
     achieved = step_bytes / (ms_per_step * 1e-3) / 1e9
     plan = msb.path_info(msb.Dims(w.d, w.inter, w.experts, args.top_e or w.top_e, args.rank, 1), B,
-                         args.k, general=general, single=bool(args.q4))  # 4-bit: single launch only
+                         args.k, general=general, single=bool(args.q4) or single)  # 4-bit: single only
     kernel = "fused_block_kernel" if plan["path"] == "single_launch" else "multi_kernel_step"
     traffic = recorded_traffic(kernel, w.name + ("_dense" if dense else "") + ("_q4" if args.q4 else ""))
     launches_per_step = block_launches(plan["path"], dense, args.rank)

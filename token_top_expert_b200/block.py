@@ -382,10 +382,11 @@ class HostCall:
 
     x_ready=True declares that nothing earlier on the stream writes x_host (the host
     produced it before the call), so that the single-launch kernel fetches it while the
-    previous launch still runs (MSB_FLAG_X_READY)."""
+    previous launch still runs (MSB_FLAG_X_READY).  general / single: as for
+    moe_sparse_block."""
 
     def __init__(self, layer: PackedLayer, k: int, batch: int, stream=None, general: bool = False,
-                 x_ready: bool = False):
+                 x_ready: bool = False, single: bool = False):
         if layer.q4:
             raise ValueError("4-bit records: use moe_sparse_block")
         import torch
@@ -404,7 +405,8 @@ class HostCall:
         self._head = (_ptr(self.x_dev), batch, _ptr(layer.router_t), _ptr(layer.records),
                       _ptr(layer.sketch), _ptr(layer.alpha), k, _ptr(layer.lr_a), _ptr(layer.lr_b),
                       _ptr(self.out_dev))
-        flags = (_lib.MSB_FLAG_GENERAL if general else 0) | (_lib.MSB_FLAG_X_READY if x_ready else 0)
+        flags = ((_lib.MSB_FLAG_GENERAL if general else 0) | (_lib.MSB_FLAG_X_READY if x_ready else 0)
+                 | (_lib.MSB_FLAG_SINGLE if single else 0))
         self._tail = (ctypes.byref(self._dims), self.workspace.ptr, self.workspace.nbytes, flags,
                       _stream(self.stream))
         self._layer = layer  # keep the weights alive
