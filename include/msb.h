@@ -146,15 +146,6 @@ int32_t msb_pack(const uint16_t* gate_host, const uint16_t* up_host, const uint1
                  uint32_t* sketch_host, float* alpha_host, uint16_t* router_t_host,
                  int32_t threads);
 
-/* The packer's ternarisation on its own, for host-side weight preparation (the
- * weight-derived compensation factors select channels with the block's own sketch):
- * rows of length d, float32, row-major in w_host [rows][d]; T (-1, 0 or 1) into
- * t_host [rows][d] and alpha into alpha_host [rows], by the rule msb_pack applies to
- * each W_gate row.  Host memory only (no CUDA).  Returns MSB_OK, or MSB_EINVAL for a
- * null pointer, rows < 1 or d < 1. */
-int32_t msb_ternary_rows(const float* w_host, int32_t rows, int32_t d, int8_t* t_host,
-                         float* alpha_host);
-
 /* ------------------------------------------------------------------ workspace
  * Bytes of device workspace a call with up to max_batch tokens needs (0 for
  * invalid dims or max_batch outside 1..MSB_MAX_BATCH).  The

@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include "msb.h"
+#include "msb_prep.h"
 #include "msb_q4.h"
 
 #define CHECK(cond)                                                  \
@@ -86,6 +87,16 @@ int main(void) {
 
   free(gate); free(up); free(down); free(router); free(rec); free(rec4);
   free(sketch); free(alpha); free(router_t);
+  {  /* the packer's ternarisation on its own: |w| > 0.7 mean|w| keeps 1 and -1 (2 and -2) */
+    const float w[8] = {1.0f, -1.0f, 0.1f, 0.0f, 2.0f, -2.0f, 0.2f, 0.0f};
+    int8_t t[8];
+    float a[2];
+    CHECK(msb_ternary_rows(w, 2, 4, t, a) == MSB_OK);
+    CHECK(t[0] == 1 && t[1] == -1 && t[2] == 0 && t[3] == 0 && a[0] == 1.0f);
+    CHECK(t[4] == 1 && t[5] == -1 && t[6] == 0 && t[7] == 0 && a[1] == 2.0f);
+    CHECK(msb_ternary_rows(NULL, 2, 4, t, a) == MSB_EINVAL);
+    CHECK(msb_ternary_rows(w, 0, 4, t, a) == MSB_EINVAL);
+  }
   printf("c abi ok\n");
   return 0;
 }

@@ -21,6 +21,7 @@
 #include <vector>
 
 #include "msb.h"
+#include "msb_prep.h"
 #include "msb_q4.h"
 
 namespace {
